@@ -1,0 +1,422 @@
+"""Benchmark of the H-Spec block-parallel draft step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl hspec|reference]
+                    [--C 128] [--K 16] [--sweep] [--no-cpu-baseline]
+
+One step = one hspec_draft_step over a batch of C requests of the 4-layer M,A,M,A
+drafter on Llama-3-8B shapes (SwiGLU 16384, shared 128256-token LM head), K block
+positions each, context lengths uniform in [512, 16384], every attention layer
+reading its own paged target KV cache in place.  Metric: drafted tokens/s
+(C*K per step), with the step time in microseconds.  Inputs (~20 GB of weights
+and KV) exceed the 126 MB L2, so no flush is needed between steps.
+
+Multi-GPU: requests are independent, so each rank runs its own batch of C
+requests (weak scaling, replicas only, no collective on the data path); the step
+time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "drafted tokens/s (draft step, C*K tokens per step)"
+UNIT = "tokens/s"
+
+
+# --------------------------------------------------------------------- helpers
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+    FIELDS = ["index", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+            target = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={','.join(self.FIELDS)}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", target], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- algorithmic work
+
+def step_work(sh, C, K, ctx_lens):
+    """Algorithmic bytes and flops of each kernel group for one launch."""
+    d, H, P, N = sh.d, sh.H, sh.P, sh.N
+    HP, HPN = H * P, H * P * N
+    n_in = 2 * HP + 2 * N + H
+    n_qkv = (sh.Hq + 2 * sh.Hkv) * sh.D
+    M = C * K
+    E = 2 if sh.dtype == "bf16" else 4
+    ctx_sum = int(ctx_lens.sum())
+    kv_bytes = ctx_sum * sh.Hkv * sh.D * 2 * E
+    w = {}
+
+    def gemm(name, m, n, k, extra_bytes=0):
+        w[name] = {"flops": 2.0 * m * n * k, "bytes": float(n * k * E + m * k * E + extra_bytes)}
+
+    gemm("in_proj", M, n_in, d, M * n_in * E)
+    gemm("inject", C, HPN, d, C * HPN * 4)
+    gemm("out_proj", M, d, HP, M * d * 8)
+    gemm("qkv_proj", M, n_qkv, d, M * n_qkv * E)
+    gemm("o_proj", M, d, sh.Hq * sh.D, M * d * 8)
+    if sh.d_ff:
+        gemm("mlp_gate_up", M, 2 * sh.d_ff, d, M * sh.d_ff * E)
+        gemm("mlp_down", M, d, sh.d_ff, M * d * 8)
+    if sh.vocab:
+        gemm("lm_head_argmax", M, sh.vocab, d)
+    w["attn_paged"] = {"flops": 4.0 * sh.Hq * sh.D * K * (ctx_sum + C * K),
+                       "bytes": float(kv_bytes + 2 * M * sh.Hq * sh.D * E + 2 * M * sh.Hkv * sh.D * E)}
+    w["ssd_scan"] = {"flops": float(C * H * (2 * K * P * N + K * K * (N + P))),
+                     "bytes": float(C * HPN * 4 + M * (HP + 2 * N + H) * E + M * HP * 4)}
+    return w
+
+
+def roofline_of(name, work, avg_ms, peaks, traffic=None, sustained=True):
+    """hbm- or tensor-bound roofline fraction of one kernel group."""
+    fl, by = work["flops"], work["bytes"]
+    tf_peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+    t_tensor = fl / (tf_peak * 1e12)
+    t_hbm = by / (peaks["hbm_gbs"] * 1e9)
+    sec = avg_ms / 1e3
+    if name in ("attn_paged", "ssd_scan") or t_hbm >= t_tensor:
+        ach = by / sec / 1e9
+        return {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(ach / peaks["hbm_gbs"], 4), "traffic": traffic}
+    ach = fl / sec / 1e12
+    return {"bound": "tensor", "achieved": round(ach, 1), "peak": tf_peak, "unit": "TFLOP/s",
+            "frac": round(ach / tf_peak, 4), "traffic": traffic}
+
+
+# ---------------------------------------------------------------------- our arm
+
+class StepRunner:
+    def __init__(self, H, I, wl, device, weights=None):
+        self.H, self.wl, self.sh = H, wl, wl.shapes
+        self.st = I.make_step_inputs(wl, device, weights=weights is None)
+        if weights is not None:
+            self.st["weights"] = weights
+        C, K, sh = wl.C, wl.K, self.sh
+        self.dr = H.Drafter(sh, self.st["weights"])
+        self.max_pages = max(c["page_table"].shape[1] for c in self.st["kv"])
+        self.ws = H.alloc_workspace(self.dr.workspace_size(C, K, self.max_pages), device)
+        self.tokens_out = torch.empty(C, K, dtype=torch.int32, device=device)
+        self.si = self.dr.step_in(C, K, self.st["h_last"], self.st["ctx_lens"], self.st["kv"],
+                                  tokens=self.st["tokens"], x_in=self.st["x_in"])
+        self.so = H.hspec_step_out(draft_tokens=self.tokens_out.data_ptr())
+
+    def step(self):
+        self.dr.step(self.si, self.so, self.ws)
+
+    def check(self):
+        s = self.H.hspec_sync_status()
+        if s != 0:
+            raise RuntimeError(f"draft step failed: {self.H.hspec_status_string(s)} ({self.H.hspec_last_error()})")
+
+    def close(self):
+        self.dr.close()
+
+
+def time_steps(runner, steps, warmup, world, profile=False):
+    H = runner.H
+    for _ in range(warmup):
+        runner.step()
+    runner.check()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if profile:
+        H.hspec_profile_enable(True)
+    n0 = H.hspec_launch_count()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(steps):
+        runner.step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    launches = H.hspec_launch_count() - n0
+    prof = H.hspec_profile_read() if profile else {}
+    if profile:
+        H.hspec_profile_enable(False)
+    runner.check()
+    return e0.elapsed_time(e1) / steps, launches, prof
+
+
+def time_e2e(runner, steps):
+    """Same step through the C-ABI with host inputs: every step copies h_last, block
+    tokens, ctx_lens and the page tables from pinned host memory and reads the
+    draft tokens back."""
+    st = runner.st
+    dev_in = [st["h_last"], st["tokens"], st["ctx_lens"]] + [c["page_table"] for c in st["kv"]]
+    host_in = [t.to("cpu").pin_memory() for t in dev_in]
+    host_out = torch.empty(runner.tokens_out.shape, dtype=torch.int32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = host_out.numel() * host_out.element_size()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    e0.record(stream)
+    for _ in range(steps):
+        for d, h in zip(dev_in, host_in):
+            d.copy_(h, non_blocking=True)
+        runner.step()
+        host_out.copy_(runner.tokens_out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    wall = (time.perf_counter() - t0) / steps
+    runner.check()
+    return e0.elapsed_time(e1) / steps, wall * 1e3, h2d, d2h
+
+
+def oracle_one_request(I, wl, runner=None, device="cpu", request=0):
+    """Times the CPU oracle on one request of the workload (requests are
+    independent, so C requests cost C times this)."""
+    import oracle
+    st = runner.st if runner is not None else I.make_step_inputs(wl, device)
+    w = oracle.host_weights(st["weights"])
+    rows = [request]
+    kv = [oracle.host_sub_cache(c, rows) for c in st["kv"]]
+    args = dict(tokens=st["tokens"].cpu()[rows] if st["tokens"] is not None else None,
+                x_in=st["x_in"].cpu()[rows] if st["x_in"] is not None else None)
+    h_last, lens = st["h_last"].cpu()[rows], st["ctx_lens"].cpu()[rows]
+    t0 = time.perf_counter()
+    oracle.draft_step(wl.shapes, w, kv, h_last, lens, **args)
+    return time.perf_counter() - t0, int(lens[0]), oracle.threads()
+
+
+def run_ours(args, rank, world, local):
+    from hybrid_mamba_attention_b200 import hspec as H
+    from hybrid_mamba_attention_b200 import inputs as I
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    wl = I.full_workload(args.C, args.K)
+    wl = I.Workload(wl.name, wl.shapes, wl.C, wl.K, wl.ctx_lo, wl.ctx_hi, seed=wl.seed + 1000 * rank)
+    runner = StepRunner(H, I, wl, dev)
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    ms, launches, prof = time_steps(runner, args.steps, args.warmup, world, profile=True)
+    clk = clocks.stop()
+    ms_max = max_over_ranks(ms, world)
+    tokens = wl.C * wl.K * world
+    value = tokens / (ms_max / 1e3)
+
+    # roofline: per kernel group, from the events recorded on the step's stream
+    work = step_work(wl.shapes, wl.C, wl.K, runner.st["ctx_lens"].cpu())
+    kernels = {}
+    for name, (tot, cnt) in prof.items():
+        avg = tot / max(cnt, 1)
+        ent = {"avg_ms": round(avg, 4), "launches_per_step": cnt / args.steps,
+               "share": round(tot / (ms * args.steps), 4)}
+        if name in work:
+            ent["roofline"] = roofline_of(name, work[name], avg, peaks)
+        kernels[name] = ent
+    dominant = max(kernels, key=lambda k: kernels[k]["share"]) if kernels else None
+    roof = dict(kernels[dominant]["roofline"]) if dominant and "roofline" in kernels[dominant] else None
+    if roof:
+        roof["kernel"] = dominant
+        roof["peak_source"] = f"{peaks['source']} (MEASURED_PEAKS.json)" if peaks["source"] == "measured" else "fallback"
+    attn_roof = kernels.get("attn_paged", {}).get("roofline")
+
+    e2e_ms, e2e_wall_ms, h2d, d2h = time_e2e(runner, args.steps)
+    e2e_ms = max_over_ranks(e2e_ms, world)
+    e2e = {"value": round(tokens / (e2e_ms / 1e3), 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4), "wall_ms_per_step": round(e2e_wall_ms, 4)}
+
+    sweep = None
+    if args.sweep:
+        sweep = []
+        for K in I.FULL_SWEEP_K:
+            for C in I.FULL_SWEEP_C:
+                w2 = I.full_workload(C, K)
+                r2 = StepRunner(H, I, w2, dev, weights=runner.st["weights"])
+                m2, _, _ = time_steps(r2, max(3, args.steps // 2), 2, 1)
+                sweep.append({"C": C, "K": K, "us_per_step": round(m2 * 1e3, 1),
+                              "tokens_per_s": round(C * K / (m2 / 1e3), 1)})
+                r2.close()
+                del r2
+                torch.cuda.empty_cache()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        secs, ctx, cores = oracle_one_request(I, wl, runner)
+        cpu = {"value": round(wl.K / secs, 3), "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"1 of {wl.C} requests (ctx {ctx}, K={wl.K}) through the full M,A,M,A step "
+                         f"+ LM head; {secs:.2f} s; requests are independent so C requests take C times as long"}
+
+    runner.close()
+    if rank == 0:
+        line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": round(ms_max, 4), "us_per_step": round(ms_max * 1e3, 1),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic (seeded random-init weights and KV of the stated shapes)",
+                "config": {"workload": f"full draft step {wl.name}: 4-layer M,A,M,A hybrid drafter, Llama-3-8B "
+                                       f"shapes, SwiGLU 16384, vocab 128256, ctx U[512,16384], 16-token pages",
+                           "C": wl.C, "K": wl.K, "global_batch": wl.C * world, "parallelism": f"replicas x{world}",
+                           "l2": "inputs ~20 GB > 126 MB L2 (no flush needed)"},
+                "roofline": roof, "attention_roofline": attn_roof, "kernels": kernels,
+                "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clk}
+        if sweep is not None:
+            line["sweep"] = sweep
+        print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- reference arm
+
+def run_reference(args, rank, world):
+    """The CPU oracle as the reference arm, on this arm's config and metric."""
+    if rank != 0:
+        return
+    from hybrid_mamba_attention_b200 import inputs as I
+    wl = I.full_workload(args.C, args.K)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    st = I.make_step_inputs(wl, dev)
+
+    class _R:
+        pass
+
+    r = _R()
+    r.st = st
+    import oracle  # noqa: F401
+    for i in range(args.warmup):
+        oracle_one_request(I, wl, r, request=i % wl.C)
+    times = []
+    for i in range(args.steps):
+        secs, ctx, cores = oracle_one_request(I, wl, r, request=i % wl.C)
+        times.append(secs)
+    sec = sum(times) / len(times)
+    value = wl.K / sec
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(sec * 1e3, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded random-init weights and KV of the stated shapes)",
+            "config": {"workload": f"full draft step {wl.name} (CPU oracle, one request per step)", "C": wl.C,
+                       "K": wl.K},
+            "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+                             "sample": f"one request of the {wl.C}-request batch per step"},
+            "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["hspec", "reference"], default="hspec")
+    ap.add_argument("--C", type=int, default=128)
+    ap.add_argument("--K", type=int, default=16)
+    ap.add_argument("--sweep", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_ours(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

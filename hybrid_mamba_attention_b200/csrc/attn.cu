@@ -1,0 +1,236 @@
+// Paged in-place GQA attention of the K block queries over the target's KV cache
+// followed by the block's own keys (H-Spec Abstract: "attention modules reuse target
+// KVs in place"), split-KV across CTAs, then a merge of the partial softmax states.
+//
+// attn_split_kernel: one CTA per (split, kv head g, request c).  Its R = K*G query
+// rows (block position j, query head g*G + i) share every key/value of kv head g,
+// so each 16-token tile of K and V is read from HBM once per CTA, translated through
+// the page table in place (token t of request c: page page_table[c][t / page],
+// slot t % page), staged in shared memory as fp32 and used by all R rows.  Threads
+// form groups of TPR lanes per row; a lane holds D/TPR interleaved dims of q and of
+// the running output, dot products are reduced across the group with shuffles, and
+// the softmax runs online in the exp2 domain.  The CTA writes its partial
+// (m, l, unnormalised acc) per row.
+//
+// attn_merge_kernel: one warp per output row (c, j, h) combines the splits of that
+// request: o = sum_s 2^(m_s - M) acc_s / sum_s 2^(m_s - M) l_s.
+#include "../../include/hspec.h"
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace hspec {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kTile = 16;
+
+template <typename T, int TPR>
+__global__ void __launch_bounds__(kThreads) attn_split_kernel(AttnArgs a, float scale_log2) {
+  constexpr int ROWS = kThreads / TPR;      // query rows one CTA can hold
+  extern __shared__ float sm[];
+  const int D = a.D, Dp = D + 1;
+  float* sK = sm;                           // [kTile][D+1]
+  float* sV = sK + kTile * Dp;              // [kTile][D+1]
+  const int split = blockIdx.x, g = blockIdx.y, c = blockIdx.z;
+  const int G = a.Hq / a.Hkv, R = a.K * G;
+  const int ctx = a.ctx_lens[c];
+  if (ctx < 0 || ctx > a.max_pages * a.page_size) {
+    if (threadIdx.x == 0 && split == 0) flag_error(a.err, kErrCtxOOB);
+    return;
+  }
+  const int T_total = ctx + a.K;
+  const int t_begin = split * a.split_tokens;
+  if (t_begin >= T_total) return;  // the merge reads only the splits that hold tokens
+  const int t_end = min(T_total, t_begin + a.split_tokens);
+
+  const int row = threadIdx.x / TPR, gl = threadIdx.x % TPR;
+  const bool active = row < R;
+  const int j = active ? row / G : 0;
+  const int h = g * G + (active ? row % G : 0);
+  constexpr int DPT_MAX = 128 / TPR > 0 ? 128 / TPR : 1;
+  const int dpt = D / TPR;
+  float qv[DPT_MAX], acc[DPT_MAX];
+  const T* q = (const T*)a.q + (size_t)(c * a.K + j) * a.q_rs + (size_t)h * D;
+#pragma unroll
+  for (int i = 0; i < DPT_MAX; ++i) {
+    qv[i] = (active && i < dpt) ? to_f(q[gl + i * TPR]) * scale_log2 : 0.f;
+    acc[i] = 0.f;
+  }
+  float m_run = -INFINITY, l_run = 0.f;
+
+  const T* kp = (const T*)a.k_pool;
+  const T* vp = (const T*)a.v_pool;
+  const T* kb = (const T*)a.kb;
+  const T* vb = (const T*)a.vb;
+  const int32_t* table = a.page_table + (size_t)c * a.max_pages;
+
+  for (int t0 = t_begin; t0 < t_end; t0 += kTile) {
+    __syncthreads();
+    for (int i = threadIdx.x; i < kTile * D; i += kThreads) {
+      const int tt = i / D, e = i % D, t = t0 + tt;
+      float kvk = 0.f, kvv = 0.f;
+      if (t < ctx) {
+        const int pg = table[t / a.page_size];
+        if (pg >= 0 && pg < a.num_pages) {
+          const size_t off = (((size_t)pg * a.page_size + t % a.page_size) * a.Hkv + g) * D + e;
+          kvk = to_f(kp[off]);
+          kvv = to_f(vp[off]);
+        } else if (e == 0) {
+          flag_error(a.err, kErrPageOOB);
+        }
+      } else if (t < t_end) {
+        const size_t off = (size_t)(c * a.K + (t - ctx)) * a.kb_rs + (size_t)g * D + e;
+        kvk = to_f(kb[off]);
+        kvv = to_f(vb[(size_t)(c * a.K + (t - ctx)) * a.vb_rs + (size_t)g * D + e]);
+      }
+      sK[tt * Dp + e] = kvk;
+      sV[tt * Dp + e] = kvv;
+    }
+    __syncthreads();
+    // rows beyond R compute on q = 0 and are never written: every lane of a warp
+    // must take part in the group shuffles below.
+    float s[kTile];
+    float tile_max = -INFINITY;
+#pragma unroll
+    for (int tt = 0; tt < kTile; ++tt) {
+      float part = 0.f;
+#pragma unroll
+      for (int i = 0; i < DPT_MAX; ++i)
+        if (i < dpt) part = fmaf(qv[i], sK[tt * Dp + gl + i * TPR], part);
+#pragma unroll
+      for (int o = TPR / 2; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+      const int t = t0 + tt;
+      bool vis = t < t_end;
+      if (a.causal_block && t >= ctx && (t - ctx) > j) vis = false;
+      s[tt] = vis ? part : -INFINITY;
+      tile_max = fmaxf(tile_max, s[tt]);
+    }
+    const float m_new = fmaxf(m_run, tile_max);
+    if (m_new == -INFINITY) continue;  // nothing visible yet
+    const float alpha = exp2f(m_run - m_new);
+    float psum = 0.f;
+#pragma unroll
+    for (int tt = 0; tt < kTile; ++tt) {
+      s[tt] = exp2f(s[tt] - m_new);
+      psum += s[tt];
+    }
+    l_run = l_run * alpha + psum;
+    m_run = m_new;
+#pragma unroll
+    for (int i = 0; i < DPT_MAX; ++i) {
+      if (i >= dpt) break;
+      float v = acc[i] * alpha;
+#pragma unroll
+      for (int tt = 0; tt < kTile; ++tt) v = fmaf(s[tt], sV[tt * Dp + gl + i * TPR], v);
+      acc[i] = v;
+    }
+  }
+  if (!active) return;
+  const size_t base = ((((size_t)c * a.Hkv + g) * a.n_splits + split) * R + row);
+  float* pacc = a.ws_acc + base * D;
+#pragma unroll
+  for (int i = 0; i < DPT_MAX; ++i)
+    if (i < dpt) pacc[gl + i * TPR] = acc[i];
+  if (gl == 0) {
+    a.ws_ml[base * 2] = m_run;
+    a.ws_ml[base * 2 + 1] = l_run;
+  }
+}
+
+template <typename T>
+__global__ void attn_merge_kernel(AttnArgs a) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  const int G = a.Hq / a.Hkv, R = a.K * G;
+  const long rows = (long)a.C * a.K * a.Hq;
+  if (warp >= rows) return;
+  const int h = warp % a.Hq;
+  const int j = (warp / a.Hq) % a.K;
+  const int c = warp / (a.Hq * a.K);
+  const int g = h / G, row = j * G + h % G;
+  const int ctx = a.ctx_lens[c];
+  T* out = (T*)a.out + (size_t)(c * a.K + j) * a.o_rs + (size_t)h * a.D;
+  if (ctx < 0 || ctx > a.max_pages * a.page_size) {
+    for (int e = lane; e < a.D; e += 32) out[e] = from_f<T>(0.f);
+    return;
+  }
+  const int ns = (ctx + a.K + a.split_tokens - 1) / a.split_tokens;
+  const size_t base0 = (((size_t)c * a.Hkv + g) * a.n_splits) * R + row;
+  float M = -INFINITY;
+  for (int s = 0; s < ns; ++s) M = fmaxf(M, a.ws_ml[(base0 + (size_t)s * R) * 2]);
+  float L = 0.f;
+  for (int s = 0; s < ns; ++s) {
+    const float ms = a.ws_ml[(base0 + (size_t)s * R) * 2];
+    if (ms != -INFINITY) L += exp2f(ms - M) * a.ws_ml[(base0 + (size_t)s * R) * 2 + 1];
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  for (int e = lane; e < a.D; e += 32) {
+    float o = 0.f;
+    for (int s = 0; s < ns; ++s) {
+      const float ms = a.ws_ml[(base0 + (size_t)s * R) * 2];
+      if (ms != -INFINITY) o = fmaf(exp2f(ms - M), a.ws_acc[(base0 + (size_t)s * R) * a.D + e], o);
+    }
+    out[e] = from_f<T>(o * inv);
+  }
+}
+
+template <typename T, int TPR>
+void launch_split(const AttnArgs& a, cudaStream_t s) {
+  const size_t smem = (size_t)2 * kTile * (a.D + 1) * sizeof(float);
+  const float scale_log2 = 1.4426950408889634f / sqrtf((float)a.D);
+  attn_split_kernel<T, TPR><<<dim3(a.n_splits, a.Hkv, a.C), kThreads, smem, s>>>(a, scale_log2);
+  note_launch();
+}
+
+template <typename T>
+void launch_all(const AttnArgs& a, cudaStream_t s) {
+  const int R = a.K * (a.Hq / a.Hkv);
+  int rows_cap = 1;
+  while (rows_cap < R) rows_cap <<= 1;
+  const int tpr = kThreads / rows_cap;  // lanes per query row (power of two, 1..32)
+  switch (tpr >= 32 ? 32 : tpr) {
+    case 32: launch_split<T, 32>(a, s); break;
+    case 16: launch_split<T, 16>(a, s); break;
+    case 8: launch_split<T, 8>(a, s); break;
+    case 4: launch_split<T, 4>(a, s); break;
+    case 2: launch_split<T, 2>(a, s); break;
+    default: launch_split<T, 1>(a, s); break;
+  }
+  const long rows = (long)a.C * a.K * a.Hq;
+  attn_merge_kernel<T><<<(int)((rows + 7) / 8), 256, 0, s>>>(a);
+  note_launch();
+}
+
+}  // namespace
+
+bool attn_supported(int K, int G, int D) {
+  // one CTA holds all R = K*G query rows; a lane holds at most 128/TPR dims of q and acc
+  const int R = K * G;
+  int cap = 1;
+  while (cap < R) cap <<= 1;
+  if (cap > kThreads || D > 128 || D % 2) return false;
+  int tpr = kThreads / cap;
+  if (tpr > 32) tpr = 32;
+  return D % tpr == 0;
+}
+
+int attn_split_tokens(int C, int Hkv, int K, int max_ctx, int requested) {
+  if (requested > 0) return requested;
+  // aim for ~16 CTAs per SM over the whole grid, in multiples of 64 tokens
+  const long target_ctas = 148L * 16;
+  long per = ((long)C * Hkv * (max_ctx + K) + target_ctas - 1) / target_ctas;
+  per = ((per + 63) / 64) * 64;
+  if (per < 64) per = 64;
+  return (int)per;
+}
+
+size_t attn_ws_bytes(int C, int Hkv, int K, int G, int D, int n_splits) {
+  const size_t rows = (size_t)C * Hkv * n_splits * K * G;
+  return rows * D * sizeof(float) + rows * 2 * sizeof(float);
+}
+
+void attn_paged(int dtype, const AttnArgs& a, cudaStream_t s) {
+  if (dtype == HSPEC_DTYPE_BF16) launch_all<bf16>(a, s);
+  else launch_all<float>(a, s);
+}
+
+}  // namespace hspec

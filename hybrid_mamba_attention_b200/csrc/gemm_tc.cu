@@ -1,0 +1,281 @@
+// bf16 GEMM on the 5th-generation tensor cores: out = epi(A . B^T), A [M,K] and
+// B [N,K] row-major (K-major) bf16, fp32 accumulation in tensor memory.
+//
+// One CTA computes a 128 x 256 output tile (SwiGLU: 128 x 128 outputs from a
+// 128 x (128 gate + 128 up) accumulator) with three roles:
+//   warp 0      TMA producer: streams 128x64 A and 256x64 B tiles (128-byte
+//               swizzle) through a 4-stage shared-memory ring of mbarriers;
+//   warp 1      allocates 256 TMEM columns; one lane issues tcgen05.mma
+//               (M=128, N=256, K=16, four per 64-wide stage) and commits each
+//               stage back to the producer, then the finished accumulator;
+//   warps 2..5  epilogue: tcgen05.ld of their 32-lane quarter of TMEM, then the
+//               fused epilogue (store, residual add, SwiGLU, per-row argmax).
+// Rows/columns beyond M/N are zero-filled by TMA and skipped by the epilogue.
+// Grids run M-tiles fastest so that the CTAs sharing one weight tile are resident
+// together and the weight is read from HBM once.
+#include <mutex>
+#include <stdint.h>
+
+#include "../../include/hspec.h"
+#include "common.cuh"
+#include "kernels.cuh"
+#include "tc_prims.cuh"
+
+namespace hspec {
+
+void gemm_simt_f32(GemmEpi epi, const GemmArgs& g, cudaStream_t s);
+
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2, B_BYTES = BN * BK * 2, STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int THREADS = 192;
+constexpr uint32_t TMEM_COLS = 256;
+
+template <int EPI>
+__global__ void __launch_bounds__(THREADS, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmB2, GemmArgs g, int* err) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = tc::smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw + 1023) & ~1023u) - raw);
+  uint64_t* full = (uint64_t*)(smem + STAGES * STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* acc_full = empty + STAGES;
+  uint32_t* tmem_slot = (uint32_t*)(acc_full + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * BM;
+  const int ncols_out = (EPI == kEpiSwiGLU) ? BN / 2 : BN;
+  const int n0 = blockIdx.y * ncols_out;
+  const int num_k = (g.K + BK - 1) / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 1);
+    }
+    tc::mbar_init(acc_full, 1);
+    tc::fence_mbar_init();
+  }
+  if (warp == 1) tc::tmem_alloc(tmem_slot, TMEM_COLS);
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------------------------------------------------- TMA producer
+    tc::tma_prefetch_desc(&tmA);
+    tc::tma_prefetch_desc(&tmB);
+    if (EPI == kEpiSwiGLU) tc::tma_prefetch_desc(&tmB2);
+    for (int kt = 0; kt < num_k; ++kt) {
+      const int s = kt % STAGES;
+      const uint32_t ph = (kt / STAGES) & 1;
+      if (!tc::mbar_wait(&empty[s], ph ^ 1, err)) break;
+      uint8_t* sa = smem + s * STAGE_BYTES;
+      uint8_t* sb = sa + A_BYTES;
+      tc::mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
+      tc::tma_load_2d(sa, &tmA, &full[s], kt * BK, m0);
+      if (EPI == kEpiSwiGLU) {
+        tc::tma_load_2d(sb, &tmB, &full[s], kt * BK, n0);
+        tc::tma_load_2d(sb + B_BYTES / 2, &tmB2, &full[s], kt * BK, n0);
+      } else {
+        tc::tma_load_2d(sb, &tmB, &full[s], kt * BK, n0);
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------------------------------------------------- MMA issuer
+    constexpr uint32_t idesc = tc::idesc_bf16_f32(BM, BN);
+    bool ok = true;
+    for (int kt = 0; kt < num_k && ok; ++kt) {
+      const int s = kt % STAGES;
+      const uint32_t ph = (kt / STAGES) & 1;
+      ok = tc::mbar_wait(&full[s], ph, err);
+      if (!ok) break;
+      tc::tc_fence_after();
+      const uint32_t sa = tc::smem_u32(smem + s * STAGE_BYTES);
+      const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+      for (int k = 0; k < BK / 16; ++k) {
+        tc::mma_bf16(tmem, tc::sdesc_k128(sa + k * 32), tc::sdesc_k128(sb + k * 32), idesc,
+                     (kt | k) != 0);
+      }
+      tc::mma_commit(&empty[s]);
+    }
+    tc::mma_commit(acc_full);
+  } else if (warp >= 2) {
+    // ---------------------------------------------------------- epilogue
+    const int quarter = warp & 3;  // TMEM lanes this warp may access
+    const int row = quarter * 32 + lane;
+    const int m = m0 + row;
+    const bool ok = tc::mbar_wait(acc_full, 0, err);
+    __syncwarp();
+    tc::tc_fence_after();
+    const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16);
+    float v[32], u[32];
+    if (EPI == kEpiArgmax) {
+      float best = -INFINITY;
+      int bidx = 0x7fffffff;
+      for (int c = 0; c < BN; c += 32) {
+        tc::tmem_ld32(taddr + c, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int n = n0 + c + i;
+          if (n < g.N && v[i] > best) best = v[i], bidx = n;
+        }
+      }
+      if (ok && m < g.M) {
+        g.pval[(size_t)m * g.n_parts + blockIdx.y] = best;
+        g.pidx[(size_t)m * g.n_parts + blockIdx.y] = bidx;
+      }
+    } else {
+      for (int c = 0; c < ncols_out; c += 32) {
+        tc::tmem_ld32(taddr + c, v);
+        if (EPI == kEpiSwiGLU) tc::tmem_ld32(taddr + BN / 2 + c, u);
+        if (!ok || m >= g.M) continue;
+        const int nb = n0 + c;
+        if (EPI == kEpiStore && g.out_f32) {
+          float* o = (float*)g.out + (size_t)m * g.ldo + nb;
+          if (nb + 32 <= g.N && (((uintptr_t)o) & 15) == 0) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) *(float4*)(o + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+          } else {
+            for (int i = 0; i < 32; ++i)
+              if (nb + i < g.N) o[i] = v[i];
+          }
+        } else if (EPI == kEpiResid) {
+          float* o = (float*)g.out + (size_t)m * g.ldo + nb;
+          if (nb + 32 <= g.N && (((uintptr_t)o) & 15) == 0) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+              float4 x = *(float4*)(o + i);
+              x.x += v[i], x.y += v[i + 1], x.z += v[i + 2], x.w += v[i + 3];
+              *(float4*)(o + i) = x;
+            }
+          } else {
+            for (int i = 0; i < 32; ++i)
+              if (nb + i < g.N) o[i] += v[i];
+          }
+        } else {
+          if (EPI == kEpiSwiGLU) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = silu(v[i]) * u[i];
+          }
+          bf16* o = (bf16*)g.out + (size_t)m * g.ldo + nb;
+          if (nb + 32 <= g.N && (((uintptr_t)o) & 15) == 0) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 8) {
+              __align__(16) bf16 t[8];
+#pragma unroll
+              for (int k = 0; k < 8; ++k) t[k] = __float2bfloat16_rn(v[i + k]);
+              *(uint4*)(o + i) = *(uint4*)t;
+            }
+          } else {
+            for (int i = 0; i < 32; ++i)
+              if (nb + i < g.N) o[i] = __float2bfloat16_rn(v[i]);
+          }
+        }
+      }
+    }
+    tc::tc_fence_before();
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------ tensor maps
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)p;
+  });
+  return fn;
+}
+
+// 2-D bf16 map of a row-major [rows, cols] matrix with leading dimension ld
+// (elements), box = box_rows x 64 columns, 128-byte swizzle, zero fill.
+bool make_map(CUtensorMap* m, const void* base, long rows, long cols, long ld, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+  cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int EPI>
+bool launch_tc(const GemmArgs& g, cudaStream_t s, int* err) {
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    if (cudaFuncSetAttribute(gemm_tc_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
+        cudaSuccess) {
+      set_error("cudaFuncSetAttribute(gemm_tc_kernel) failed");
+      return false;
+    }
+    attr_set[dev] = true;
+  }
+  CUtensorMap ta, tb, tb2;
+  const int brows = (EPI == kEpiSwiGLU) ? BN / 2 : BN;
+  bool ok = make_map(&ta, g.A, g.M, g.K, g.lda, BM) && make_map(&tb, g.B, g.N, g.K, g.ldb, brows);
+  if (EPI == kEpiSwiGLU) ok = ok && make_map(&tb2, g.B2, g.N, g.K, g.ldb, brows);
+  else tb2 = tb;
+  if (!ok) {
+    set_error("cuTensorMapEncodeTiled failed (M=%d N=%d K=%d)", g.M, g.N, g.K);
+    return false;
+  }
+  const int ncols_out = (EPI == kEpiSwiGLU) ? BN / 2 : BN;
+  dim3 grid(cdiv(g.M, BM), cdiv(g.N, ncols_out));
+  gemm_tc_kernel<EPI><<<grid, THREADS, SMEM_BYTES, s>>>(ta, tb, tb2, g, err);
+  note_launch();
+  return true;
+}
+
+}  // namespace
+
+int* device_error_word();  // hspec_abi.cu
+
+int argmax_tile_n(int dtype) { return dtype == HSPEC_DTYPE_BF16 ? BN : 64; }
+
+bool gemm(int dtype, GemmEpi epi, const GemmArgs& g, cudaStream_t s) {
+  if (dtype != HSPEC_DTYPE_BF16) {
+    gemm_simt_f32(epi, g, s);
+    return true;
+  }
+  // TMA needs 16-byte aligned bases and row strides.
+  if ((g.lda % 8) || (g.ldb % 8) || (((uintptr_t)g.A) & 15) || (((uintptr_t)g.B) & 15) ||
+      (g.B2 && (((uintptr_t)g.B2) & 15))) {
+    set_error("bf16 GEMM operands need 16-byte aligned bases and leading dimensions (lda=%ld ldb=%ld)",
+              g.lda, g.ldb);
+    return false;
+  }
+  int* err = device_error_word();
+  switch (epi) {
+    case kEpiStore: return launch_tc<kEpiStore>(g, s, err);
+    case kEpiResid: return launch_tc<kEpiResid>(g, s, err);
+    case kEpiSwiGLU: return launch_tc<kEpiSwiGLU>(g, s, err);
+    case kEpiArgmax: return launch_tc<kEpiArgmax>(g, s, err);
+  }
+  return false;
+}
+
+}  // namespace hspec

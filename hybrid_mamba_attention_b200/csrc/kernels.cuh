@@ -1,0 +1,92 @@
+// Internal launchers of the libhspec kernels (called by hspec_abi.cu).
+// `dtype` is HSPEC_DTYPE_F32 (elements are float) or HSPEC_DTYPE_BF16 (bf16).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace hspec {
+
+// ------------------------------------------------------------ rows.cu
+// x[m][:] = float(table[tokens[m]][:])  (embedding rows of the tied LM head)
+void embed_rows(int dtype, const int32_t* tokens, const void* table, int vocab, float* x, int M, int d,
+                int* err, cudaStream_t s);
+// x[i] = float(in[i])
+void rows_to_f32(int dtype, const void* in, float* x, long n, cudaStream_t s);
+// out[m][:] = x[m][:] / sqrt(mean(x[m]^2) + eps) * w   (out in dtype)
+void rmsnorm_rows(int dtype, const float* x, const float* w, void* out, int M, int n, float eps,
+                  cudaStream_t s);
+// out[m][:] = gate ? rmsnorm(y[m] * silu(z[m])) * w : y[m]   (z rows at z_stride elements)
+void gated_rmsnorm_rows(int dtype, const float* y, const void* z, long z_stride, const float* w,
+                        void* out, int M, int n, float eps, bool gate, cudaStream_t s);
+// In-place rotate-half RoPE on heads [0, n_heads) of every row m = c*K + j of qkv, at
+// position ctx_lens[c] + j.
+void rope_rows(int dtype, void* qkv, long row_stride, const int32_t* ctx_lens, int C, int K,
+               int n_heads, int D, float theta, cudaStream_t s);
+// tokens[m] = argmax over parts of (pval, pidx)[m][:] (lowest id on ties); top[m] = its value.
+void argmax_reduce(const float* pval, const int32_t* pidx, int M, int n_parts, int32_t* tokens,
+                   float* top, cudaStream_t s);
+
+// ------------------------------------------------------------ gemm_simt.cu / gemm_tc.cu
+enum GemmEpi : int {
+  kEpiStore = 0,      // out (dtype, or fp32 if out_f32) = acc
+  kEpiResid = 1,      // x (fp32) += acc
+  kEpiSwiGLU = 2,     // out (dtype) = silu(acc(B)) * acc(B2)
+  kEpiArgmax = 3,     // (pval, pidx)[m][n_tile] = per-row max / argmax over the tile's columns
+};
+
+struct GemmArgs {
+  int M, N, K;
+  const void* A; long lda;     // [M, K] row-major (dtype)
+  const void* B; long ldb;     // [N, K] row-major (dtype)
+  const void* B2;              // second [N, K] operand (SwiGLU up projection)
+  void* out; long ldo;         // output (see epilogue)
+  bool out_f32;                // kEpiStore: fp32 output instead of dtype
+  float* pval; int32_t* pidx;  // kEpiArgmax partials [M, n_parts]
+  int n_parts;
+};
+
+// Column tile width of the argmax partials (n_parts = ceil(N / argmax_tile_n(dtype))).
+int argmax_tile_n(int dtype);
+// out = epilogue(A . B^T); false (with the message recorded) if it cannot launch.
+bool gemm(int dtype, GemmEpi epi, const GemmArgs& g, cudaStream_t s);
+
+// ------------------------------------------------------------ ssd.cu
+struct SsdArgs {
+  int C, K, H, P, N, Q;        // Q: chunk length
+  const void* x; long x_rs;    // dtype, token row stride (head h at column h*P)
+  const void* dt; long dt_rs;  // dt (fp32) or, with dt_bias, dt_raw (dtype); head h at column h
+  const float* dt_bias;        // NULL: dt given; else dt = softplus(dt_raw + dt_bias)
+  const float* A; const float* D;
+  const void* B; const void* Cm; long bc_rs;  // dtype, token row stride
+  const float* h0;             // [C,H,P,N] or NULL
+  float* y; long y_rs;         // fp32, token row stride (head h at column h*P)
+  float* hK;                   // [C,H,P,N] or NULL
+};
+size_t ssd_smem_bytes(int P, int N, int Q);
+void ssd_scan(int dtype, const SsdArgs& a, cudaStream_t s);
+
+// ------------------------------------------------------------ attn.cu
+struct AttnArgs {
+  int C, K, Hq, Hkv, D;
+  const void* q; long q_rs;              // token row stride; head h at column h*D
+  const void* k_pool; const void* v_pool; int num_pages; int page_size;
+  const int32_t* page_table; int max_pages;
+  const int32_t* ctx_lens;
+  const void* kb; long kb_rs;            // block keys, kv head g at column g*D
+  const void* vb; long vb_rs;
+  void* out; long o_rs;                  // dtype, token row stride
+  int split_tokens;                      // tokens per split (multiple of 16)
+  int n_splits;                          // splits per (request, kv head) upper bound
+  bool causal_block;
+  float* ws_acc; float* ws_ml;           // split partials
+  int* err;
+};
+// Split policy and workspace bytes for the partials.
+int attn_split_tokens(int C, int Hkv, int K, int max_ctx, int requested);
+size_t attn_ws_bytes(int C, int Hkv, int K, int G, int D, int n_splits);
+bool attn_supported(int K, int G, int D);
+void attn_paged(int dtype, const AttnArgs& a, cudaStream_t s);
+
+}  // namespace hspec

@@ -1,0 +1,182 @@
+// Row-wise kernels of the draft step: embedding gather, RMSNorm, the Mamba-2 gated
+// RMSNorm, rotary embedding and the final argmax reduction.  All are HBM-bound
+// streaming kernels: one CTA per row (or per group of rows), fp32 arithmetic,
+// coalesced loads along the row.
+#include "common.cuh"
+#include "kernels.cuh"
+#include "../../include/hspec.h"
+
+namespace hspec {
+namespace {
+
+constexpr int kRowThreads = 256;
+
+template <typename T>
+__global__ void embed_kernel(const int32_t* __restrict__ tokens, const T* __restrict__ table, int vocab,
+                             float* __restrict__ x, int d, int* err) {
+  const int m = blockIdx.x;
+  const int tok = tokens[m];
+  const bool ok = tok >= 0 && tok < vocab;
+  if (!ok && threadIdx.x == 0) flag_error(err, kErrTokenOOB);
+  for (int e = threadIdx.x; e < d; e += blockDim.x)
+    x[(size_t)m * d + e] = ok ? to_f(table[(size_t)tok * d + e]) : 0.f;
+}
+
+template <typename T>
+__global__ void to_f32_kernel(const T* __restrict__ in, float* __restrict__ x, long n) {
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x)
+    x[i] = to_f(in[i]);
+}
+
+// RMSNorm of one fp32 row per CTA: out = x * rsqrt(mean(x^2) + eps) * w.
+template <typename T>
+__global__ void rmsnorm_kernel(const float* __restrict__ x, const float* __restrict__ w,
+                               T* __restrict__ out, int n, float eps) {
+  __shared__ float red[32];
+  const float* row = x + (size_t)blockIdx.x * n;
+  float ss = 0.f;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) ss += row[i] * row[i];
+  ss = block_sum(ss, red);
+  const float inv = 1.f / sqrtf(ss / n + eps);  // correctly rounded: fewer bf16 rounding flips
+  T* o = out + (size_t)blockIdx.x * n;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) o[i] = from_f<T>(row[i] * inv * w[i]);
+}
+
+// Mamba-2 output gate: g = y * silu(z), then RMSNorm over the H*P features.
+template <typename T>
+__global__ void gated_rmsnorm_kernel(const float* __restrict__ y, const T* __restrict__ z, long z_stride,
+                                     const float* __restrict__ w, T* __restrict__ out, int n, float eps,
+                                     bool gate) {
+  __shared__ float red[32];
+  const float* yr = y + (size_t)blockIdx.x * n;
+  T* o = out + (size_t)blockIdx.x * n;
+  if (!gate) {
+    for (int i = threadIdx.x; i < n; i += blockDim.x) o[i] = from_f<T>(yr[i]);
+    return;
+  }
+  const T* zr = z + (size_t)blockIdx.x * z_stride;
+  float ss = 0.f;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    float g = yr[i] * silu(to_f(zr[i]));
+    ss += g * g;
+  }
+  ss = block_sum(ss, red);
+  const float inv = 1.f / sqrtf(ss / n + eps);
+  for (int i = threadIdx.x; i < n; i += blockDim.x)
+    o[i] = from_f<T>(yr[i] * silu(to_f(zr[i])) * inv * w[i]);
+}
+
+// Rotate-half RoPE in place.  One thread per (row, head, pair i); the angle
+// pos * theta^(-2i/D) is formed and reduced in double so that positions up to
+// 10^5 keep full fp32 accuracy in cos/sin.
+template <typename T>
+__global__ void rope_kernel(T* __restrict__ qkv, long row_stride, const int32_t* __restrict__ ctx_lens,
+                            int K, int n_heads, int D, double log_theta, long total) {
+  const long idx = blockIdx.x * (long)blockDim.x + threadIdx.x;
+  if (idx >= total) return;
+  const int half = D / 2;
+  const int i = (int)(idx % half);
+  const long rh = idx / half;
+  const int h = (int)(rh % n_heads);
+  const long m = rh / n_heads;
+  const int c = (int)(m / K), j = (int)(m % K);
+  const double pos = (double)ctx_lens[c] + j;
+  const double ang = pos * exp(-2.0 * i / D * log_theta);
+  double sn, cs;
+  sincos(ang, &sn, &cs);
+  T* v = qkv + m * row_stride + (long)h * D;
+  const double a = to_f(v[i]), b = to_f(v[i + half]);
+  v[i] = from_f<T>((float)(a * cs - b * sn));
+  v[i + half] = from_f<T>((float)(a * sn + b * cs));
+}
+
+// One warp per row: scans the per-tile partial maxima in column order, keeping
+// the first (lowest id) of equal maxima.
+__global__ void argmax_reduce_kernel(const float* __restrict__ pval, const int32_t* __restrict__ pidx,
+                                     int M, int n_parts, int32_t* __restrict__ tokens,
+                                     float* __restrict__ top) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (warp >= M) return;
+  float best = -INFINITY;
+  int bidx = 0x7fffffff;
+  for (int p = lane; p < n_parts; p += 32) {
+    float v = pval[(size_t)warp * n_parts + p];
+    int id = pidx[(size_t)warp * n_parts + p];
+    if (v > best || (v == best && id < bidx)) best = v, bidx = id;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    float v = __shfl_xor_sync(0xffffffffu, best, o);
+    int id = __shfl_xor_sync(0xffffffffu, bidx, o);
+    if (v > best || (v == best && id < bidx)) best = v, bidx = id;
+  }
+  if (lane == 0) {
+    tokens[warp] = bidx;
+    if (top) top[warp] = best;
+  }
+}
+
+}  // namespace
+
+void embed_rows(int dtype, const int32_t* tokens, const void* table, int vocab, float* x, int M, int d,
+                int* err, cudaStream_t s) {
+  if (dtype == HSPEC_DTYPE_BF16)
+    embed_kernel<bf16><<<M, kRowThreads, 0, s>>>(tokens, (const bf16*)table, vocab, x, d, err);
+  else
+    embed_kernel<float><<<M, kRowThreads, 0, s>>>(tokens, (const float*)table, vocab, x, d, err);
+  note_launch();
+}
+
+void rows_to_f32(int dtype, const void* in, float* x, long n, cudaStream_t s) {
+  int grid = (int)((n + kRowThreads - 1) / kRowThreads);
+  if (grid > 148 * 16) grid = 148 * 16;
+  if (dtype == HSPEC_DTYPE_BF16)
+    to_f32_kernel<bf16><<<grid, kRowThreads, 0, s>>>((const bf16*)in, x, n);
+  else
+    to_f32_kernel<float><<<grid, kRowThreads, 0, s>>>((const float*)in, x, n);
+  note_launch();
+}
+
+void rmsnorm_rows(int dtype, const float* x, const float* w, void* out, int M, int n, float eps,
+                  cudaStream_t s) {
+  if (dtype == HSPEC_DTYPE_BF16)
+    rmsnorm_kernel<bf16><<<M, kRowThreads, 0, s>>>(x, w, (bf16*)out, n, eps);
+  else
+    rmsnorm_kernel<float><<<M, kRowThreads, 0, s>>>(x, w, (float*)out, n, eps);
+  note_launch();
+}
+
+void gated_rmsnorm_rows(int dtype, const float* y, const void* z, long z_stride, const float* w,
+                        void* out, int M, int n, float eps, bool gate, cudaStream_t s) {
+  if (dtype == HSPEC_DTYPE_BF16)
+    gated_rmsnorm_kernel<bf16><<<M, kRowThreads, 0, s>>>(y, (const bf16*)z, z_stride, w, (bf16*)out, n,
+                                                         eps, gate);
+  else
+    gated_rmsnorm_kernel<float><<<M, kRowThreads, 0, s>>>(y, (const float*)z, z_stride, w, (float*)out,
+                                                          n, eps, gate);
+  note_launch();
+}
+
+void rope_rows(int dtype, void* qkv, long row_stride, const int32_t* ctx_lens, int C, int K,
+               int n_heads, int D, float theta, cudaStream_t s) {
+  const long total = (long)C * K * n_heads * (D / 2);
+  const int grid = (int)((total + kRowThreads - 1) / kRowThreads);
+  const double lt = log((double)theta);
+  if (dtype == HSPEC_DTYPE_BF16)
+    rope_kernel<bf16><<<grid, kRowThreads, 0, s>>>((bf16*)qkv, row_stride, ctx_lens, K, n_heads, D, lt,
+                                                   total);
+  else
+    rope_kernel<float><<<grid, kRowThreads, 0, s>>>((float*)qkv, row_stride, ctx_lens, K, n_heads, D,
+                                                    lt, total);
+  note_launch();
+}
+
+void argmax_reduce(const float* pval, const int32_t* pidx, int M, int n_parts, int32_t* tokens,
+                   float* top, cudaStream_t s) {
+  const int warps_per_block = 8;
+  argmax_reduce_kernel<<<(M + warps_per_block - 1) / warps_per_block, 32 * warps_per_block, 0, s>>>(
+      pval, pidx, M, n_parts, tokens, top);
+  note_launch();
+}
+
+}  // namespace hspec

@@ -1,0 +1,254 @@
+/*
+ * hspec.h -- C-ABI of libhspec.so: the block-parallel draft step of the H-Spec
+ * hybrid Mamba-attention drafter on NVIDIA B200 (sm_100a).
+ *
+ * What the library computes (H-Spec: Parallel Speculative Decoding Without a
+ * Drafter-Side KV Cache, arXiv 2609.24197, Abstract; evolve.pub review, Summary):
+ * a drafter proposes K tokens of a block in parallel.  Its attention layers read the
+ * target model's paged KV cache IN PLACE (the drafter keeps no KV cache of its own),
+ * and its Mamba-2 layers start from a state projected from the target's last-token
+ * hidden state, h0 = reshape(W_inj . h_last).  The Mamba-2 scan over the K block
+ * positions is evaluated in parallel chunks (the SSD form of Dao & Gu, 2024):
+ *     h_t = exp(dt_t A) h_{t-1} + dt_t x_t (x) B_t,     y_t = C_t . h_t + D x_t.
+ *
+ * Conventions for every entry point
+ *  - Pointers marked "device" are caller-owned CUDA device memory; the library never
+ *    frees, copies or keeps them beyond the call (the target KV pool is read in place
+ *    and never written).  Host structs are read during the call only.
+ *  - Matrices are row-major; weights are [out_features, in_features].
+ *  - Element type: hspec_cfg.dtype selects fp32 or bf16 for weights, activations and
+ *    the KV pool.  Recurrent state (h0, hK), dt, A, D, norm weights and the SSD
+ *    output y are always fp32.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t, NULL = legacy default
+ *    stream).  The returned status covers host-side validation and launch errors.
+ *    Invalid arguments are rejected before anything is launched.  Errors that only
+ *    the device can see (a page id outside the pool, a context longer than the page
+ *    table, a token id outside the vocabulary) set a device error word; the kernels
+ *    skip the offending read (it contributes nothing) and hspec_sync_status() reports
+ *    HSPEC_ERR_DEVICE_CHECK.
+ *  - No entry point allocates device memory.  Scratch space comes from a
+ *    caller-provided workspace whose size the *_workspace_size functions return.
+ *  - Thread safety: calls on different streams may run concurrently if their
+ *    workspaces differ.
+ */
+#ifndef HSPEC_H
+#define HSPEC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define HSPEC_API __attribute__((visibility("default")))
+#else
+#define HSPEC_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int hspec_status;
+#define HSPEC_OK 0
+#define HSPEC_ERR_INVALID_ARG 1     /* null pointer, non-positive size, bad flag        */
+#define HSPEC_ERR_SHAPE_MISMATCH 2  /* e.g. Hq not a multiple of Hkv, dims inconsistent  */
+#define HSPEC_ERR_PAGE_OOB 3        /* page table width / pool size inconsistent (host)  */
+#define HSPEC_ERR_UNSUPPORTED 4     /* shape outside what the kernels implement          */
+#define HSPEC_ERR_CUDA 5            /* a CUDA runtime call or kernel launch failed        */
+#define HSPEC_ERR_DEVICE_CHECK 6    /* a kernel saw a bad page id / ctx length / token   */
+#define HSPEC_ERR_WORKSPACE 7       /* workspace missing, too small or misaligned         */
+
+#define HSPEC_DTYPE_F32 0
+#define HSPEC_DTYPE_BF16 1
+
+#define HSPEC_FLAG_ROPE 1           /* rotary embedding on q and block keys at ctx_c + j */
+#define HSPEC_FLAG_GATE 2           /* Mamba-2 gated RMSNorm y <- norm(y * silu(z)) w_g  */
+#define HSPEC_FLAG_CAUSAL_BLOCK 4   /* block query j sees block key i only when i <= j   */
+
+#define HSPEC_MAX_LAYERS 16
+
+/* Shapes and options of one drafter.  The attention dims must equal the target's
+ * (the drafter reads the target KV as is: evolve.pub review, limitations). */
+typedef struct hspec_cfg {
+  int d_model;                      /* d: hidden size (= target hidden size)              */
+  int n_q_heads;                    /* Hq                                                  */
+  int n_kv_heads;                   /* Hkv; GQA group G = Hq / Hkv                         */
+  int head_dim;                     /* D (attention), even                                 */
+  int n_ssm_heads;                  /* H  (Mamba-2 heads)                                  */
+  int ssm_head_dim;                 /* P  (Mamba-2 head dim)                               */
+  int d_state;                      /* N  (Mamba-2 state size)                             */
+  int page_size;                    /* tokens per KV page (vLLM block size)                */
+  int d_ff;                         /* SwiGLU intermediate size, 0 = no MLP sub-layer      */
+  int vocab;                        /* LM-head rows, 0 = no head (step returns hidden)     */
+  int n_layers;                     /* <= HSPEC_MAX_LAYERS                                 */
+  char layer_kinds[HSPEC_MAX_LAYERS];/* 'M' = Mamba-2 layer, 'A' = attention layer         */
+  int dtype;                        /* HSPEC_DTYPE_F32 or HSPEC_DTYPE_BF16                 */
+  int flags;                        /* HSPEC_FLAG_*                                        */
+  float rope_theta;                 /* RoPE base                                           */
+  float norm_eps;                   /* RMSNorm epsilon                                     */
+  int ssd_chunk;                    /* SSD chunk length Q (0 = whole block in one chunk)   */
+  int attn_split_tokens;            /* tokens per split-KV partition, multiple of 16 (0 = auto) */
+} hspec_cfg;
+
+/* Weights of one layer (caller-owned device memory; fields of the other layer kind
+ * and of an absent MLP are ignored). */
+typedef struct hspec_layer_weights {
+  const float* norm;      /* [d]            pre-mixer RMSNorm weight                     */
+  const void* W_in;       /* [2HP+2N+H, d]  Mamba-2 in_proj, rows [z | x | B | C | dt]  */
+  const float* dt_bias;   /* [H]            dt = softplus(dt_raw + dt_bias)             */
+  const float* A;         /* [H]            negative per-head decay rate                */
+  const float* D;         /* [H]            skip coefficient                            */
+  const float* gnorm;     /* [HP]           gated-RMSNorm weight                        */
+  const void* W_out;      /* [d, HP]        Mamba-2 out_proj                            */
+  const void* W_inj;      /* [HPN, d]       state injection, rows (h*P + p)*N + n       */
+  const void* W_qkv;      /* [(Hq+2Hkv)D, d] attention projections, rows [q | k | v]    */
+  const void* W_o;        /* [d, Hq D]      attention output projection                 */
+  const float* mlp_norm;  /* [d]            pre-MLP RMSNorm weight                      */
+  const void* W_gate;     /* [d_ff, d]                                                  */
+  const void* W_up;       /* [d_ff, d]                                                  */
+  const void* W_down;     /* [d, d_ff]                                                  */
+} hspec_layer_weights;
+
+typedef struct hspec_model_weights {
+  hspec_layer_weights layers[HSPEC_MAX_LAYERS];
+  const float* final_norm; /* [d]                                                        */
+  const void* W_lm;        /* [vocab, d] shared LM head, also the token embedding table  */
+} hspec_model_weights;
+
+/* The target's paged KV cache, read in place (never written, never copied). */
+typedef struct hspec_kv_view {
+  const void* k_pool;          /* device [num_pages, page_size, Hkv, D]                  */
+  const void* v_pool;          /* device [num_pages, page_size, Hkv, D]                  */
+  int num_pages;               /* pages in the pool                                       */
+  const int32_t* page_table;   /* device [C, max_pages]; token t of request c lives in
+                                  page page_table[c][t / page_size], slot t % page_size   */
+  int max_pages;               /* page-table width; ctx_lens[c] <= max_pages * page_size  */
+} hspec_kv_view;
+
+/* ------------------------------------------------------------------ kernels
+ * Each of the three calls below is one step of the draft step, usable alone. */
+
+/* State injection (H-Spec Abstract: "Mamba modules are initialized with projected
+ * last-token target hidden states").
+ *   h0[c][h][p][n] = sum_j W_inj[(h*P+p)*N+n][j] * h_last[c][j]
+ * W_inj  device [H*P*N, d] (dtype); h_last device [C, d] (dtype);
+ * h0     device [C, H, P, N] fp32, written.  C >= 1. */
+HSPEC_API hspec_status hspec_inject_state(const hspec_cfg* cfg, const void* W_inj, const void* h_last, int C,
+                                float* h0, void* stream);
+
+/* Mamba-2 SSD scan over the K block positions of every request, started from h0
+ * (H-Spec Abstract: "Mamba's parallel scan allows H-Spec to preserve block-parallel
+ * drafting"), evaluated in chunks of cfg->ssd_chunk positions:
+ *   h_t = exp(dt_t A_h) h_{t-1} + dt_t x_t (x) B_t;  y_t = C_t . h_t + D_h x_t.
+ * x  device [C, K, H, P] (dtype);  dt device [C, K, H] fp32 (already positive);
+ * A, D device [H] fp32;  B, Cm device [C, K, N] (dtype, one group for all heads);
+ * h0 device [C, H, P, N] fp32 (NULL = zero state);
+ * y  device [C, K, H, P] fp32, written;  hK device [C, H, P, N] fp32 final state,
+ * written when not NULL.  1 <= K <= 64. */
+HSPEC_API hspec_status hspec_ssd_block_scan(const hspec_cfg* cfg, const void* x, const float* dt,
+                                  const float* A, const void* B, const void* Cm, const float* D,
+                                  const float* h0, int C, int K, float* y, float* hK, void* stream);
+
+/* Workspace bytes hspec_attn_paged_block needs for C requests of K block tokens and
+ * a page table of width max_pages (the split-KV partials). */
+HSPEC_API size_t hspec_attn_workspace_size(const hspec_cfg* cfg, int C, int K, int max_pages);
+
+/* Paged in-place GQA attention of the K block queries (H-Spec Abstract: "attention
+ * modules reuse target KVs in place").  Query (c, j, h) attends, with scale
+ * 1/sqrt(D), over the ctx_lens[c] context tokens of request c read through the page
+ * table, followed by the K block keys of request c (all visible unless
+ * HSPEC_FLAG_CAUSAL_BLOCK); kv head = h / (Hq/Hkv).  Long contexts are split across
+ * CTAs and the partial (max, sum, acc) merged.
+ * q      device [C, K, Hq, D] (dtype);   kv: the target cache;
+ * ctx_lens device [C] int32, 0 <= ctx_lens[c] <= kv->max_pages * page_size;
+ * k_blk, v_blk device [C, K, Hkv, D] (dtype);
+ * out    device [C, K, Hq, D] (dtype), written;
+ * workspace device, >= hspec_attn_workspace_size() bytes, 256-byte aligned. */
+HSPEC_API hspec_status hspec_attn_paged_block(const hspec_cfg* cfg, const void* q, const hspec_kv_view* kv,
+                                    const int32_t* ctx_lens, const void* k_blk, const void* v_blk,
+                                    int C, int K, void* out, void* workspace, size_t ws_bytes,
+                                    void* stream);
+
+/* ------------------------------------------------------------- draft step */
+
+typedef struct hspec_drafter hspec_drafter;
+
+/* Validates cfg and keeps a host copy of it and of the weight pointers (device
+ * memory stays caller-owned and must outlive the drafter).  Allocates no device
+ * memory.  *out receives the handle. */
+HSPEC_API hspec_status hspec_drafter_create(const hspec_cfg* cfg, const hspec_model_weights* weights,
+                                  hspec_drafter** out);
+HSPEC_API void hspec_drafter_destroy(hspec_drafter* drafter);
+
+typedef struct hspec_step_in {
+  int C;                       /* requests in the batch                                   */
+  int K;                       /* block size (tokens drafted in parallel), 1..64          */
+  const int32_t* tokens;       /* device [C, K] block tokens, used when vocab > 0         */
+  const void* x_in;            /* device [C, K, d] (dtype) block input, used when vocab == 0 */
+  const void* h_last;          /* device [C, d] (dtype) target last-token hidden state    */
+  const int32_t* ctx_lens;     /* device [C] target context length per request            */
+  hspec_kv_view kv[HSPEC_MAX_LAYERS]; /* one target cache per attention layer, in order   */
+} hspec_step_in;
+
+typedef struct hspec_step_out {
+  int32_t* draft_tokens;       /* device [C, K] argmax token ids (vocab > 0), or NULL     */
+  float* hidden;               /* device [C, K, d] fp32 residual stream after the last
+                                  layer, or NULL                                          */
+  void* final_normed;          /* device [C, K, d] (dtype) final RMSNorm output (the LM-head
+                                  input), or NULL                                         */
+  float* top_logit;            /* device [C, K] logit of the argmax token, or NULL        */
+  float* layer_hidden;         /* device [n_layers, C, K, d] fp32 residual stream after each
+                                  layer (for layer-by-layer validation), or NULL          */
+} hspec_step_out;
+
+/* Workspace bytes hspec_draft_step needs (activations, h0 of one Mamba layer,
+ * split-KV partials, argmax partials). */
+HSPEC_API size_t hspec_step_workspace_size(const hspec_cfg* cfg, int C, int K, int max_pages);
+
+/* One block-parallel draft step (all layers, then the LM-head argmax when vocab > 0):
+ * per layer, pre-norm residual blocks
+ *   M: x += W_out gnorm(SSD(in_proj(norm(x)); h0 = W_inj h_last) * silu(z))
+ *   A: x += W_o attn(rope(q), target KV in place ++ rope(k_blk), v_blk)
+ *   MLP (d_ff > 0): x += W_down (silu(W_gate norm(x)) * W_up norm(x))
+ * then draft_tokens = argmax(W_lm final_norm(x)).  max_pages of every kv view must be
+ * <= the max_pages given to hspec_step_workspace_size. */
+HSPEC_API hspec_status hspec_draft_step(hspec_drafter* drafter, const hspec_step_in* in,
+                              const hspec_step_out* out, void* workspace, size_t ws_bytes,
+                              void* stream);
+
+/* --------------------------------------------------------------- status */
+
+/* Synchronises `stream`, then returns HSPEC_ERR_DEVICE_CHECK if any kernel of this
+ * library flagged a bad page id, context length or token id since the last call (and
+ * clears the flag), HSPEC_ERR_CUDA on a CUDA error, else HSPEC_OK. */
+HSPEC_API hspec_status hspec_sync_status(void* stream);
+
+/* Static description of a status code. */
+HSPEC_API const char* hspec_status_string(hspec_status status);
+
+/* Message of the most recent failure in this thread ("" if none). */
+HSPEC_API const char* hspec_last_error(void);
+
+/* Kernels this library has launched since load (all threads). */
+HSPEC_API unsigned long long hspec_launch_count(void);
+
+/* Kernel timing (tracing aid).  hspec_profile_enable(1) clears the record and makes
+ * hspec_draft_step record a CUDA event pair on its stream around each group of
+ * kernels it launches (one group per step of the draft step: "in_proj",
+ * "attn_paged", "lm_head_argmax", ...); hspec_profile_enable(0) stops recording.
+ * Events are created on demand, so do not enable it during CUDA graph capture. */
+HSPEC_API hspec_status hspec_profile_enable(int on);
+
+/* Synchronises the recorded events and writes, per kernel group, its name into
+ * names[i*32 .. i*32+31] (NUL-terminated), the summed event time in milliseconds
+ * into total_ms[i] and the number of recorded occurrences into count[i], for at
+ * most max_entries groups.  Returns the number of groups written, or -1 on a CUDA
+ * error. */
+HSPEC_API int hspec_profile_read(char* names, double* total_ms, int* count, int max_entries);
+
+/* Library version string. */
+HSPEC_API const char* hspec_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HSPEC_H */

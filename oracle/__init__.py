@@ -170,6 +170,29 @@ def lm_head_argmax(hn, W_lm):
     return am, t1, t2
 
 
+# ------------------------------------------------------------ host copies
+
+def host_weights(w: dict) -> dict:
+    """Host copy of a weights dict (inputs.make_weights layout)."""
+    cpu = lambda v: v.detach().to("cpu") if torch.is_tensor(v) else v
+    return {"layers": [{k: cpu(v) for k, v in L.items()} for L in w["layers"]],
+            **{k: cpu(v) for k, v in w.items() if k != "layers"}}
+
+
+def host_sub_cache(cache: dict, rows) -> dict:
+    """Host copy of the pages that `rows` of the page table use, with the table
+    rewritten to the copied order (the oracle still gathers through the table)."""
+    tbl = cache["page_table"].detach().to("cpu")[rows]
+    used = tbl[tbl >= 0].unique()
+    remap = torch.full((int(cache["k_pool"].shape[0]),), -1, dtype=torch.int32)
+    remap[used.long()] = torch.arange(used.numel(), dtype=torch.int32)
+    new_tbl = torch.where(tbl >= 0, remap[tbl.clamp(min=0).long()], tbl)
+    idx = used.long().to(cache["k_pool"].device)
+    return {"k_pool": cache["k_pool"].index_select(0, idx).to("cpu"),
+            "v_pool": cache["v_pool"].index_select(0, idx).to("cpu"),
+            "page_table": new_tbl.contiguous()}
+
+
 # ----------------------------------------------------------------- draft step
 
 class _Cfg(ct.Structure):
@@ -192,7 +215,7 @@ class _Layer(ct.Structure):
 
 class _Step(ct.Structure):
     _fields_ = [("C", ct.c_int), ("K", ct.c_int), ("tokens", ct.c_void_p), ("x_in", ct.c_void_p),
-                ("h_last", ct.c_void_p), ("ctx_lens", ct.c_void_p), ("final_norm", ct.c_void_p),
+                ("x_in_type", ct.c_int), ("h_last", ct.c_void_p), ("ctx_lens", ct.c_void_p), ("final_norm", ct.c_void_p),
                 ("W_lm", ct.c_void_p), ("hidden", ct.c_void_p), ("layer_out", ct.c_void_p),
                 ("final_normed", ct.c_void_p), ("draft_tokens", ct.c_void_p), ("top1", ct.c_void_p),
                 ("top2", ct.c_void_p)]
@@ -265,7 +288,9 @@ def draft_step(shapes, weights, kv, h_last, ctx_lens, tokens=None, x_in=None, la
         io.draft_tokens = _dptr(res["draft_tokens"]).value
         io.top1, io.top2 = _dptr(res["top1"]).value, _dptr(res["top2"]).value
     else:
-        io.x_in = hold(x_in)
+        xt, io.x_in_type = _cpu(x_in)
+        keep.append(xt)
+        io.x_in = xt.data_ptr()
     rc = lib().oracle_draft_step(ct.byref(cfg), layers, ct.byref(io))
     if rc != 0:
         raise ValueError("oracle_draft_step: page table or context length out of range")

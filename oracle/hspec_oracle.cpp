@@ -298,7 +298,7 @@ int oracle_draft_step(const oracle_cfg* cfg, const oracle_layer* layers, oracle_
       for (int e = 0; e < d; ++e)
         x[(size_t)j * d + e] = cfg->vocab > 0
             ? load(io->W_lm, dtype, (size_t)io->tokens[(size_t)c * K + j] * d + e)
-            : load(io->x_in, dtype, ((size_t)c * K + j) * d + e);
+            : load(io->x_in, io->x_in_type, ((size_t)c * K + j) * d + e);
     std::vector<double> hl(d);
     for (int e = 0; e < d; ++e) hl[e] = load(io->h_last, dtype, (size_t)c * d + e);
 

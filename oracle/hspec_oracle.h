@@ -106,6 +106,7 @@ typedef struct {
   int C, K;
   const int32_t* tokens;   /* [C,K] block tokens (used when vocab > 0) */
   const void* x_in;        /* [C,K,d] direct block input (used when vocab == 0) */
+  int x_in_type;           /* element type of x_in (ORACLE_F32 or ORACLE_BF16) */
   const void* h_last;      /* [C,d] target last-token hidden state */
   const int32_t* ctx_lens; /* [C] */
   const float* final_norm; const void* W_lm;   /* [d], [vocab,d]; W_lm is also the embedding */

@@ -1,0 +1,67 @@
+"""Helpers shared by the GPU parity tests: tolerance metrics, host copies for the
+oracle, and sampling of requests from a large batch (requests are independent, so
+the oracle may check any subset one by one).
+
+Tolerances (stated for the draft step of the H-Spec drafter):
+  fp32 outputs   max|gpu - oracle| / max|oracle|  <= 1e-4
+  bf16 outputs   max|gpu - oracle| / rms(oracle)  <= 2e-2
+  page gathers, argmax (where the oracle's top-2 gap >= 1e-3): exact
+"""
+import numpy as np
+import torch
+
+import oracle
+
+F32_TOL = 1e-4
+BF16_TOL = 2e-2
+
+
+def rel_max(gpu, ref) -> float:
+    g = np.asarray(gpu, dtype=np.float64)
+    r = np.asarray(ref, dtype=np.float64)
+    return float(np.abs(g - r).max() / max(np.abs(r).max(), 1e-300))
+
+
+def rel_rms(gpu, ref) -> float:
+    g = np.asarray(gpu, dtype=np.float64)
+    r = np.asarray(ref, dtype=np.float64)
+    return float(np.abs(g - r).max() / max(np.sqrt((r ** 2).mean()), 1e-300))
+
+
+def assert_close(gpu, ref, dtype: str, what: str = ""):
+    """fp32: max-abs relative to max|ref|; bf16: max-abs relative to rms(ref)."""
+    assert np.isfinite(np.asarray(gpu, dtype=np.float64)).all(), f"{what}: non-finite GPU output"
+    if dtype == "f32":
+        e = rel_max(gpu, ref)
+        assert e <= F32_TOL, f"{what}: fp32 max-abs/max|ref| = {e:.3e} > {F32_TOL}"
+    else:
+        e = rel_rms(gpu, ref)
+        assert e <= BF16_TOL, f"{what}: bf16 max-abs/rms(ref) = {e:.3e} > {BF16_TOL}"
+    return e
+
+
+def host(t):
+    return t.detach().to("cpu")
+
+
+def to_np(t):
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+sub_cache = oracle.host_sub_cache
+host_weights = oracle.host_weights
+
+
+def sample_requests(C: int, n: int, seed: int = 0):
+    if C <= n:
+        return list(range(C))
+    g = np.random.default_rng(seed)
+    return sorted(g.choice(C, size=n, replace=False).tolist())
+
+
+def oracle_step_for(shapes, weights_host, st: dict, rows):
+    """Oracle draft step over the requests `rows` of the batch `st` (device tensors)."""
+    kv = [sub_cache(c, rows) for c in st["kv"]]
+    return oracle.draft_step(shapes, weights_host, kv, host(st["h_last"])[rows], host(st["ctx_lens"])[rows],
+                             tokens=None if st["tokens"] is None else host(st["tokens"])[rows],
+                             x_in=None if st["x_in"] is None else host(st["x_in"])[rows])

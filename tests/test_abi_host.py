@@ -1,0 +1,169 @@
+"""CPU checks of the C-ABI library: it loads, exports every function include/hspec.h
+declares, its ctypes structs match the C layout, and host-side validation rejects
+bad arguments before anything is launched (no GPU is touched here)."""
+import ctypes as ct
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hspec.h")
+
+
+@pytest.fixture(scope="module")
+def H():
+    from hybrid_mamba_attention_b200 import hspec
+    return hspec
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"^HSPEC_API[^;(]*?\b(hspec_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_library_exports_every_declared_function(H):
+    names = declared_functions()
+    assert len(names) >= 13
+    lib = ct.CDLL(H.LIBRARY_PATH)
+    for n in names:
+        assert hasattr(lib, n), f"libhspec.so does not export {n}"
+    assert set(names) == set(H.EXPORTS)
+
+
+def test_struct_layouts_match_header(H, tmp_path):
+    prog = tmp_path / "sz.c"
+    fields = {"hspec_cfg": ["d_model", "layer_kinds", "dtype", "rope_theta", "attn_split_tokens"],
+              "hspec_step_in": ["C", "h_last", "ctx_lens", "kv"],
+              "hspec_kv_view": ["v_pool", "num_pages", "page_table", "max_pages"],
+              "hspec_model_weights": ["layers", "final_norm", "W_lm"],
+              "hspec_layer_weights": ["W_inj", "W_down"],
+              "hspec_step_out": ["draft_tokens", "top_logit"]}
+    lines = ['#include <stdio.h>', '#include <stddef.h>', f'#include "{HEADER}"', "int main(void){"]
+    for s, fs in fields.items():
+        lines.append(f'printf("%zu\\n", sizeof({s}));')
+        for f in fs:
+            lines.append(f'printf("%zu\\n", offsetof({s}, {f}));')
+    lines.append("return 0;}")
+    prog.write_text("\n".join(lines))
+    exe = tmp_path / "sz"
+    subprocess.run(["gcc", str(prog), "-o", str(exe)], check=True)
+    got = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()]
+    want = []
+    for s, fs in fields.items():
+        cls = getattr(H, s)
+        want.append(ct.sizeof(cls))
+        for f in fs:
+            want.append(getattr(cls, f).offset)
+    assert got == want
+
+
+def small_cfg(H, **kw):
+    from hybrid_mamba_attention_b200 import inputs as I
+    cfg = H.make_cfg(I.TINY)
+    for k, v in kw.items():
+        setattr(cfg, k, v)
+    return cfg
+
+
+def test_status_strings_and_version(H):
+    assert "sm_100a" in H.hspec_version()
+    for s in range(8):
+        assert H.hspec_status_string(s)
+    assert H.hspec_launch_count() >= 0
+
+
+def test_null_pointers_rejected_before_launch(H):
+    cfg = small_cfg(H)
+    n0 = H.hspec_launch_count()
+    assert H._lib.hspec_inject_state(ct.byref(cfg), None, None, 1, None, None) == H.HSPEC_ERR_INVALID_ARG
+    assert H._lib.hspec_ssd_block_scan(ct.byref(cfg), None, None, None, None, None, None, None, 1, 8, None,
+                                       None, None) == H.HSPEC_ERR_INVALID_ARG
+    assert H.hspec_launch_count() == n0
+
+
+def test_bad_config_rejected(H):
+    cfg = small_cfg(H, dtype=7)
+    assert H._lib.hspec_inject_state(ct.byref(cfg), 16, 16, 1, 16, None) == H.HSPEC_ERR_INVALID_ARG
+    assert "dtype" in H.hspec_last_error()
+    cfg = small_cfg(H, n_kv_heads=3)
+    kv = H.hspec_kv_view(k_pool=16, v_pool=16, num_pages=4, page_table=16, max_pages=4)
+    st = H._lib.hspec_attn_paged_block(ct.byref(cfg), 16, ct.byref(kv), 16, 16, 16, 1, 8, 16, 256, 1 << 20, None)
+    assert st == H.HSPEC_ERR_SHAPE_MISMATCH
+    cfg = small_cfg(H, flags=64)
+    assert H._lib.hspec_inject_state(ct.byref(cfg), 16, 16, 1, 16, None) == H.HSPEC_ERR_INVALID_ARG
+
+
+def test_unsupported_block_size_rejected(H):
+    cfg = small_cfg(H)
+    st = H._lib.hspec_ssd_block_scan(ct.byref(cfg), 16, 16, 16, 16, 16, 16, None, 1, 65, 16, None, None)
+    assert st == H.HSPEC_ERR_UNSUPPORTED
+    st = H._lib.hspec_ssd_block_scan(ct.byref(cfg), 16, 16, 16, 16, 16, 16, None, 1, 0, 16, None, None)
+    assert st == H.HSPEC_ERR_UNSUPPORTED
+
+
+def test_attention_workspace_checked(H):
+    cfg = small_cfg(H)
+    kv = H.hspec_kv_view(k_pool=16, v_pool=16, num_pages=4, page_table=16, max_pages=4)
+    need = H.hspec_attn_workspace_size(cfg, 1, 8, 4)
+    assert need > 0 and need % 256 == 0
+    st = H._lib.hspec_attn_paged_block(ct.byref(cfg), 16, ct.byref(kv), 16, 16, 16, 1, 8, 16, 256, need - 1, None)
+    assert st == H.HSPEC_ERR_WORKSPACE
+    st = H._lib.hspec_attn_paged_block(ct.byref(cfg), 16, ct.byref(kv), 16, 16, 16, 1, 8, 16, 1024 + 16, need, None)
+    assert st == H.HSPEC_ERR_WORKSPACE  # misaligned
+    bad = H.hspec_kv_view(k_pool=16, v_pool=16, num_pages=0, page_table=16, max_pages=4)
+    st = H._lib.hspec_attn_paged_block(ct.byref(cfg), 16, ct.byref(bad), 16, 16, 16, 1, 8, 16, 256, need, None)
+    assert st == H.HSPEC_ERR_PAGE_OOB
+
+
+def test_workspace_sizes_grow_with_batch_and_context(H):
+    from hybrid_mamba_attention_b200 import inputs as I
+    cfg = H.make_cfg(I.LLAMA_FULL)
+    a = H.hspec_step_workspace_size(cfg, 1, 16, 128)
+    b = H.hspec_step_workspace_size(cfg, 8, 16, 128)
+    c = H.hspec_step_workspace_size(cfg, 8, 16, 1024)
+    assert 0 < a < b <= c
+    assert a % 256 == 0
+
+
+def test_drafter_create_validates(H):
+    from hybrid_mamba_attention_b200 import inputs as I
+    cfg = H.make_cfg(I.TINY)
+    mw = H.hspec_model_weights()
+    h = ct.c_void_p()
+    assert H._lib.hspec_drafter_create(ct.byref(cfg), ct.byref(mw), ct.byref(h)) == H.HSPEC_ERR_INVALID_ARG
+    cfg.layer_kinds = b"MX"
+    assert H._lib.hspec_drafter_create(ct.byref(cfg), ct.byref(mw), ct.byref(h)) == H.HSPEC_ERR_INVALID_ARG
+    cfg = H.make_cfg(I.TINY)
+    cfg.n_layers = 0
+    assert H._lib.hspec_drafter_create(ct.byref(cfg), ct.byref(mw), ct.byref(h)) == H.HSPEC_ERR_INVALID_ARG
+    # bf16 drafters need TMA-friendly dims
+    cfg = H.make_cfg(I.LLAMA)
+    cfg.d_model = 4100
+    for i in range(2):
+        for f, _ in H.hspec_layer_weights._fields_:
+            setattr(mw.layers[i], f, 256)
+    assert H._lib.hspec_drafter_create(ct.byref(cfg), ct.byref(mw), ct.byref(h)) == H.HSPEC_ERR_UNSUPPORTED
+    cfg.d_model = 4096
+    assert H._lib.hspec_drafter_create(ct.byref(cfg), ct.byref(mw), ct.byref(h)) == H.HSPEC_OK
+    H.hspec_drafter_destroy(h)
+
+
+def test_step_rejects_missing_inputs(H):
+    from hybrid_mamba_attention_b200 import inputs as I
+    cfg = H.make_cfg(I.TINY)
+    mw = H.hspec_model_weights()
+    for i in range(2):
+        for f, _ in H.hspec_layer_weights._fields_:
+            setattr(mw.layers[i], f, 256)
+    h = H.hspec_drafter_create(cfg, mw)
+    si = H.hspec_step_in(C=1, K=8)
+    so = H.hspec_step_out()
+    st = H._lib.hspec_draft_step(h, ct.byref(si), ct.byref(so), 256, 1 << 30, None)
+    assert st == H.HSPEC_ERR_INVALID_ARG
+    si = H.hspec_step_in(C=1, K=8, h_last=256, x_in=256, ctx_lens=256)
+    si.kv[0] = H.hspec_kv_view(k_pool=256, v_pool=256, num_pages=4, page_table=256, max_pages=4)
+    st = H._lib.hspec_draft_step(h, ct.byref(si), ct.byref(so), 256, 16, None)
+    assert st == H.HSPEC_ERR_WORKSPACE
+    H.hspec_drafter_destroy(h)

@@ -1,0 +1,233 @@
+"""GPU parity of the three kernel-level C-ABI calls against the CPU oracle, on the
+seeded workloads (tiny fp32; Llama-3-8B shapes at 1 and 32 requests; Qwen-32B
+shapes at 128 requests, sampled), plus the invariants the method fixes: paged
+in-place reads equal any page placement, the split count does not matter, requests
+are independent, and bad page ids / context lengths are reported, not read.
+
+H-Spec (arXiv 2609.24197) Abstract: attention reuses target KVs in place; Mamba
+modules start from projected last-token hidden states; the parallel scan keeps the
+block parallel.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from hybrid_mamba_attention_b200 import inputs as I
+from tests.parity_util import assert_close, host, rel_max, sample_requests, sub_cache, to_np
+
+pytestmark = pytest.mark.gpu
+
+KERNEL_WORKLOADS = ["tiny", "llama_c1", "llama_c32", "qwen_c128"]
+
+
+@pytest.fixture(scope="module")
+def H(cuda):
+    from hybrid_mamba_attention_b200 import hspec
+    return hspec
+
+
+def cfg_for(H, sh, **kw):
+    return H.make_cfg(sh, **kw)
+
+
+# ------------------------------------------------------------------ inject
+
+@pytest.mark.parametrize("name", KERNEL_WORKLOADS)
+def test_inject_state_matches_oracle(H, cuda, name):
+    wl = I.WORKLOADS[name]
+    sh = wl.shapes
+    inp = I.make_inject_inputs(sh, wl.C, wl.seed, cuda)
+    h0 = torch.empty(wl.C, sh.H * sh.P * sh.N, device=cuda)
+    H.hspec_inject_state(cfg_for(H, sh), inp["W_inj"], inp["h_last"], h0)
+    assert H.hspec_sync_status() == 0
+    rows = sample_requests(wl.C, 2, seed=wl.seed)
+    ref = oracle.inject(host(inp["W_inj"]), host(inp["h_last"])[rows])
+    assert_close(to_np(h0[rows]), ref, "f32", f"inject {name}")
+
+
+@pytest.mark.parametrize("C,d,HPN", [(3, 200, 3 * 1000), (130, 64, 520), (1, 8, 8)])
+def test_inject_ragged_tiles(H, cuda, C, d, HPN):
+    # M, N and K all off the 128 / 256 / 64 tile grid (TMA zero-fills the edges)
+    sh = I.Shapes("ragged", d=d, Hq=1, Hkv=1, D=2, H=1, P=HPN, N=1, dtype="bf16", rope_theta=1e4)
+    g = torch.Generator(device=cuda).manual_seed(9)
+    W = torch.randn(HPN, d, device=cuda, generator=g).to(torch.bfloat16)
+    h = torch.randn(C, d, device=cuda, generator=g).to(torch.bfloat16)
+    h0 = torch.full((C, HPN), float("nan"), device=cuda)
+    H.hspec_inject_state(cfg_for(H, sh), W, h, h0)
+    assert H.hspec_sync_status() == 0
+    assert_close(to_np(h0), oracle.inject(host(W), host(h)), "f32", "inject ragged")
+
+
+# --------------------------------------------------------------------- SSD
+
+def run_ssd(H, sh, inp, K, chunk=0, want_state=False, h0=True):
+    C = inp["x"].shape[0]
+    y = torch.empty(C, K, sh.H, sh.P, device=inp["x"].device)
+    hK = torch.empty(C, sh.H, sh.P, sh.N, device=y.device) if want_state else None
+    H.hspec_ssd_block_scan(cfg_for(H, sh, ssd_chunk=chunk), inp["x"], inp["dt"], inp["A"], inp["B"], inp["Cm"],
+                           inp["D"], inp["h0"] if h0 else None, y, hK)
+    assert H.hspec_sync_status() == 0
+    return y, hK
+
+
+@pytest.mark.parametrize("name", KERNEL_WORKLOADS)
+def test_ssd_scan_matches_sequential_recurrence(H, cuda, name):
+    wl = I.WORKLOADS[name]
+    sh = wl.shapes
+    C = min(wl.C, 8)
+    inp = I.make_ssd_inputs(sh, C, wl.K, wl.seed, cuda)
+    y, hK = run_ssd(H, sh, inp, wl.K, want_state=True)
+    ref_y, ref_h = oracle.ssd_scan(host(inp["x"]), host(inp["dt"]), host(inp["A"]), host(inp["B"]),
+                                   host(inp["Cm"]), host(inp["D"]), host(inp["h0"]), want_state=True)
+    assert_close(to_np(y), ref_y, "f32", f"ssd y {name}")
+    assert_close(to_np(hK), ref_h, "f32", f"ssd hK {name}")
+
+
+@pytest.mark.parametrize("K,chunks", [(16, (1, 4, 5, 8, 16)), (32, (8, 16, 32)), (7, (3, 7)), (1, (1,))])
+def test_ssd_chunk_length_is_only_an_evaluation_order(H, cuda, K, chunks):
+    sh = I.LLAMA
+    inp = I.make_ssd_inputs(sh, 2, K, 11, cuda)
+    ref = oracle.ssd_scan(host(inp["x"]), host(inp["dt"]), host(inp["A"]), host(inp["B"]), host(inp["Cm"]),
+                          host(inp["D"]), host(inp["h0"]))
+    for q in chunks:
+        y, _ = run_ssd(H, sh, inp, K, chunk=q)
+        assert_close(to_np(y), ref, "f32", f"ssd K={K} chunk={q}")
+
+
+def test_ssd_zero_injection_equals_zero_state(H, cuda):
+    sh = I.TINY
+    inp = I.make_ssd_inputs(sh, 2, 8, 5, cuda)
+    inp["h0"].zero_()
+    a, _ = run_ssd(H, sh, inp, 8)
+    b, _ = run_ssd(H, sh, inp, 8, h0=False)
+    assert torch.equal(a, b)
+
+
+# --------------------------------------------------------------- attention
+
+def run_attn(H, sh, inp, K, split=0, causal=False):
+    from dataclasses import replace
+    sh2 = replace(sh, causal_block=causal)
+    cfg = cfg_for(H, sh2, attn_split_tokens=split)
+    C = inp["q"].shape[0]
+    kv = H.kv_view(inp)
+    ws = H.alloc_workspace(H.hspec_attn_workspace_size(cfg, C, K, kv.max_pages))
+    out = torch.full_like(inp["q"], float("nan"))
+    H.hspec_attn_paged_block(cfg, inp["q"], kv, inp["ctx_lens"], inp["k_blk"], inp["v_blk"], out, ws)
+    return out
+
+
+def oracle_attn(inp, rows, causal=False):
+    sc = sub_cache(inp, rows)
+    return oracle.attn_paged(host(inp["q"])[rows], sc["k_pool"], sc["v_pool"], sc["page_table"],
+                             host(inp["ctx_lens"])[rows], host(inp["k_blk"])[rows], host(inp["v_blk"])[rows],
+                             causal_block=causal)
+
+
+def compare_attn(gpu, ref, sh, what):
+    if sh.dtype == "bf16":
+        ref = oracle.bf16_round(ref)  # the C-ABI stores the attention output in bf16
+    return assert_close(gpu, ref, sh.dtype, what)
+
+
+@pytest.mark.parametrize("name", KERNEL_WORKLOADS)
+def test_paged_attention_matches_oracle(H, cuda, name):
+    wl = I.WORKLOADS[name]
+    sh = wl.shapes
+    inp = I.make_attn_inputs(sh, wl, wl.K, wl.seed, cuda, shuffle=wl.shuffle, slack=wl.slack)
+    out = run_attn(H, sh, inp, wl.K)
+    assert H.hspec_sync_status() == 0
+    rows = sample_requests(wl.C, 3, seed=wl.seed)
+    compare_attn(to_np(out[rows]), oracle_attn(inp, rows), sh, f"attn {name}")
+
+
+def test_paged_attention_causal_block(H, cuda):
+    wl = I.WORKLOADS["llama_c32"]
+    sh = wl.shapes
+    lens = torch.tensor([0, 5, 16, 17, 700, 1024], dtype=torch.int32)
+    inp = I.make_attn_inputs(sh, lens, 16, 3, cuda)
+    out = run_attn(H, sh, inp, 16, causal=True)
+    assert H.hspec_sync_status() == 0
+    rows = list(range(len(lens)))
+    compare_attn(to_np(out), oracle_attn(inp, rows, causal=True), sh, "attn causal")
+
+
+def test_page_placement_is_invisible(H, cuda):
+    # the same pages stored at other pool slots (table rewritten) give bit-identical output
+    wl = I.WORKLOADS["llama_c32"]
+    sh = wl.shapes
+    inp = I.make_attn_inputs(sh, wl, wl.K, 7, cuda)
+    n = inp["k_pool"].shape[0]
+    perm = torch.randperm(n, generator=torch.Generator().manual_seed(1)).to(cuda)
+    inv = torch.empty_like(perm)
+    inv[perm] = torch.arange(n, device=cuda)
+    tbl = inp["page_table"].clone()
+    m = tbl >= 0
+    tbl[m] = inv[tbl[m].long()].to(torch.int32)
+    moved = dict(inp, k_pool=inp["k_pool"][perm].contiguous(), v_pool=inp["v_pool"][perm].contiguous(),
+                 page_table=tbl)
+    a = run_attn(H, sh, inp, wl.K)
+    b = run_attn(H, sh, moved, wl.K)
+    assert H.hspec_sync_status() == 0
+    assert torch.equal(a, b)
+
+
+def test_split_count_does_not_change_the_result(H, cuda):
+    wl = I.WORKLOADS["llama_c32"]
+    sh = wl.shapes
+    inp = I.make_attn_inputs(sh, wl, wl.K, 8, cuda)
+    rows = sample_requests(wl.C, 3, seed=1)
+    ref = oracle_attn(inp, rows)
+    for split in (16, 64, 1024, 16384):
+        out = run_attn(H, sh, inp, wl.K, split=split)
+        assert H.hspec_sync_status() == 0
+        compare_attn(to_np(out[rows]), ref, sh, f"attn split {split}")
+
+
+def test_request_order_permutes_output(H, cuda):
+    wl = I.WORKLOADS["llama_c32"]
+    sh = wl.shapes
+    inp = I.make_attn_inputs(sh, wl, wl.K, 9, cuda)
+    perm = torch.randperm(wl.C, generator=torch.Generator().manual_seed(2)).to(cuda)
+    p = {k: (v[perm] if k in ("q", "k_blk", "v_blk", "page_table", "ctx_lens") else v) for k, v in inp.items()}
+    a = run_attn(H, sh, inp, wl.K)
+    b = run_attn(H, sh, p, wl.K)
+    assert H.hspec_sync_status() == 0
+    assert torch.equal(a[perm], b)
+
+
+def test_empty_context_single_token_returns_block_value(H, cuda):
+    sh = I.TINY
+    lens = torch.zeros(3, dtype=torch.int32)
+    inp = I.make_attn_inputs(sh, lens, 1, 4, cuda, slack=0.0)
+    out = run_attn(H, sh, inp, 1)
+    assert H.hspec_sync_status() == 0
+    G = sh.Hq // sh.Hkv
+    want = inp["v_blk"].repeat_interleave(G, dim=2)
+    assert rel_max(to_np(out), to_np(want)) <= 1e-6
+
+
+def test_nan_slack_pages_are_never_read(H, cuda):
+    wl = I.WORKLOADS["llama_c32"]
+    inp = I.make_attn_inputs(wl.shapes, wl, wl.K, 10, cuda, slack=0.5)
+    out = run_attn(H, wl.shapes, inp, wl.K)
+    assert H.hspec_sync_status() == 0
+    assert torch.isfinite(out.float()).all()
+
+
+def test_bad_page_id_is_reported_not_read(H, cuda):
+    wl = I.WORKLOADS["tiny"]
+    inp = I.make_attn_inputs(wl.shapes, wl, wl.K, 11, cuda, shuffle=False, slack=0.0)
+    inp["page_table"][0, 1] = inp["k_pool"].shape[0] + 5  # beyond the pool
+    run_attn(H, wl.shapes, inp, wl.K)
+    assert H.hspec_sync_status() == H.HSPEC_ERR_DEVICE_CHECK
+    assert H.hspec_sync_status() == 0  # the flag is cleared once reported
+
+
+def test_context_longer_than_page_table_is_reported(H, cuda):
+    wl = I.WORKLOADS["tiny"]
+    inp = I.make_attn_inputs(wl.shapes, wl, wl.K, 12, cuda, shuffle=False, slack=0.0)
+    inp["ctx_lens"][0] = inp["page_table"].shape[1] * wl.shapes.page + 1
+    run_attn(H, wl.shapes, inp, wl.K)
+    assert H.hspec_sync_status() == H.HSPEC_ERR_DEVICE_CHECK

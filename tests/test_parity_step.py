@@ -1,0 +1,183 @@
+"""GPU parity of the whole draft step (hspec_draft_step) against the CPU oracle on
+all five seeded workloads, the large ones on sampled requests (requests are
+independent).
+
+Two views:
+  stage-wise  every layer of the GPU step is compared with the oracle running that
+              same layer from the GPU's own input to it (the layer_hidden output of
+              the previous layer), at the bf16 bound (max-abs / rms <= 2e-2); the
+              final RMSNorm and the LM-head argmax likewise (tokens must agree
+              wherever the oracle's top-2 logit gap is >= 1e-3).
+  end to end  the GPU step vs the oracle step from the block input.  For the
+              two-layer workloads this meets the 2e-2 bound.  Through four bf16
+              layers with SwiGLU, one-ulp rounding differences at the bf16 storage
+              points cascade through the dense projections (fp32 vs fp64
+              accumulation decides a few roundings differently, each of which moves
+              whole rows at the next rounding point), so the end-to-end difference
+              is a drift that any fp32 implementation shows against an fp64
+              reference; it is asserted against DRIFT_BOUND and printed.
+
+H-Spec (arXiv 2609.24197) Abstract: block-parallel drafting with attention over the
+target KV in place and Mamba-2 layers started from the projected last-token hidden
+state; evolve.pub review, Summary: M,A hybrid backbone.
+"""
+from dataclasses import replace
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from hybrid_mamba_attention_b200 import inputs as I
+from tests.parity_util import (BF16_TOL, assert_close, host, host_weights, oracle_step_for, rel_rms,
+                               sample_requests, sub_cache, to_np)
+
+pytestmark = pytest.mark.gpu
+
+GAP = 1e-3
+DRIFT_BOUND = 6e-2  # end-to-end bound for the four-layer bf16 step (see module docstring)
+
+
+@pytest.fixture(scope="module")
+def H(cuda):
+    from hybrid_mamba_attention_b200 import hspec
+    return hspec
+
+
+def run_step(H, wl, st, ssd_chunk=0, split=0, layers=True):
+    sh = wl.shapes
+    dev = st["h_last"].device
+    dr = H.Drafter(sh, st["weights"], ssd_chunk=ssd_chunk, attn_split_tokens=split)
+    C, K = wl.C, wl.K
+    max_pages = max((c["page_table"].shape[1] for c in st["kv"]), default=1)
+    ws = H.alloc_workspace(dr.workspace_size(C, K, max_pages), dev)
+    si = dr.step_in(C, K, st["h_last"], st["ctx_lens"], st["kv"], tokens=st["tokens"], x_in=st["x_in"])
+    out = {"hidden": torch.full((C, K, sh.d), float("nan"), device=dev)}
+    so = H.hspec_step_out(hidden=out["hidden"].data_ptr())
+    if layers:
+        out["layer_hidden"] = torch.full((len(sh.layers), C, K, sh.d), float("nan"), device=dev)
+        so.layer_hidden = out["layer_hidden"].data_ptr()
+    if sh.vocab:
+        out["tokens"] = torch.full((C, K), -1, dtype=torch.int32, device=dev)
+        out["final_normed"] = torch.empty(C, K, sh.d, dtype=sh.torch_dtype, device=dev)
+        out["top"] = torch.empty(C, K, device=dev)
+        so.draft_tokens, so.final_normed = out["tokens"].data_ptr(), out["final_normed"].data_ptr()
+        so.top_logit = out["top"].data_ptr()
+    dr.step(si, so, ws)
+    assert H.hspec_sync_status() == 0, H.hspec_last_error()
+    dr.close()
+    return out
+
+
+def check_stagewise(wl, st, out, rows, wh):
+    """Each layer from the GPU's own input, then the final norm and the argmax."""
+    sh = wl.shapes
+    kv = [sub_cache(c, rows) for c in st["kv"]]
+    lh = out["layer_hidden"]
+    if sh.vocab:
+        x0 = host(st["weights"]["W_lm"])[host(st["tokens"])[rows].long()]
+    else:
+        x0 = host(st["x_in"])[rows]
+    errs, ai = [], 0
+    for li, kind in enumerate(sh.layers):
+        sh1 = replace(sh, layers=kind, vocab=0)
+        kv1 = [kv[ai]] if kind == "A" else []
+        ai += kind == "A"
+        xin = x0 if li == 0 else host(lh[li - 1])[rows]
+        ref = oracle.draft_step(sh1, {"layers": [wh["layers"][li]]}, kv1, host(st["h_last"])[rows],
+                                host(st["ctx_lens"])[rows], x_in=xin)
+        errs.append(assert_close(to_np(lh[li][rows]), ref["hidden"], sh.dtype, f"{wl.name} layer {li} ({kind})"))
+    if sh.vocab:
+        fn_ref = oracle.rmsnorm(to_np(lh[-1][rows]), wh["final_norm"], sh.eps)
+        fn_ref = oracle.bf16_round(fn_ref) if sh.dtype == "bf16" else fn_ref
+        assert_close(to_np(out["final_normed"][rows]), fn_ref, sh.dtype, f"{wl.name} final norm")
+        fn = out["final_normed"][rows]
+        am, t1, t2 = oracle.lm_head_argmax(host(fn).reshape(-1, sh.d), wh["W_lm"])
+        gpu_tok = host(out["tokens"][rows]).reshape(-1).numpy()
+        decided = (t1 - t2) >= GAP
+        assert decided.mean() > 0.5
+        assert np.array_equal(gpu_tok[decided], am[decided]), "draft tokens differ where the top-2 gap >= 1e-3"
+        np.testing.assert_allclose(host(out["top"][rows]).reshape(-1).numpy(), t1, rtol=1e-3, atol=1e-3)
+    return errs
+
+
+def check_end_to_end(wl, st, out, rows, wh, bound):
+    sh = wl.shapes
+    ref = oracle_step_for(sh, wh, st, rows)
+    e = rel_rms(to_np(out["hidden"][rows]), ref["hidden"])
+    msg = f"{wl.name}: end-to-end hidden max-abs/rms {e:.3e}"
+    if sh.vocab:
+        gpu_tok = host(out["tokens"][rows]).reshape(-1).numpy()
+        agree = float((gpu_tok == ref["draft_tokens"].reshape(-1)).mean())
+        msg += f", draft-token agreement {agree:.3f}"
+    print(msg)
+    assert np.isfinite(to_np(out["hidden"])).all()
+    assert e <= bound, msg
+    return e
+
+
+@pytest.mark.parametrize("name,n_sample", [("tiny", 1), ("llama_c1", 1), ("llama_c32", 2), ("qwen_c128", 2)])
+def test_draft_step_kernel_workloads(H, cuda, name, n_sample):
+    wl = I.WORKLOADS[name]
+    st = I.make_step_inputs(wl, cuda)
+    out = run_step(H, wl, st)
+    rows = sample_requests(wl.C, n_sample, seed=wl.seed)
+    wh = host_weights(st["weights"])
+    check_stagewise(wl, st, out, rows, wh)
+    bound = 1e-4 if wl.shapes.dtype == "f32" else BF16_TOL
+    if wl.shapes.dtype == "f32":
+        ref = oracle_step_for(wl.shapes, wh, st, rows)
+        assert_close(to_np(out["hidden"][rows]), ref["hidden"], "f32", f"{name} hidden")
+    else:
+        check_end_to_end(wl, st, out, rows, wh, bound)
+
+
+@pytest.mark.parametrize("C,K", [(8, 16), (128, 16), (1, 8), (32, 32)])
+def test_full_draft_step(H, cuda, C, K):
+    wl = I.full_workload(C, K)
+    st = I.make_step_inputs(wl, cuda)
+    out = run_step(H, wl, st)
+    rows = sample_requests(wl.C, 2, seed=wl.seed)
+    wh = host_weights(st["weights"])
+    check_stagewise(wl, st, out, rows, wh)
+    check_end_to_end(wl, st, out, rows, wh, DRIFT_BOUND)
+
+
+def test_step_ssd_chunking_and_split_do_not_change_the_result(H, cuda):
+    wl = I.WORKLOADS["llama_c32"]
+    st = I.make_step_inputs(wl, cuda)
+    a = run_step(H, wl, st, layers=False)
+    b = run_step(H, wl, st, ssd_chunk=4, split=128, layers=False)
+    assert_close(to_np(b["hidden"]), to_np(a["hidden"]), "bf16", "chunk/split variant")
+
+
+def test_step_request_permutation(H, cuda):
+    wl = I.full_workload(8, 16)
+    st = I.make_step_inputs(wl, cuda)
+    perm = torch.randperm(wl.C, generator=torch.Generator().manual_seed(3)).to(cuda)
+    st2 = dict(st, h_last=st["h_last"][perm], ctx_lens=st["ctx_lens"][perm], tokens=st["tokens"][perm],
+               kv=[dict(c, page_table=c["page_table"][perm]) for c in st["kv"]])
+    a = run_step(H, wl, st, layers=False)
+    b = run_step(H, wl, st2, layers=False)
+    assert torch.equal(a["hidden"][perm], b["hidden"])
+    assert torch.equal(a["tokens"][perm], b["tokens"])
+
+
+def test_step_counts_its_kernel_launches(H, cuda):
+    wl = I.WORKLOADS["tiny"]
+    st = I.make_step_inputs(wl, cuda)
+    n0 = H.hspec_launch_count()
+    run_step(H, wl, st, layers=False)
+    assert H.hspec_launch_count() - n0 >= 10
+
+
+def test_profile_groups_cover_the_step(H, cuda):
+    wl = I.full_workload(8, 16)
+    st = I.make_step_inputs(wl, cuda)
+    H.hspec_profile_enable(True)
+    run_step(H, wl, st, layers=False)
+    prof = H.hspec_profile_read()
+    H.hspec_profile_enable(False)
+    for name in ("in_proj", "inject", "ssd_scan", "attn_paged", "mlp_gate_up", "mlp_down", "lm_head_argmax"):
+        assert name in prof and prof[name][0] > 0
+    assert prof["attn_paged"][1] == 2 and prof["inject"][1] == 2
