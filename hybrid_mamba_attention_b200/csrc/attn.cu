@@ -1,8 +1,10 @@
 // Paged in-place GQA attention of the K block queries over the target's KV cache
 // followed by the block's own keys (H-Spec Abstract: "attention modules reuse target
 // KVs in place"), split-KV across CTAs, then a merge of the partial softmax states.
+// bf16 runs on the tensor cores (attn_tc.cu); this file holds the exact fp32 split
+// kernel, the merge shared by both, and the split policy.
 //
-// attn_split_kernel: one CTA per (split, kv head g, request c).  Its R = K*G query
+// attn_split_kernel (fp32): one CTA per (split, kv head g, request c).  Its R = K*G query
 // rows (block position j, query head g*G + i) share every key/value of kv head g,
 // so each 16-token tile of K and V is read from HBM once per CTA, translated through
 // the page table in place (token t of request c: page page_table[c][t / page],
@@ -26,7 +28,6 @@ constexpr int kTile = 16;
 
 template <typename T, int TPR>
 __global__ void __launch_bounds__(kThreads) attn_split_kernel(AttnArgs a, float scale_log2) {
-  constexpr int ROWS = kThreads / TPR;      // query rows one CTA can hold
   extern __shared__ float sm[];
   const int D = a.D, Dp = D + 1;
   float* sK = sm;                           // [kTile][D+1]
@@ -153,7 +154,8 @@ __global__ void attn_merge_kernel(AttnArgs a) {
     for (int e = lane; e < a.D; e += 32) out[e] = from_f<T>(0.f);
     return;
   }
-  const int ns = (ctx + a.K + a.split_tokens - 1) / a.split_tokens;
+  const int ns = a.block_in_last_split ? max(1, (ctx + a.split_tokens - 1) / a.split_tokens)
+                                      : (ctx + a.K + a.split_tokens - 1) / a.split_tokens;
   const size_t base0 = (((size_t)c * a.Hkv + g) * a.n_splits) * R + row;
   float M = -INFINITY;
   for (int s = 0; s < ns; ++s) M = fmaxf(M, a.ws_ml[(base0 + (size_t)s * R) * 2]);
@@ -182,7 +184,7 @@ void launch_split(const AttnArgs& a, cudaStream_t s) {
 }
 
 template <typename T>
-void launch_all(const AttnArgs& a, cudaStream_t s) {
+void launch_simt(const AttnArgs& a, cudaStream_t s) {
   const int R = a.K * (a.Hq / a.Hkv);
   int rows_cap = 1;
   while (rows_cap < R) rows_cap <<= 1;
@@ -195,6 +197,10 @@ void launch_all(const AttnArgs& a, cudaStream_t s) {
     case 2: launch_split<T, 2>(a, s); break;
     default: launch_split<T, 1>(a, s); break;
   }
+}
+
+template <typename T>
+void launch_merge(const AttnArgs& a, cudaStream_t s) {
   const long rows = (long)a.C * a.K * a.Hq;
   attn_merge_kernel<T><<<(int)((rows + 7) / 8), 256, 0, s>>>(a);
   note_launch();
@@ -202,20 +208,35 @@ void launch_all(const AttnArgs& a, cudaStream_t s) {
 
 }  // namespace
 
-bool attn_supported(int K, int G, int D) {
-  // one CTA holds all R = K*G query rows; a lane holds at most 128/TPR dims of q and acc
+bool attn_supported(int dtype, int K, int G, int D, const char** why) {
+  if (K < 1 || K > 64) return *why = "K must be in 1..64", false;
+  if (dtype == HSPEC_DTYPE_BF16) {
+    if (D != 64 && D != 128) return *why = "bf16 attention needs head_dim 64 or 128", false;
+    return true;
+  }
+  // fp32: one CTA holds all R = K*G query rows; a lane holds at most 128/TPR dims
   const int R = K * G;
   int cap = 1;
   while (cap < R) cap <<= 1;
-  if (cap > kThreads || D > 128 || D % 2) return false;
+  if (cap > kThreads || D > 128 || D % 2) return *why = "fp32 attention needs K*G <= 256 and head_dim <= 128", false;
   int tpr = kThreads / cap;
   if (tpr > 32) tpr = 32;
-  return D % tpr == 0;
+  if (D % tpr) return *why = "head_dim not divisible by lanes per row", false;
+  return true;
 }
 
-int attn_split_tokens(int C, int Hkv, int K, int max_ctx, int requested) {
+int attn_split_tokens(int dtype, int C, int Hkv, int K, int max_ctx, int requested) {
+  if (dtype == HSPEC_DTYPE_BF16) {
+    // tensor-core path: 64-token tiles; long splits amortise the partial write, but
+    // at least ~2 CTAs per SM over the grid
+    if (requested > 0) return ((requested + 63) / 64) * 64;
+    long per = ((long)C * Hkv * max_ctx + 2L * 148 - 1) / (2L * 148);
+    per = ((per + 63) / 64) * 64;
+    if (per < 128) per = 128;
+    if (per > 4096) per = 4096;
+    return (int)per;
+  }
   if (requested > 0) return requested;
-  // aim for ~16 CTAs per SM over the whole grid, in multiples of 64 tokens
   const long target_ctas = 148L * 16;
   long per = ((long)C * Hkv * (max_ctx + K) + target_ctas - 1) / target_ctas;
   per = ((per + 63) / 64) * 64;
@@ -223,14 +244,30 @@ int attn_split_tokens(int C, int Hkv, int K, int max_ctx, int requested) {
   return (int)per;
 }
 
+int attn_num_splits(int dtype, int K, int max_ctx, int split_tokens) {
+  if (dtype == HSPEC_DTYPE_BF16) return max(1, (max_ctx + split_tokens - 1) / split_tokens);
+  return (max_ctx + K + split_tokens - 1) / split_tokens;
+}
+
 size_t attn_ws_bytes(int C, int Hkv, int K, int G, int D, int n_splits) {
   const size_t rows = (size_t)C * Hkv * n_splits * K * G;
   return rows * D * sizeof(float) + rows * 2 * sizeof(float);
 }
 
-void attn_paged(int dtype, const AttnArgs& a, cudaStream_t s) {
-  if (dtype == HSPEC_DTYPE_BF16) launch_all<bf16>(a, s);
-  else launch_all<float>(a, s);
+bool attn_paged(int dtype, const AttnArgs& a, cudaStream_t s) {
+  if (dtype == HSPEC_DTYPE_BF16) {
+    const char* why = "";
+    if (!attn_tc_supported(a, &why)) {
+      set_error("paged attention: %s", why);
+      return false;
+    }
+    if (!attn_tc_launch(a, s)) return false;
+    launch_merge<bf16>(a, s);
+  } else {
+    launch_simt<float>(a, s);
+    launch_merge<float>(a, s);
+  }
+  return true;
 }
 
 }  // namespace hspec

@@ -178,8 +178,8 @@ struct AttnPlan {
 AttnPlan attn_plan(const hspec_cfg* c, int C, int K, int max_pages) {
   AttnPlan p;
   const int max_ctx = max_pages * c->page_size;
-  p.split_tokens = attn_split_tokens(C, c->n_kv_heads, K, max_ctx, c->attn_split_tokens);
-  p.n_splits = (max_ctx + K + p.split_tokens - 1) / p.split_tokens;
+  p.split_tokens = attn_split_tokens(c->dtype, C, c->n_kv_heads, K, max_ctx, c->attn_split_tokens);
+  p.n_splits = attn_num_splits(c->dtype, K, max_ctx, p.split_tokens);
   p.ws = align256(attn_ws_bytes(C, c->n_kv_heads, K, c->n_q_heads / c->n_kv_heads, c->head_dim, p.n_splits));
   return p;
 }
@@ -203,6 +203,7 @@ AttnArgs attn_args(const hspec_cfg* c, const AttnPlan& p, const hspec_kv_view* k
   a.split_tokens = p.split_tokens;
   a.n_splits = p.n_splits;
   a.causal_block = (c->flags & HSPEC_FLAG_CAUSAL_BLOCK) != 0;
+  a.block_in_last_split = c->dtype == HSPEC_DTYPE_BF16;
   const size_t rows = (size_t)C * a.Hkv * p.n_splits * K * (a.Hq / a.Hkv);
   a.ws_acc = (float*)ws;
   a.ws_ml = a.ws_acc + rows * a.D;
@@ -384,8 +385,8 @@ hspec_status hspec_attn_paged_block(const hspec_cfg* cfg, const void* q, const h
   if (!q || !ctx_lens || !k_blk || !v_blk || !out) FAIL(HSPEC_ERR_INVALID_ARG, "q, ctx_lens, k_blk, v_blk, out must be non-NULL");
   if (C < 1 || K < 1 || K > 64) FAIL(HSPEC_ERR_UNSUPPORTED, "C=%d K=%d (need C >= 1, 1 <= K <= 64)", C, K);
   const int G = cfg->n_q_heads / cfg->n_kv_heads;
-  if (!attn_supported(K, G, cfg->head_dim))
-    FAIL(HSPEC_ERR_UNSUPPORTED, "attention with K*G=%d rows and head_dim %d is not implemented", K * G, cfg->head_dim);
+  const char* why = "";
+  if (!attn_supported(cfg->dtype, K, G, cfg->head_dim, &why)) FAIL(HSPEC_ERR_UNSUPPORTED, "attention: %s", why);
   AttnPlan p = attn_plan(cfg, C, K, kv->max_pages);
   if (!workspace || ((uintptr_t)workspace & 255) || ws_bytes < p.ws)
     FAIL(HSPEC_ERR_WORKSPACE, "attention needs a 256-byte aligned workspace of %zu bytes (got %zu)", p.ws, ws_bytes);
@@ -395,7 +396,7 @@ hspec_status hspec_attn_paged_block(const hspec_cfg* cfg, const void* q, const h
   a.kb = k_blk, a.kb_rs = krow;
   a.vb = v_blk, a.vb_rs = krow;
   a.out = out, a.o_rs = qrow;
-  attn_paged(cfg->dtype, a, (cudaStream_t)stream);
+  if (!attn_paged(cfg->dtype, a, (cudaStream_t)stream)) return HSPEC_ERR_UNSUPPORTED;
   return check_launch("hspec_attn_paged_block");
 }
 
@@ -412,11 +413,10 @@ hspec_status hspec_drafter_create(const hspec_cfg* cfg, const hspec_model_weight
   if (st) return st;
   if (cfg->d_ff < 0 || cfg->vocab < 0) FAIL(HSPEC_ERR_INVALID_ARG, "d_ff and vocab must be >= 0");
   if (cfg->dtype == HSPEC_DTYPE_BF16) {
-    // tensor-core GEMM operands are streamed by TMA: K dims and row strides in multiples of 8
+    // tensor-core GEMM operands are streamed by TMA: every GEMM reduction dimension
+    // (= operand row stride) must be a multiple of 8 elements (16 bytes)
     const long HP = (long)cfg->n_ssm_heads * cfg->ssm_head_dim;
-    const long dims[] = {cfg->d_model, HP, 2 * HP + 2L * cfg->d_state + cfg->n_ssm_heads,
-                         (long)cfg->n_q_heads * cfg->head_dim,
-                         (long)(cfg->n_q_heads + 2 * cfg->n_kv_heads) * cfg->head_dim, cfg->d_ff};
+    const long dims[] = {cfg->d_model, HP, (long)cfg->n_q_heads * cfg->head_dim, cfg->d_ff};
     for (long v : dims)
       if (v % 8) FAIL(HSPEC_ERR_UNSUPPORTED, "bf16 drafter dims must be multiples of 8 (got %ld)", v);
   }
@@ -465,9 +465,9 @@ hspec_status hspec_draft_step(hspec_drafter* dr, const hspec_step_in* in, const 
   int max_pages = 1, n_att = 0;
   if (att) {
     if (!in->ctx_lens) FAIL(HSPEC_ERR_INVALID_ARG, "ctx_lens is NULL");
-    if (!attn_supported(K, c->n_q_heads / c->n_kv_heads, c->head_dim))
-      FAIL(HSPEC_ERR_UNSUPPORTED, "attention with K*G=%d rows and head_dim %d is not implemented",
-           K * (c->n_q_heads / c->n_kv_heads), c->head_dim);
+    const char* why = "";
+    if (!attn_supported(c->dtype, K, c->n_q_heads / c->n_kv_heads, c->head_dim, &why))
+      FAIL(HSPEC_ERR_UNSUPPORTED, "attention: %s", why);
     for (int i = 0; i < c->n_layers; ++i) {
       if (c->layer_kinds[i] != 'A') continue;
       if ((st = validate_kv(c, &in->kv[n_att]))) return st;
@@ -564,7 +564,7 @@ hspec_status hspec_draft_step(hspec_drafter* dr, const hspec_step_in* in, const 
       a.out = g, a.o_rs = (long)Hq * Dh;
       {
         ProfScope p("attn_paged", s);
-        attn_paged(dtype, a, s);
+        if (!attn_paged(dtype, a, s)) return HSPEC_ERR_UNSUPPORTED;
       }
       {
         ProfScope p("o_proj", s);

@@ -80,13 +80,19 @@ struct AttnArgs {
   int split_tokens;                      // tokens per split (multiple of 16)
   int n_splits;                          // splits per (request, kv head) upper bound
   bool causal_block;
+  bool block_in_last_split;              // tensor-core path: block keys ride with the last context split
   float* ws_acc; float* ws_ml;           // split partials
   int* err;
 };
-// Split policy and workspace bytes for the partials.
-int attn_split_tokens(int C, int Hkv, int K, int max_ctx, int requested);
+// Split policy (tokens per split, splits per request) and workspace bytes.
+int attn_split_tokens(int dtype, int C, int Hkv, int K, int max_ctx, int requested);
+int attn_num_splits(int dtype, int K, int max_ctx, int split_tokens);
 size_t attn_ws_bytes(int C, int Hkv, int K, int G, int D, int n_splits);
-bool attn_supported(int K, int G, int D);
-void attn_paged(int dtype, const AttnArgs& a, cudaStream_t s);
+bool attn_supported(int dtype, int K, int G, int D, const char** why);
+// Checks the pointer / stride requirements of the tensor-core path (bf16).
+bool attn_tc_supported(const AttnArgs& a, const char** why);
+bool attn_tc_launch(const AttnArgs& a, cudaStream_t s);
+// Split kernel + merge; false (message recorded) if it cannot launch.
+bool attn_paged(int dtype, const AttnArgs& a, cudaStream_t s);
 
 }  // namespace hspec

@@ -231,3 +231,50 @@ def test_context_longer_than_page_table_is_reported(H, cuda):
     inp["ctx_lens"][0] = inp["page_table"].shape[1] * wl.shapes.page + 1
     run_attn(H, wl.shapes, inp, wl.K)
     assert H.hspec_sync_status() == H.HSPEC_ERR_DEVICE_CHECK
+
+
+# ------------------------------------------- tensor-core attention edge shapes
+
+@pytest.mark.parametrize("K,lens", [(1, [0, 1, 15, 16, 63, 64, 65, 4097]), (3, [0, 7, 130, 2000]),
+                                    (16, [64, 128, 4096, 4100, 8191])])
+def test_bf16_attention_ragged_tiles(H, cuda, K, lens):
+    # contexts that end inside a page, on a page, on a 64-token tile and past a split
+    sh = I.LLAMA
+    lens_t = torch.tensor(lens, dtype=torch.int32)
+    inp = I.make_attn_inputs(sh, lens_t, K, 21, cuda)
+    out = run_attn(H, sh, inp, K)
+    assert H.hspec_sync_status() == 0
+    compare_attn(to_np(out), oracle_attn(inp, list(range(len(lens)))), sh, f"attn K={K}")
+
+
+def test_bf16_attention_more_than_128_query_rows(H, cuda):
+    # Qwen shapes with K=32: K*G = 256 query rows per kv head -> two row blocks
+    sh = I.QWEN
+    lens = torch.tensor([100, 3000], dtype=torch.int32)
+    inp = I.make_attn_inputs(sh, lens, 32, 22, cuda)
+    out = run_attn(H, sh, inp, 32)
+    assert H.hspec_sync_status() == 0
+    compare_attn(to_np(out), oracle_attn(inp, [0, 1]), sh, "attn 256 rows")
+
+
+def test_bf16_attention_head_dim_64(H, cuda):
+    sh = I.Shapes("d64", d=256, Hq=4, Hkv=2, D=64, H=4, P=64, N=16, dtype="bf16", rope_theta=1e4)
+    lens = torch.tensor([0, 33, 700], dtype=torch.int32)
+    inp = I.make_attn_inputs(sh, lens, 8, 23, cuda)
+    for causal in (False, True):
+        out = run_attn(H, sh, inp, 8, causal=causal)
+        assert H.hspec_sync_status() == 0
+        compare_attn(to_np(out), oracle_attn(inp, [0, 1, 2], causal=causal), sh, f"attn D=64 causal={causal}")
+
+
+def test_bf16_bad_page_id_is_reported(H, cuda):
+    wl = I.WORKLOADS["llama_c1"]
+    inp = I.make_attn_inputs(wl.shapes, wl, wl.K, 24, cuda)
+    inp["page_table"][0, 3] = -7
+    run_attn(H, wl.shapes, inp, wl.K)
+    assert H.hspec_sync_status() == H.HSPEC_ERR_DEVICE_CHECK
+    inp["page_table"][0, 3] = 0
+    inp["ctx_lens"][0] = inp["page_table"].shape[1] * wl.shapes.page + 16
+    run_attn(H, wl.shapes, inp, wl.K)
+    assert H.hspec_sync_status() == H.HSPEC_ERR_DEVICE_CHECK
+    assert H.hspec_sync_status() == 0
