@@ -40,6 +40,28 @@ def assert_close(gpu, ref, dtype: str, what: str = ""):
     return e
 
 
+def half_ulp_bf16(x):
+    """Half the spacing of bf16 numbers at |x| (the rounding a bf16 store may add)."""
+    a = np.abs(np.asarray(x, dtype=np.float64))
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -126)))
+    return 2.0 ** (e - 8)
+
+
+def assert_close_stored_bf16(gpu, ref, what: str = ""):
+    """A bf16-stored GPU output against the oracle's exact value: the kernel's own
+    error, max(|gpu - ref| - half_ulp_bf16(ref), 0) / rms(ref), must meet the bf16
+    bound; the raw max-abs / rms (which includes the store's rounding) is returned
+    alongside."""
+    g = np.asarray(gpu, dtype=np.float64)
+    r = np.asarray(ref, dtype=np.float64)
+    assert np.isfinite(g).all(), f"{what}: non-finite GPU output"
+    rms = max(np.sqrt((r ** 2).mean()), 1e-300)
+    raw = float(np.abs(g - r).max() / rms)
+    kern = float(np.maximum(np.abs(g - r) - half_ulp_bf16(r), 0.0).max() / rms)
+    assert kern <= BF16_TOL, f"{what}: bf16 kernel error {kern:.3e} (raw {raw:.3e}) > {BF16_TOL}"
+    return kern, raw
+
+
 def host(t):
     return t.detach().to("cpu")
 

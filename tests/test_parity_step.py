@@ -29,7 +29,7 @@ import torch
 
 import oracle
 from hybrid_mamba_attention_b200 import inputs as I
-from tests.parity_util import (BF16_TOL, assert_close, host, host_weights, oracle_step_for, rel_rms,
+from tests.parity_util import (BF16_TOL, assert_close, assert_close_stored_bf16, host, host_weights, oracle_step_for, rel_rms,
                                sample_requests, sub_cache, to_np)
 
 pytestmark = pytest.mark.gpu
@@ -89,8 +89,10 @@ def check_stagewise(wl, st, out, rows, wh):
         errs.append(assert_close(to_np(lh[li][rows]), ref["hidden"], sh.dtype, f"{wl.name} layer {li} ({kind})"))
     if sh.vocab:
         fn_ref = oracle.rmsnorm(to_np(lh[-1][rows]), wh["final_norm"], sh.eps)
-        fn_ref = oracle.bf16_round(fn_ref) if sh.dtype == "bf16" else fn_ref
-        assert_close(to_np(out["final_normed"][rows]), fn_ref, sh.dtype, f"{wl.name} final norm")
+        if sh.dtype == "bf16":
+            assert_close_stored_bf16(to_np(out["final_normed"][rows]), fn_ref, f"{wl.name} final norm")
+        else:
+            assert_close(to_np(out["final_normed"][rows]), fn_ref, sh.dtype, f"{wl.name} final norm")
         fn = out["final_normed"][rows]
         am, t1, t2 = oracle.lm_head_argmax(host(fn).reshape(-1, sh.d), wh["W_lm"])
         gpu_tok = host(out["tokens"][rows]).reshape(-1).numpy()
