@@ -371,6 +371,71 @@ hspec_status hspec_ssd_block_scan(const hspec_cfg* cfg, const void* x, const flo
   return check_launch("hspec_ssd_block_scan");
 }
 
+}  // extern "C"
+
+// Scratch of hspec_attn_paged_block_noalloc: a fixed device array, so that callers
+// that cannot allocate still get the split-KV partials somewhere.  Host code must not
+// pass the symbol itself to a kernel (on the host it names a shadow, not device
+// memory); the device address is looked up once per device below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[HSPEC_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+// Device address of g_noalloc_scratch on the current device; NULL (message recorded)
+// if the lookup fails.  The first call on a device does the lookup.
+void* noalloc_scratch_address() {
+  static std::mutex mu;
+  static void* addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    set_error("no current CUDA device");
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) {
+      set_error("cudaGetSymbolAddress(scratch) failed: %s", cudaGetErrorString(e));
+      return nullptr;
+    }
+    addr[dev] = p;
+  }
+  return addr[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+hspec_status hspec_attn_paged_block_noalloc(const hspec_cfg* cfg, const void* q, const hspec_kv_view* kv,
+                                            const int32_t* ctx_lens, const void* k_blk, const void* v_blk, int C,
+                                            int K, void* out, void* stream) {
+  hspec_status st = validate_cfg(cfg, true, false);
+  if (st) return st;
+  if ((st = validate_kv(cfg, kv))) return st;
+  if (!q || !ctx_lens || !k_blk || !v_blk || !out)
+    FAIL(HSPEC_ERR_INVALID_ARG, "q, ctx_lens, k_blk, v_blk, out must be non-NULL");
+  if (C < 1 || K < 1 || K > 64) FAIL(HSPEC_ERR_UNSUPPORTED, "C=%d K=%d (need C >= 1, 1 <= K <= 64)", C, K);
+  const int G = cfg->n_q_heads / cfg->n_kv_heads;
+  const char* why = "";
+  if (!attn_supported(cfg->dtype, K, G, cfg->head_dim, &why)) FAIL(HSPEC_ERR_UNSUPPORTED, "attention: %s", why);
+  AttnPlan p = attn_plan(cfg, C, K, kv->max_pages);
+  if (p.ws > HSPEC_NOALLOC_SCRATCH_BYTES)
+    FAIL(HSPEC_ERR_WORKSPACE, "allocation-free attention needs %zu bytes of split partials; its static scratch holds %zu",
+         p.ws, (size_t)HSPEC_NOALLOC_SCRATCH_BYTES);
+  void* scratch = noalloc_scratch_address();
+  if (!scratch) return HSPEC_ERR_CUDA;
+  AttnArgs a = attn_args(cfg, p, kv, ctx_lens, C, K, scratch);
+  const long qrow = (long)cfg->n_q_heads * cfg->head_dim, krow = (long)cfg->n_kv_heads * cfg->head_dim;
+  a.q = q, a.q_rs = qrow;
+  a.kb = k_blk, a.kb_rs = krow;
+  a.vb = v_blk, a.vb_rs = krow;
+  a.out = out, a.o_rs = qrow;
+  if (!attn_paged(cfg->dtype, a, (cudaStream_t)stream)) return HSPEC_ERR_UNSUPPORTED;
+  return check_launch("hspec_attn_paged_block_noalloc");
+}
+
 size_t hspec_attn_workspace_size(const hspec_cfg* cfg, int C, int K, int max_pages) {
   if (validate_cfg(cfg, true, false) || C < 1 || K < 1 || max_pages < 1) return 0;
   return attn_plan(cfg, C, K, max_pages).ws;

@@ -35,7 +35,8 @@ EXPORTS = ("hspec_inject_state", "hspec_ssd_block_scan", "hspec_attn_workspace_s
            "hspec_attn_paged_block", "hspec_drafter_create", "hspec_drafter_destroy",
            "hspec_step_workspace_size", "hspec_draft_step", "hspec_sync_status",
            "hspec_status_string", "hspec_last_error", "hspec_launch_count", "hspec_version",
-           "hspec_profile_enable", "hspec_profile_read")
+           "hspec_profile_enable", "hspec_profile_read", "hspec_attn_paged_block_noalloc")
+HSPEC_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 class HspecError(RuntimeError):
@@ -105,6 +106,7 @@ def _load():
         "hspec_version": (ct.c_char_p, []),
         "hspec_profile_enable": (I, [I]),
         "hspec_profile_read": (I, [P, P, P, I]),
+        "hspec_attn_paged_block_noalloc": (I, [cfgp, P, ct.POINTER(hspec_kv_view), P, P, P, I, I, P, V]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -191,6 +193,17 @@ def hspec_attn_paged_block(cfg: hspec_cfg, q, kv: hspec_kv_view, ctx_lens, k_blk
                                        _ptr(v_blk), C, K, _ptr(out), _ptr(workspace),
                                        workspace.numel() * workspace.element_size(), _stream(stream)),
            "hspec_attn_paged_block")
+
+
+def hspec_attn_paged_block_noalloc(cfg: hspec_cfg, q, kv: hspec_kv_view, ctx_lens, k_blk, v_blk, out,
+                                   stream=None):
+    """hspec_attn_paged_block without a workspace argument: the split partials live in
+    the library's static scratch (HSPEC_NOALLOC_SCRATCH_BYTES); for callers that
+    cannot allocate device memory.  Calls that overlap on the GPU race on it."""
+    C, K = int(q.shape[0]), int(q.shape[1])
+    _check(_lib.hspec_attn_paged_block_noalloc(ct.byref(cfg), _ptr(q), ct.byref(kv), _ptr(ctx_lens), _ptr(k_blk),
+                                               _ptr(v_blk), C, K, _ptr(out), _stream(stream)),
+           "hspec_attn_paged_block_noalloc")
 
 
 def hspec_drafter_create(cfg: hspec_cfg, weights: hspec_model_weights) -> ct.c_void_p:

@@ -168,6 +168,32 @@ HSPEC_API hspec_status hspec_attn_paged_block(const hspec_cfg* cfg, const void* 
                                     int C, int K, void* out, void* workspace, size_t ws_bytes,
                                     void* stream);
 
+/* Allocation-free variant of hspec_attn_paged_block.  The H-Spec paper has no
+ * counterpart to this entry point; it exists for deployment.  Some callers cannot allocate
+ * device memory when they call in: a serving engine that handed nearly all HBM to
+ * its KV-cache pool at start-up (a cudaMalloc could fail, or would break the
+ * engine's memory accounting), or a plain C host program that links only this
+ * library and has no device allocator of its own to provide a workspace.  This entry
+ * point takes the same inputs and output as hspec_attn_paged_block but keeps its
+ * split-KV partials in a static device array of HSPEC_NOALLOC_SCRATCH_BYTES bytes
+ * inside the library; every GPU that loads the library holds that array until the
+ * process exits.
+ *  - Calls whose partials need more than HSPEC_NOALLOC_SCRATCH_BYTES (that is,
+ *    hspec_attn_workspace_size(cfg, C, K, kv->max_pages) is larger) are rejected
+ *    with HSPEC_ERR_WORKSPACE before anything is launched.
+ *  - The first call on each device looks up the array's device address (a runtime
+ *    call, no allocation); make that first call before any CUDA stream capture.
+ *  - All calls share the one array, which keeps the previous call's contents.
+ *    Nothing in it has to start at zero: each call writes every partial it later
+ *    reads.  Calls that overlap on the GPU (different streams, or different host
+ *    threads on one device) race on the array; serialise them.
+ *  - Calls no cudaMalloc, cudaFree or other allocating routine. */
+#define HSPEC_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+HSPEC_API hspec_status hspec_attn_paged_block_noalloc(const hspec_cfg* cfg, const void* q,
+                                                      const hspec_kv_view* kv, const int32_t* ctx_lens,
+                                                      const void* k_blk, const void* v_blk, int C, int K,
+                                                      void* out, void* stream);
+
 /* ------------------------------------------------------------- draft step */
 
 typedef struct hspec_drafter hspec_drafter;
