@@ -356,6 +356,76 @@ def run_ours(args, rank, world, local):
         print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------- kernel-level mode
+
+def run_kernel(args, rank, world, local):
+    """Times one C-ABI call (attn / inject / ssd) on a kernel-level workload, with
+    CUDA events on the launching stream; inputs exceed L2 except the tiny workload."""
+    from hybrid_mamba_attention_b200 import hspec as H
+    from hybrid_mamba_attention_b200 import inputs as I
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    wl = I.WORKLOADS[args.workload]
+    sh, C, K = wl.shapes, wl.C, wl.K
+    cfg = H.make_cfg(sh)
+    E = 2 if sh.dtype == "bf16" else 4
+    if args.kernel == "attn":
+        inp = I.make_attn_inputs(sh, wl, K, wl.seed, dev, shuffle=wl.shuffle, slack=wl.slack)
+        kv = H.kv_view(inp)
+        ws = H.alloc_workspace(H.hspec_attn_workspace_size(cfg, C, K, kv.max_pages), dev)
+        out = torch.empty_like(inp["q"])
+        call = lambda: H.hspec_attn_paged_block(cfg, inp["q"], kv, inp["ctx_lens"], inp["k_blk"], inp["v_blk"], out, ws)
+        ctx = int(inp["ctx_lens"].sum())
+        work = {"bytes": float(ctx * sh.Hkv * sh.D * 2 * E + 2 * C * K * sh.Hq * sh.D * E),
+                "flops": 4.0 * sh.Hq * sh.D * K * (ctx + C * K)}
+        name = "attn_paged"
+    elif args.kernel == "inject":
+        inp = I.make_inject_inputs(sh, C, wl.seed, dev)
+        HPN = sh.H * sh.P * sh.N
+        h0 = torch.empty(C, HPN, device=dev)
+        call = lambda: H.hspec_inject_state(cfg, inp["W_inj"], inp["h_last"], h0)
+        work = {"bytes": float(HPN * sh.d * E + C * HPN * 4 + C * sh.d * E), "flops": 2.0 * C * HPN * sh.d}
+        name = "inject"
+    else:
+        inp = I.make_ssd_inputs(sh, C, K, wl.seed, dev)
+        y = torch.empty(C, K, sh.H, sh.P, device=dev)
+        call = lambda: H.hspec_ssd_block_scan(cfg, inp["x"], inp["dt"], inp["A"], inp["B"], inp["Cm"], inp["D"],
+                                              inp["h0"], y)
+        HPN = sh.H * sh.P * sh.N
+        work = {"bytes": float(C * HPN * 4 + C * K * (sh.H * sh.P + 2 * sh.N) * E + C * K * sh.H * 4
+                               + C * K * sh.H * sh.P * 4),
+                "flops": float(C * sh.H * (2 * K * sh.P * sh.N + K * K * (sh.N + sh.P)))}
+        name = "ssd_scan"
+    for _ in range(args.warmup):
+        call()
+    if H.hspec_sync_status() != 0:
+        raise RuntimeError(H.hspec_last_error())
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n0 = H.hspec_launch_count()
+    clocks = ClockSampler(local)
+    clocks.start()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if H.hspec_sync_status() != 0:
+        raise RuntimeError(H.hspec_last_error())
+    ms = e0.elapsed_time(e1) / args.steps
+    roof = roofline_of(name, work, ms, peaks, sustained=False)
+    line = {"metric": f"{name} call time", "value": round(ms * 1e3, 2), "unit": "us", "higher_is_better": False,
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "dtype": sh.dtype,
+            "config": {"workload": wl.description, "kernel": name, "C": C, "K": K},
+            "roofline": roof, "gpu_launches": H.hspec_launch_count() - n0, "clocks": clk,
+            "algorithmic_bytes": work["bytes"], "algorithmic_flops": work["flops"]}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 # ---------------------------------------------------------------- reference arm
 
 def run_reference(args, rank, world):
@@ -403,6 +473,9 @@ def main():
     ap.add_argument("--K", type=int, default=16)
     ap.add_argument("--sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel", choices=["step", "attn", "inject", "ssd"], default="step",
+                    help="time one C-ABI call on --workload instead of the full draft step")
+    ap.add_argument("--workload", default="llama_c32", help="kernel-level workload (tiny, llama_c1, llama_c32, qwen_c128)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -410,6 +483,8 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, rank, world)
+        elif args.kernel != "step":
+            run_kernel(args, rank, world, local)
         else:
             run_ours(args, rank, world, local)
     finally:

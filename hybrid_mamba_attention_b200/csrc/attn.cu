@@ -154,22 +154,37 @@ __global__ void attn_merge_kernel(AttnArgs a) {
     for (int e = lane; e < a.D; e += 32) out[e] = from_f<T>(0.f);
     return;
   }
-  const int ns = a.block_in_last_split ? max(1, (ctx + a.split_tokens - 1) / a.split_tokens)
-                                      : (ctx + a.K + a.split_tokens - 1) / a.split_tokens;
-  const size_t base0 = (((size_t)c * a.Hkv + g) * a.n_splits) * R + row;
+  const int ns = (a.block_in_last_split ? max(1, (ctx + a.split_tokens - 1) / a.split_tokens)
+                                       : (ctx + a.K + a.split_tokens - 1) / a.split_tokens) * a.sub_splits;
+  const size_t base0 = (((size_t)c * a.Hkv + g) * a.n_splits * a.sub_splits) * R + row;
+  // Partial q exists when its split has keys for it: on the tensor-core path half h of
+  // split s holds the split's tiles of parity h, so it exists iff the split has more
+  // than h tiles (the rest of the workspace is never written and never read); a
+  // partial with l = 0 saw no key and is skipped.
+  const int n_units = ns / a.sub_splits;
+  auto has = [&](int q) -> bool {
+    if (!a.block_in_last_split) return true;
+    const int sp = q / a.sub_splits, h = q % a.sub_splits;
+    const int b = sp * a.split_tokens, e = min(ctx, b + a.split_tokens);
+    const int tiles = (e > b ? (e - b + kAttnTcTile - 1) / kAttnTcTile : 0) + (sp == n_units - 1 ? 1 : 0);
+    return tiles > h;
+  };
   float M = -INFINITY;
-  for (int s = 0; s < ns; ++s) M = fmaxf(M, a.ws_ml[(base0 + (size_t)s * R) * 2]);
+  for (int q = 0; q < ns; ++q) {
+    const float* ml = a.ws_ml + (base0 + (size_t)q * R) * 2;
+    if (has(q) && ml[1] > 0.f) M = fmaxf(M, ml[0]);
+  }
   float L = 0.f;
-  for (int s = 0; s < ns; ++s) {
-    const float ms = a.ws_ml[(base0 + (size_t)s * R) * 2];
-    if (ms != -INFINITY) L += exp2f(ms - M) * a.ws_ml[(base0 + (size_t)s * R) * 2 + 1];
+  for (int q = 0; q < ns; ++q) {
+    const float* ml = a.ws_ml + (base0 + (size_t)q * R) * 2;
+    if (has(q) && ml[1] > 0.f) L += exp2f(ml[0] - M) * ml[1];
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
   for (int e = lane; e < a.D; e += 32) {
     float o = 0.f;
-    for (int s = 0; s < ns; ++s) {
-      const float ms = a.ws_ml[(base0 + (size_t)s * R) * 2];
-      if (ms != -INFINITY) o = fmaf(exp2f(ms - M), a.ws_acc[(base0 + (size_t)s * R) * a.D + e], o);
+    for (int q = 0; q < ns; ++q) {
+      const float* ml = a.ws_ml + (base0 + (size_t)q * R) * 2;
+      if (has(q) && ml[1] > 0.f) o = fmaf(exp2f(ml[0] - M), a.ws_acc[(base0 + (size_t)q * R) * a.D + e], o);
     }
     out[e] = from_f<T>(o * inv);
   }
@@ -229,11 +244,14 @@ int attn_split_tokens(int dtype, int C, int Hkv, int K, int max_ctx, int request
   if (dtype == HSPEC_DTYPE_BF16) {
     // tensor-core path: 64-token tiles; long splits amortise the partial write, but
     // at least ~2 CTAs per SM over the grid
+    // the persistent kernel balances items dynamically: splits only need to spread
+    // long requests over several SMs (about 4 items per SM), and long splits keep the
+    // partial traffic (two halves of R x D fp32 per split) small against the K/V read
     if (requested > 0) return ((requested + 63) / 64) * 64;
-    long per = ((long)C * Hkv * max_ctx + 2L * 148 - 1) / (2L * 148);
+    long per = ((long)C * Hkv * max_ctx + 4L * 148 - 1) / (4L * 148);
     per = ((per + 63) / 64) * 64;
-    if (per < 128) per = 128;
-    if (per > 4096) per = 4096;
+    if (per < 256) per = 256;
+    if (per > 8192) per = 8192;
     return (int)per;
   }
   if (requested > 0) return requested;
@@ -249,9 +267,12 @@ int attn_num_splits(int dtype, int K, int max_ctx, int split_tokens) {
   return (max_ctx + K + split_tokens - 1) / split_tokens;
 }
 
-size_t attn_ws_bytes(int C, int Hkv, int K, int G, int D, int n_splits) {
-  const size_t rows = (size_t)C * Hkv * n_splits * K * G;
-  return rows * D * sizeof(float) + rows * 2 * sizeof(float);
+int attn_sub_splits(int dtype) { return dtype == HSPEC_DTYPE_BF16 ? 2 : 1; }
+
+size_t attn_ws_bytes(int C, int Hkv, int K, int G, int D, int n_splits, int sub_splits) {
+  const size_t rows = (size_t)C * Hkv * n_splits * sub_splits * K * G;
+  // + work counter and unit count, + unit list of the tensor-core path
+  return rows * D * sizeof(float) + rows * 2 * sizeof(float) + 256 + (size_t)C * n_splits * 2 * sizeof(int);
 }
 
 bool attn_paged(int dtype, const AttnArgs& a, cudaStream_t s) {

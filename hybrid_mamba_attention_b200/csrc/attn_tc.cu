@@ -3,26 +3,39 @@
 // the target KVs in place -- here the K/V pages are streamed by TMA straight out of
 // the target's pool through the page table, never copied to a drafter-side cache.
 //
-// One CTA per (context split, kv head g, request c [, row block]).  The R = K*G
-// queries of kv head g (block position j, query head g*G + i) form the rows of a
-// 128-row Q tile (rows >= R are zero), so every K/V byte read from HBM feeds all R
-// queries.  Warp roles (192 threads):
-//   warp 0      TMA producer: per 64-token tile, one 3-D box of 16 tokens x 64 dims
-//               of head g per page and column block (128-byte swizzle), K and V into
-//               a 4-stage ring; the block's own K keys come as one extra tile from
-//               the projection output, loaded by the last context split.
-//   warp 1      TMEM owner and single-thread MMA issuer:
-//                 S_b  = Q . K_i^T        (M=128, N=64, K=D; S double-buffered in TMEM)
-//                 O   += P_b . V_i        (M=128, N=D, K=64; V as an MN-major operand)
-//   warps 2..5  softmax, one TMEM lane (query row) per thread: mask, running max in
-//               the exp2 domain, P = exp2(s - m) written to shared memory as bf16;
-//               O is rescaled in TMEM only when the running max grows by more than
-//               8 (2^8 headroom keeps P exact enough in bf16); zeroes V rows past the
-//               end of the context in a partial tile; finally writes the split's
-//               partial (m, l, unnormalised O) for the merge kernel.
-// Synchronisation is by mbarriers (one per ring slot / per double buffer, so that no
-// waiter can fall two phases behind); every wait gives up after a time bound and
-// sets the device error word.
+// Work units are (request, context split) pairs; a unit expands into one item per
+// (row block, kv head g).  A one-CTA schedule kernel lists the units longest first
+// (counting sort on the unit's tile count), so that the short units are the last
+// ones taken and the SMs finish together.  The persistent kernel (one CTA per SM)
+// takes items from an atomic counter, the heads of one unit adjacent so that
+// concurrent CTAs read the same pages.  The R = K*G queries of kv head g (block
+// position j, query head g*G + i) form the rows of a 128-row Q tile, so every K/V
+// byte read from HBM feeds all R queries; with R <= 64 the rows are spread 16 per
+// 32-lane TMEM quarter so that all four SM sub-partitions share the softmax work;
+// rows without a query are zero.
+// Warp roles (320 threads):
+//   warp 0      producer: takes the next item, loads its Q tile (TMA) into one of
+//               two Q buffers, reads page ids two tiles ahead, and streams its
+//               64-token K/V tiles through a 4-stage ring -- per tile one 3-D TMA box
+//               of 16 tokens x 64 dims of head g per page and column block (128-byte
+//               swizzle), all boxes of a tile issued at once, one lane each -- and
+//               writes the tile's description next to it.  The last context split
+//               of a request also streams the block's own keys as one more tile.
+//   warp 1      TMEM owner and single-thread MMA issuer, driven by readiness rather
+//               than by a fixed order: it issues O_w += P_w . V_i (M=128, N=D, K=64)
+//               as soon as the P of tile i is in shared memory, and S_b = Q . K_i^T
+//               (M=128, N=64, K=D) into S buffer b = i % 4 as soon as tile i has
+//               landed and softmax has read S_b's previous tile, so that the S of a
+//               group's next tile is ready while it still works on the current one.
+//   warps 2..5  softmax warpgroup 0 (tiles i even), warps 6..9 warpgroup 1 (i odd):
+//               one TMEM lane (query row) per thread; mask, running max in the exp2
+//               domain, P = exp2(s - m) to shared memory as bf16; O_w is rescaled in
+//               TMEM only when the running max grows by more than 8.  Each group
+//               keeps its own (m, l, O) per item and writes its own partial when its
+//               last tile of the item is done -- the half of the split made of the
+//               item's even (or odd) tiles, so the arithmetic does not depend on
+//               scheduling; the merge kernel combines the halves and the splits.
+// Every wait gives up after a time bound and sets the device error word.
 #include <stdint.h>
 
 #include "../../include/hspec.h"
@@ -36,65 +49,133 @@ int* device_error_word();
 
 namespace {
 
-constexpr int TT = 64;        // tokens per tile
-constexpr int NS = 4;         // K/V ring stages
-constexpr int THREADS = 192;
+constexpr int TT = kAttnTcTile;  // tokens per tile
+constexpr int NS = 5;         // K/V ring stages
+constexpr int THREADS = 320;
 constexpr int ROWS = 128;     // MMA M
+constexpr int NSB = 4;        // S buffers in TMEM, two per softmax warpgroup
+constexpr int kLenBuckets = 256;  // schedule: units sorted by tile count (capped)
+
+struct TileMeta {  // written by the producer before the stage's barrier arrive
+  int c, g, split, rb;
+  int valid;       // keys in the tile
+  int local;       // tile index within the item
+  int n_tiles;     // tiles of the item
+  int block;       // 1: the block's own keys
+  int qslot, qseq; // Q buffer of the item and the item's use count of that buffer
+  int end;         // 1: no more work
+  int pad;
+};
 
 template <int D>
 struct Lay {
   static constexpr int DB = D / 64;                     // 64-element column blocks
   static constexpr int Q_BLK = ROWS * 128;              // 16 KB per Q column block
-  static constexpr int KV_BLK = TT * 128;               // 8 KB per K (or V) column block
-  static constexpr int K_BYTES = DB * KV_BLK;
+  static constexpr int Q_BYTES = DB * Q_BLK;
+  static constexpr int KV_BLK = TT * 128;               // 8 KB per K column block
+  static constexpr int K_BYTES = DB * KV_BLK;           // K: [column block][64 tokens][128 B]
+  static constexpr int V_PAGE = DB * 2048;              // V: [page][column block][16 tokens][128 B]
   static constexpr int STAGE = 2 * K_BYTES;             // K then V
-  static constexpr int P_BYTES = ROWS * TT * 2;         // 16 KB
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_KV = DB * Q_BLK;
-  static constexpr int OFF_P = OFF_KV + NS * STAGE;
-  static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
+  static constexpr int OFF_Q = 0;                       // two Q buffers
+  static constexpr int OFF_KV = 2 * Q_BYTES;
+  static constexpr int OFF_META = OFF_KV + NS * STAGE;
+  static constexpr int OFF_BAR = OFF_META + 64 * NS;
   static constexpr int SMEM = OFF_BAR + 256 + 1024;
-  static constexpr uint32_t TMEM_COLS = 256;            // S0 [0,64) S1 [64,128) O [128,128+D)
+  // TMEM columns: S_b [64b, 64b+64) for b < 4 (P of the tile, bf16 packed, overwrites
+  // its first 32 columns), O_w [256 + 128w, 256 + 128w + D)
+  static constexpr uint32_t TMEM_COLS = 512;
+  __host__ __device__ static constexpr uint32_t S_COL(int b) { return (uint32_t)(b * 64); }
+  __host__ __device__ static constexpr uint32_t O_COL(int w) { return (uint32_t)(256 + w * 128); }
 };
 
 struct TcMaps {
-  CUtensorMap k, v, kb, vb;
+  CUtensorMap k, v, kb, vb, q;
 };
+
+// TMEM lane (0..127) -> query row of the row block: identity for R > 64; for
+// R <= 64, 16 rows per 32-lane quarter (lanes 0..15 of each quarter), else -1.
+__device__ __forceinline__ int row_of_lane(int lane128, bool spread) {
+  if (!spread) return lane128;
+  const int q = lane128 >> 5, l = lane128 & 31;
+  return l < 16 ? q * 16 + l : -1;
+}
+
+// Tiles (64-token tiles, plus the block tile in a request's last split) of unit
+// (ctx, split sp of n).
+__host__ __device__ inline int unit_tiles(int ctx, int sp, int n, int split_tokens) {
+  const int b = sp * split_tokens, e = min(ctx, b + split_tokens);
+  return (e > b ? (e - b + TT - 1) / TT : 0) + (sp == n - 1 ? 1 : 0);
+}
+
+// One CTA: lists the (request, split) units longest first into `units` and resets the
+// work counter; sched[1] = number of units.  Requests with an invalid context length
+// get no unit (their output rows are written as zeros by the merge).
+__global__ void __launch_bounds__(1024) attn_sched_kernel(const int32_t* ctx_lens, int C, int split_tokens,
+                                                          long max_ctx, int* sched, int2* units, int* err) {
+  __shared__ int hist[kLenBuckets];
+  for (int b = threadIdx.x; b < kLenBuckets; b += blockDim.x) hist[b] = 0;
+  __syncthreads();
+  for (int c = threadIdx.x; c < C; c += blockDim.x) {
+    const int ctx = ctx_lens[c];
+    if (ctx < 0 || ctx > max_ctx) {
+      flag_error(err, kErrCtxOOB);
+      continue;
+    }
+    const int n = ctx > 0 ? (ctx + split_tokens - 1) / split_tokens : 1;
+    for (int sp = 0; sp < n; ++sp) atomicAdd(&hist[min(unit_tiles(ctx, sp, n, split_tokens), kLenBuckets - 1)], 1);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int b = kLenBuckets - 1; b >= 0; --b) {
+      const int h = hist[b];
+      hist[b] = run;
+      run += h;
+    }
+    sched[0] = 0;
+    sched[1] = run;
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < C; c += blockDim.x) {
+    const int ctx = ctx_lens[c];
+    if (ctx < 0 || ctx > max_ctx) continue;
+    const int n = ctx > 0 ? (ctx + split_tokens - 1) / split_tokens : 1;
+    for (int sp = 0; sp < n; ++sp) {
+      const int pos = atomicAdd(&hist[min(unit_tiles(ctx, sp, n, split_tokens), kLenBuckets - 1)], 1);
+      units[pos] = make_int2(c, sp);
+    }
+  }
+}
 
 template <int D>
 __global__ void __launch_bounds__(THREADS, 1)
-    attn_tc_kernel(const __grid_constant__ TcMaps maps, AttnArgs a, float scale_log2, int n_rb) {
+    attn_tc_kernel(const __grid_constant__ TcMaps maps, AttnArgs a, float scale_log2, int n_rb, int* sched,
+                   const int2* units) {
   using L = Lay<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = tc::smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023) & ~1023u) - raw);
   uint8_t* sQ = smem + L::OFF_Q;
   uint8_t* sKV = smem + L::OFF_KV;
-  uint8_t* sP = smem + L::OFF_P;
+  volatile TileMeta* meta = (volatile TileMeta*)(smem + L::OFF_META);
   uint64_t* kv_full = (uint64_t*)(smem + L::OFF_BAR);
   uint64_t* kv_empty = kv_full + NS;
-  uint64_t* s_full = kv_empty + NS;
-  uint64_t* p_full = s_full + 2;
-  uint64_t* pv_done = p_full + 2;
-  uint64_t* q_ready = pv_done + 2;
-  uint32_t* tmem_slot = (uint32_t*)(q_ready + 1);
+  uint64_t* s_full = kv_empty + NS;   // [NSB] S_b written by Q.K^T
+  uint64_t* s_free = s_full + NSB;    // [NSB] P.V of S_b's tile finished (S_b / P free)
+  // P of S_b's tile written (one barrier per S buffer: a group's next tile may finish
+  // its softmax before the MMA thread has taken this one, and the phases of one
+  // barrier must not run two ahead of its waiter)
+  uint64_t* p_full = s_free + NSB;    // [NSB]
+  uint64_t* pv_done = p_full + NSB;   // [2]   group w's P.V finished (O_w quiescent)
+  uint64_t* q_full = pv_done + 2;     // [2]
+  uint64_t* q_empty = q_full + 2;     // [2]
+  uint64_t* drain = q_empty + 2;      // every MMA (and its barrier arrivals) finished
+  uint32_t* tmem_slot = (uint32_t*)(drain + 1);
+  volatile int* end_tile = (volatile int*)(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int split = blockIdx.x, g = blockIdx.y;
-  const int c = blockIdx.z / n_rb, rb = blockIdx.z % n_rb;
   const int G = a.Hq / a.Hkv, R = a.K * G;
-  const int ctx = a.ctx_lens[c];
-  if (ctx < 0 || ctx > a.max_pages * a.page_size) {
-    if (threadIdx.x == 0 && split == 0 && rb == 0) flag_error(a.err, kErrCtxOOB);
-    return;
-  }
-  const int n_ctx_splits = (ctx + a.split_tokens - 1) / a.split_tokens;
-  const int last_split = n_ctx_splits > 0 ? n_ctx_splits - 1 : 0;
-  if (split > last_split) return;  // CTA-uniform: nothing of this request here
-  const int c_begin = split * a.split_tokens;
-  const int c_end = min(ctx, c_begin + a.split_tokens);
-  const int n_ctx_tiles = c_end > c_begin ? (c_end - c_begin + TT - 1) / TT : 0;
-  const int n_tiles = n_ctx_tiles + (split == last_split ? 1 : 0);
+  const bool spread = R <= 64;
   int* err = a.err;
 
   if (threadIdx.x == 0) {
@@ -102,58 +183,148 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc::mbar_init(&kv_full[s], 1);
       tc::mbar_init(&kv_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NSB; ++b) {
       tc::mbar_init(&s_full[b], 1);
+      tc::mbar_init(&s_free[b], 1);
       tc::mbar_init(&p_full[b], 4);
-      tc::mbar_init(&pv_done[b], 1);
     }
-    tc::mbar_init(q_ready, 4);
+    for (int w = 0; w < 2; ++w) {
+      tc::mbar_init(&pv_done[w], 1);
+      tc::mbar_init(&q_full[w], 1);
+      tc::mbar_init(&q_empty[w], 1);
+    }
+    tc::mbar_init(drain, 1);
+    *end_tile = 0x7fffffff;
     tc::fence_mbar_init();
   }
   if (warp == 1) tc::tmem_alloc(tmem_slot, L::TMEM_COLS);
+  // Q rows without a query are never written by TMA: zero both Q buffers once
+  for (int e = threadIdx.x; e < 2 * L::Q_BYTES / 16; e += THREADS) ((uint4*)sQ)[e] = make_uint4(0, 0, 0, 0);
+  tc::fence_proxy_async();
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tO = tmem + 128;
 
   if (warp == 0) {
+    // ------------------------------------------------------------ producer
     if (lane == 0) {
-      // ---------------------------------------------------------- TMA producer
       tc::tma_prefetch_desc(&maps.k);
       tc::tma_prefetch_desc(&maps.v);
       tc::tma_prefetch_desc(&maps.kb);
       tc::tma_prefetch_desc(&maps.vb);
+      tc::tma_prefetch_desc(&maps.q);
+    }
+    // Q boxes: with spread rows, one per 32-lane quarter holding 16 / G block positions
+    // (16 rows); otherwise one holding 128 / G positions (128 rows)
+    const int q_boxes = spread ? (R + 15) / 16 : 1;
+    const int q_pos = spread ? 16 / G : ROWS / G;
+    const int per_unit = a.Hkv * n_rb;
+    const int n_items = sched[1] * per_unit;
+    int tile_i = 0;
+    bool ok = true;
+    int it_next = lane == 0 ? atomicAdd(sched, 1) : 0;  // the following item's index, in flight
+    for (int seq = 0; ok; ++seq) {
+      int item = lane == 0 ? it_next : 0;
+      item = __shfl_sync(0xffffffffu, item, 0);
+      if (item >= n_items) break;
+      if (lane == 0) it_next = atomicAdd(sched, 1);  // prefetch: used by the next item
+      const int u = item / per_unit, g = item % a.Hkv, rb = (item % per_unit) / a.Hkv;
+      const int2 cu = units[u];
+      const int c = cu.x, split = cu.y;
+      const int ctx = a.ctx_lens[c];
+      const int n_ctx_splits = ctx > 0 ? (ctx + a.split_tokens - 1) / a.split_tokens : 1;
+      const int c_begin = split * a.split_tokens;
+      const int c_end = min(ctx, c_begin + a.split_tokens);
+      const int n_ctx_tiles = c_end > c_begin ? (c_end - c_begin + TT - 1) / TT : 0;
+      const int n_tiles = n_ctx_tiles + (split == n_ctx_splits - 1 ? 1 : 0);
+      const int slot = seq & 1;
+
+      // Q tile of the item into Q buffer `slot` once the item two back is done with it
+      if (lane == 0) ok = tc::mbar_wait(&q_empty[slot], ((seq >> 1) & 1) ^ 1, err);
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      uint8_t* qbuf = sQ + slot * L::Q_BYTES;
+      if (lane == 0) tc::mbar_arrive_expect_tx(&q_full[slot], (uint32_t)(q_boxes * L::DB * q_pos * G * 128));
+      __syncwarp();
+      if (lane < q_boxes * L::DB) {
+        const int qb = lane / L::DB, bk = lane % L::DB;
+        const int pos0 = c * a.K + (spread ? qb * q_pos : rb * q_pos);
+        tc::tma_load_3d(qbuf + bk * L::Q_BLK + qb * 32 * 128, &maps.q, &q_full[slot], bk * 64, g * G, pos0);
+      }
+      __syncwarp();
+
+      // Page ids: lane L holds the id of page q16 = L % 4 of the tile (a 64-token tile
+      // spans four 16-token pages) for the current tile and the next two.  K boxes are
+      // issued by lanes 0 .. 4 DB - 1 (column block L / 4), V boxes by lanes 16..19.
+      // The table reads are unconditional (the index is clamped into the request's
+      // row of the table) and their values are used two tiles later, so nothing waits
+      // for them; ids of tokens past the split's end are never used.
       const int32_t* table = a.page_table + (size_t)c * a.max_pages;
-      for (int i = 0; i < n_tiles; ++i) {
-        const int s = i % NS;
-        if (!tc::mbar_wait(&kv_empty[s], ((i / NS) & 1) ^ 1, err)) break;
+      const int q16 = lane & 3, lj = lane >> 2;
+      const bool k_lane = lj < L::DB, v_lane = lj == 4;
+      auto page_of = [&](int local) -> int {
+        const int idx = (c_begin + local * TT + 16 * q16) / a.page_size;
+        return table[idx < a.max_pages ? idx : a.max_pages - 1];
+      };
+      int pid0 = page_of(0), pid1 = page_of(1);
+
+      for (int local = 0; local < n_tiles && ok; ++local, ++tile_i) {
+        const int pid = pid0;
+        pid0 = pid1;
+        pid1 = page_of(local + 2);
+        const int s = tile_i % NS;
+        if (lane == 0) ok = tc::mbar_wait(&kv_empty[s], ((tile_i / NS) & 1) ^ 1, err);
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
         uint8_t* kd = sKV + s * L::STAGE;
         uint8_t* vd = kd + L::K_BYTES;
-        if (i < n_ctx_tiles) {
-          const int t0 = c_begin + i * TT;
-          const int groups = (min(TT, c_end - t0) + 15) / 16;
-          tc::mbar_arrive_expect_tx(&kv_full[s], (uint32_t)(groups * L::DB * 2048 * 2));
-          for (int q16 = 0; q16 < groups; ++q16) {
+        const bool block = local >= n_ctx_tiles;
+        const int t0 = c_begin + local * TT;
+        const int valid = block ? a.K : min(TT, c_end - t0);
+        if (lane == 0) {
+          volatile TileMeta& m = meta[s];
+          m.c = c, m.g = g, m.split = split, m.rb = rb, m.valid = valid, m.local = local;
+          m.n_tiles = n_tiles, m.block = block ? 1 : 0, m.qslot = slot, m.qseq = seq, m.end = 0;
+        }
+        if (!block) {
+          const int groups = (valid + 15) / 16;
+          if (lane == 0) tc::mbar_arrive_expect_tx(&kv_full[s], (uint32_t)(groups * L::DB * 2048 * 2));
+          __syncwarp();
+          if ((k_lane || v_lane) && q16 < groups) {
             const int t = t0 + 16 * q16;
-            int pg = table[t / a.page_size];
+            int pg = pid;
             if (pg < 0 || pg >= a.num_pages) {
               flag_error(err, kErrPageOOB);
               pg = 0;  // keep the copy in bounds; the request's output is flagged as invalid
             }
             const int z = pg * a.page_size + t % a.page_size;
-            for (int bk = 0; bk < L::DB; ++bk) {
+            if (k_lane) {
+              const int bk = lj;
               tc::tma_load_3d(kd + bk * L::KV_BLK + q16 * 2048, &maps.k, &kv_full[s], bk * 64, g, z);
-              tc::tma_load_3d(vd + bk * L::KV_BLK + q16 * 2048, &maps.v, &kv_full[s], bk * 64, g, z);
+            } else {
+              tc::tma_load_4d(vd + q16 * L::V_PAGE, &maps.v, &kv_full[s], 0, z, g, 0);
             }
           }
         } else {
-          tc::mbar_arrive_expect_tx(&kv_full[s], (uint32_t)(L::DB * L::KV_BLK * 2));
-          for (int bk = 0; bk < L::DB; ++bk) {
-            tc::tma_load_3d(kd + bk * L::KV_BLK, &maps.kb, &kv_full[s], bk * 64, g, c * a.K);
-            tc::tma_load_3d(vd + bk * L::KV_BLK, &maps.vb, &kv_full[s], bk * 64, g, c * a.K);
+          const int nq = (a.K + 15) / 16;
+          if (lane == 0) tc::mbar_arrive_expect_tx(&kv_full[s], (uint32_t)(L::DB * L::KV_BLK + nq * L::V_PAGE));
+          __syncwarp();
+          if (lane < L::DB) {
+            tc::tma_load_3d(kd + lane * L::KV_BLK, &maps.kb, &kv_full[s], lane * 64, g, c * a.K);
+          } else if (lane >= 16 && lane < 16 + nq) {
+            tc::tma_load_4d(vd + (lane - 16) * L::V_PAGE, &maps.vb, &kv_full[s], 0, c * a.K + 16 * (lane - 16), g, 0);
           }
         }
+        __syncwarp();
+      }
+    }
+    // sentinel stage: no more work
+    if (ok && lane == 0) {
+      const int s = tile_i % NS;
+      if (tc::mbar_wait(&kv_empty[s], ((tile_i / NS) & 1) ^ 1, err)) {
+        meta[s].end = 1;
+        tc::mbar_arrive(&kv_full[s]);
       }
     }
   } else if (warp == 1) {
@@ -161,163 +332,209 @@ __global__ void __launch_bounds__(THREADS, 1)
       // ---------------------------------------------------------- MMA issuer
       constexpr uint32_t idesc_qk = tc::idesc_bf16_f32(ROWS, TT);
       constexpr uint32_t idesc_pv = tc::idesc_bf16_f32(ROWS, D) | (1u << 16);  // B (= V) MN-major
-      bool ok = tc::mbar_wait(q_ready, 0, err);
-      auto issue_qk = [&](int i) -> bool {
-        const int s = i % NS;
-        if (!tc::mbar_wait(&kv_full[s], (i / NS) & 1, err)) return false;
-        tc::tc_fence_after();
-        const uint32_t q = tc::smem_u32(sQ), k = tc::smem_u32(sKV + s * L::STAGE);
-        const uint32_t dS = tmem + (uint32_t)((i & 1) * TT);
+      int q_seen[2] = {-1, -1};
+      int qk = 0, pv = 0, end_at = 0x7fffffff;
+      bool ok = true;
+      uint64_t idle_since = 0;
+      while (pv < end_at) {
+        bool progress = false;
+        // P.V of the oldest tile whose P is in shared memory
+        if (pv < qk && tc::mbar_test_wait(&p_full[pv & (NSB - 1)], (pv / NSB) & 1)) {
+          tc::tc_fence_after();
+          const int w = pv & 1, s = pv % NS;
+          const bool first = meta[s].local < 2;  // this group's first tile of the item
+          const uint32_t pt = tmem + L::S_COL(pv & (NSB - 1));  // P of the tile, in its S buffer
+          const uint32_t v = tc::smem_u32(sKV + s * L::STAGE + L::K_BYTES);
+          // K slice kk = the 16 keys of page kk: V [column block][16 tokens] blocks 2 KB apart
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          tc::mma_bf16(dS, tc::sdesc_k128(q + (kk / 4) * L::Q_BLK + (kk % 4) * 32),
-                       tc::sdesc_k128(k + (kk / 4) * L::KV_BLK + (kk % 4) * 32), idesc_qk, kk > 0);
-        tc::mma_commit(&s_full[i & 1]);
-        return true;
-      };
-      if (ok) ok = issue_qk(0);
-      if (ok && n_tiles > 1) ok = issue_qk(1);
-      for (int i = 0; i < n_tiles && ok; ++i) {
-        const int b = i & 1, s = i % NS;
-        if (!(ok = tc::mbar_wait(&p_full[b], (i >> 1) & 1, err))) break;
-        tc::tc_fence_after();
-        const uint32_t p = tc::smem_u32(sP + b * L::P_BYTES);
-        const uint32_t v = tc::smem_u32(sKV + s * L::STAGE + L::K_BYTES);
+          for (int kk = 0; kk < TT / 16; ++kk)
+            tc::mma_bf16_ts(tmem + L::O_COL(w), pt + kk * 8, tc::sdesc_mn128(v + kk * L::V_PAGE, 2048), idesc_pv,
+                            (kk > 0 || !first) ? 1u : 0u);
+          tc::mma_commit(&kv_empty[s]);
+          tc::mma_commit(&pv_done[w]);
+          tc::mma_commit(&s_free[pv & (NSB - 1)]);  // P read: S buffer free for tile pv + 4
+          ++pv;
+          progress = true;
+        }
+        // Q.K^T of the next tile once it has landed, its S buffer is free (the P.V of the
+        // tile four back has read its P) and its Q is loaded
+        if (qk < end_at) {
+          const int s = qk % NS, b = qk & (NSB - 1);
+          if ((qk < NSB || tc::mbar_test_wait(&s_free[b], ((qk / NSB) - 1) & 1)) &&
+              tc::mbar_test_wait(&kv_full[s], (qk / NS) & 1)) {
+            if (meta[s].end) {
+              end_at = qk;
+              progress = true;
+            } else {
+              const int slot = meta[s].qslot, seq = meta[s].qseq;
+              if (seq <= q_seen[slot] || tc::mbar_test_wait(&q_full[slot], (seq >> 1) & 1)) {
+                q_seen[slot] = seq > q_seen[slot] ? seq : q_seen[slot];
+                tc::tc_fence_after();
+                const uint32_t q = tc::smem_u32(sQ + slot * L::Q_BYTES), k = tc::smem_u32(sKV + s * L::STAGE);
 #pragma unroll
-        for (int kk = 0; kk < TT / 16; ++kk)
-          tc::mma_bf16(tO, tc::sdesc_k128(p + kk * 32), tc::sdesc_mn128(v + kk * 2048, L::KV_BLK), idesc_pv,
-                       (i | kk) != 0);
-        tc::mma_commit(&kv_empty[s]);
-        tc::mma_commit(&pv_done[b]);
-        if (i + 2 < n_tiles) ok = issue_qk(i + 2);
+                for (int kk = 0; kk < D / 16; ++kk)
+                  tc::mma_bf16(tmem + L::S_COL(b), tc::sdesc_k128(q + (kk / 4) * L::Q_BLK + (kk % 4) * 32),
+                               tc::sdesc_k128(k + (kk / 4) * L::KV_BLK + (kk % 4) * 32), idesc_qk, kk > 0);
+                tc::mma_commit(&s_full[b]);
+                if (meta[s].local == meta[s].n_tiles - 1) tc::mma_commit(&q_empty[slot]);  // item's last QK
+                ++qk;
+                progress = true;
+              }
+            }
+          }
+        }
+        if (progress) {
+          idle_since = 0;
+        } else {
+          const uint64_t t = tc::global_ns();
+          if (idle_since == 0) {
+            idle_since = t;
+          } else if (t - idle_since > tc::kWaitLimitNs) {
+            flag_error(err, tc::kErrTimeout);
+            ok = false;
+            break;
+          }
+        }
       }
+      if (ok) {
+        // wake both softmax groups: their next tiles are end_at and end_at + 1
+        *end_tile = end_at;
+        tc::mbar_arrive(&s_full[end_at & (NSB - 1)]);
+        tc::mbar_arrive(&s_full[(end_at + 1) & (NSB - 1)]);
+      }
+      // no MMA or commit arrival may land after the CTA has finished
+      tc::mma_commit(drain);
+      tc::mbar_wait(drain, 0, err);
     }
   } else {
-    // ------------------------------------------------------------ softmax warps
-    const int quarter = warp & 3;
-    const int row = quarter * 32 + lane;
-    const int gr = rb * ROWS + row;
-    const bool active = gr < R;
-    const int jq = active ? gr / G : 0;
-    const int hq = g * G + (active ? gr % G : 0);
+    // ------------------------------------------------------------ softmax warpgroups
+    const int wg = (warp - 2) >> 2;         // 0: warps 2..5, 1: warps 6..9
+    const int quarter = warp & 3;           // TMEM lanes this warp may access
+    const int lane128 = quarter * 32 + lane;
+    const int r_local = row_of_lane(lane128, spread);
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-
-    // Q row -> shared memory (128-byte swizzle, K-major)
-    {
-      const bf16* qrow = (const bf16*)a.q + (size_t)(c * a.K + jq) * a.q_rs + (size_t)hq * D;
-#pragma unroll
-      for (int ch = 0; ch < D / 8; ++ch) {
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (active) v = *(const uint4*)(qrow + ch * 8);
-        *(uint4*)(sQ + (ch / 8) * L::Q_BLK + row * 128 + (((ch % 8) ^ (row & 7)) << 4)) = v;
-      }
-      tc::fence_proxy_async();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(q_ready);
-    }
+    const uint32_t tOw = tmem + lane_off + L::O_COL(wg);
 
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int i = 0; i < n_tiles && ok; ++i) {
-      const int b = i & 1;
-      ok = __all_sync(0xffffffffu, tc::mbar_wait(&s_full[b], (i >> 1) & 1, err));
-      if (!ok) break;
+    for (int i = wg; ok; i += 2) {
+      const int n = i >> 1;                 // this group's tile count so far
+      const int b = i & (NSB - 1);
+      ok = __all_sync(0xffffffffu, tc::mbar_wait(&s_full[b], (i / NSB) & 1, err));
+      if (!ok || i >= *end_tile) break;
       tc::tc_fence_after();
-      const bool block_tile = i >= n_ctx_tiles;
-      const int valid = block_tile ? a.K : min(TT, c_end - (c_begin + i * TT));
-      float s[TT];
-      {
-        float* s0 = s;
-        float(&h0)[32] = *reinterpret_cast<float(*)[32]>(s0);
-        float(&h1)[32] = *reinterpret_cast<float(*)[32]>(s0 + 32);
-        tc::tmem_ld32(tmem + lane_off + (uint32_t)(b * TT), h0);
-        tc::tmem_ld32(tmem + lane_off + (uint32_t)(b * TT + 32), h1);
+      const int s = i % NS;
+      // acquire the producer's description of the tile (this phase completed long ago;
+      // the stage cannot move on before this group's P.V of the tile)
+      ok = __all_sync(0xffffffffu, tc::mbar_wait(&kv_full[s], (i / NS) & 1, err));
+      if (!ok) break;
+      const int c = meta[s].c, g = meta[s].g, split = meta[s].split, rb = meta[s].rb;
+      const int local = meta[s].local, n_tiles = meta[s].n_tiles, valid = meta[s].valid;
+      const bool block_tile = meta[s].block != 0;
+      const int gr = rb * ROWS + (r_local < 0 ? 0 : r_local);
+      const bool active = r_local >= 0 && gr < R;
+      const int jq = active ? gr / G : 0;
+      if (local < 2) {  // this group's first tile of a new item
+        m_used = -INFINITY;
+        l = 0.f;
       }
+      float sv[TT];
+      tc::tmem_ld64(tmem + lane_off + L::S_COL(b), sv);
       float mx = -INFINITY;
+      if (valid == TT && !(block_tile && a.causal_block)) {
 #pragma unroll
-      for (int j = 0; j < TT; ++j) {
-        bool vis = j < valid;
-        if (block_tile && a.causal_block && j > jq) vis = false;
-        s[j] = vis ? s[j] * scale_log2 : -INFINITY;
-        mx = fmaxf(mx, s[j]);
+        for (int j = 0; j < TT; ++j) {
+          sv[j] *= scale_log2;
+          mx = fmaxf(mx, sv[j]);
+        }
+      } else {
+        const int vis_end = (block_tile && a.causal_block) ? min(valid, jq + 1) : valid;
+#pragma unroll
+        for (int j = 0; j < TT; ++j) {
+          sv[j] = j < vis_end ? sv[j] * scale_log2 : -INFINITY;
+          mx = fmaxf(mx, sv[j]);
+        }
       }
       const float m_new = fmaxf(m_used, mx);
+      float alpha = 1.f;
+      bool rescale = false;
       if (m_new > m_used + 8.f) {
-        if (i > 0 && m_used != -INFINITY) {
-          // O holds earlier tiles: wait for the last P.V, then rescale it in TMEM
-          ok = __all_sync(0xffffffffu, tc::mbar_wait(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, err));
-          if (!ok) break;
-          tc::tc_fence_after();
-          const float alpha = exp2f(m_used - m_new);
-#pragma unroll
-          for (int cb = 0; cb < D / 32; ++cb) {
-            float v[32];
-            tc::tmem_ld32(tO + lane_off + cb * 32, v);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] *= alpha;
-            tc::tmem_st32(tO + lane_off + cb * 32, v);
-          }
+        if (local >= 2 && m_used != -INFINITY) {
+          alpha = exp2f(m_used - m_new);
+          rescale = true;
           l *= alpha;
         }
         m_used = m_new;
       }
+      // with no visible key yet (m = -inf) every s is -inf: subtract 0 so p = 0, not NaN
+      const float mu = m_used == -INFINITY ? 0.f : m_used;
       float psum = 0.f;
       uint32_t pk[TT / 2];
 #pragma unroll
       for (int j = 0; j < TT; j += 2) {
-        const float p0 = (s[j] == -INFINITY) ? 0.f : exp2f(s[j] - m_used);
-        const float p1 = (s[j + 1] == -INFINITY) ? 0.f : exp2f(s[j + 1] - m_used);
+        const float p0 = exp2f(sv[j] - mu);  // exp2(-inf) = 0 for masked columns
+        const float p1 = exp2f(sv[j + 1] - mu);
         psum += p0 + p1;
         __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
         pk[j / 2] = *reinterpret_cast<uint32_t*>(&h2);
       }
       l += psum;
-      if (i >= 2) {  // P buffer b was read by the P.V of tile i-2
-        ok = __all_sync(0xffffffffu, tc::mbar_wait(&pv_done[b], ((i - 2) >> 1) & 1, err));
+      tc::tmem_st32u(tmem + lane_off + L::S_COL(b), pk);  // P over the first half of S_b
+      if (__any_sync(0xffffffffu, rescale)) {
+        // O_w holds this group's earlier tiles of the item; their P.V must be done
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(&pv_done[wg], (n - 1) & 1, err));
         if (!ok) break;
-      }
-      uint8_t* prow = sP + b * L::P_BYTES + row * 128;
+        tc::tc_fence_after();
 #pragma unroll
-      for (int cc = 0; cc < 8; ++cc)
-        *(uint4*)(prow + ((cc ^ (row & 7)) << 4)) = make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
-      if (valid < TT) {
-        // V rows past the last valid token may hold stale data: zero them (P is 0 there)
-        uint8_t* vbase = sKV + (i % NS) * L::STAGE + L::K_BYTES;
-        const int n_chunks = (TT - valid) * L::DB * 8;
-        for (int e = threadIdx.x - 64; e < n_chunks; e += 128) {
-          const int r2 = valid + e / (L::DB * 8), rest = e % (L::DB * 8);
-          const int bk = rest / 8, cc = rest % 8;
-          *(uint4*)(vbase + bk * L::KV_BLK + r2 * 128 + ((cc ^ (r2 & 7)) << 4)) = make_uint4(0, 0, 0, 0);
+        for (int cb = 0; cb < D / 32; ++cb) {
+          float v[32];
+          tc::tmem_ld32(tOw + cb * 32, v);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] *= alpha;
+          tc::tmem_st32(tOw + cb * 32, v);
         }
       }
-      tc::fence_proxy_async();
+      if (valid < TT) {
+        // V rows past the last valid token may hold stale data: zero them (P is 0 there)
+        uint8_t* vbase = sKV + s * L::STAGE + L::K_BYTES;
+        const int n_chunks = (TT - valid) * L::DB * 8;
+        for (int e = (warp - 2 - 4 * wg) * 32 + lane; e < n_chunks; e += 128) {
+          const int r2 = valid + e / (L::DB * 8), rest = e % (L::DB * 8);
+          const int bk = rest / 8, cc = rest % 8, rr = r2 & 15;
+          *(uint4*)(vbase + (r2 >> 4) * L::V_PAGE + bk * 2048 + rr * 128 + ((cc ^ (rr & 7)) << 4)) =
+              make_uint4(0, 0, 0, 0);
+        }
+        tc::fence_proxy_async();
+      }
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&p_full[b]);
-    }
 
-    // epilogue: the split's partial state for the merge kernel
-    if (ok && n_tiles > 0) {
-      const int last = n_tiles - 1;
-      ok = __all_sync(0xffffffffu, tc::mbar_wait(&pv_done[last & 1], (last >> 1) & 1, err));
-      tc::tc_fence_after();
-      const size_t base = (((size_t)c * a.Hkv + g) * a.n_splits + split) * R + gr;
+      if (local >= n_tiles - 2) {
+        // this group's last tile of the item: write its partial (half of the split)
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(&pv_done[wg], n & 1, err));
+        if (!ok) break;
+        tc::tc_fence_after();
+        // half (local & 1): the item's even or odd tiles, whichever group ran them,
+        // so the result does not depend on how items were scheduled
+        const size_t base = ((((size_t)c * a.Hkv + g) * a.n_splits + split) * 2 + (local & 1)) * R + gr;
 #pragma unroll
-      for (int cb = 0; cb < D / 32; ++cb) {
-        float v[32];
-        tc::tmem_ld32(tO + lane_off + cb * 32, v);
-        if (ok && active) {
-          float* o = a.ws_acc + base * D + cb * 32;
+        for (int cb = 0; cb < D / 32; ++cb) {
+          float v[32];
+          tc::tmem_ld32(tOw + cb * 32, v);
+          if (active) {
+            float* o = a.ws_acc + base * D + cb * 32;
 #pragma unroll
-          for (int e = 0; e < 32; e += 4) *(float4*)(o + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+            for (int e = 0; e < 32; e += 4) *(float4*)(o + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+          }
         }
-      }
-      if (ok && active) {
-        a.ws_ml[base * 2] = m_used;
-        a.ws_ml[base * 2 + 1] = l;
+        if (active) {
+          a.ws_ml[base * 2] = m_used;
+          a.ws_ml[base * 2 + 1] = l;
+        }
+        tc::tc_fence_before();
       }
     }
-    tc::tc_fence_before();
   }
   __syncthreads();
   if (warp == 1) {
@@ -361,9 +578,39 @@ bool make_kv_map(CUtensorMap* m, const void* base, long rows, int Hkv, int D, lo
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 4-D map of [rows][Hkv][D] seen as (x = 64 elements, y = token row, z = kv head,
+// w = 64-element column block, 128 B apart) with box 64 x 16 x 1 x D/64: one box
+// holds 16 token rows of one head in both column blocks, stored [column block][row].
+bool make_kv_map4(CUtensorMap* m, const void* base, long rows, int Hkv, int D, long row_stride_elems) {
+  EncodeTiledFn fn = encode_fn_attn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {64, (cuuint64_t)rows, (cuuint64_t)Hkv, (cuuint64_t)(D / 64)};
+  cuuint64_t strides[3] = {(cuuint64_t)row_stride_elems * 2, (cuuint64_t)D * 2, 128};
+  cuuint32_t box[4] = {64, 16, 1, (cuuint32_t)(D / 64)};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D map of q [positions][Hq][D] with box 64 x G x pos_rows, 128-byte swizzle.
+bool make_q_map(CUtensorMap* m, const void* base, long positions, int Hq, int D, long row_stride_elems, int G,
+                int pos_rows) {
+  EncodeTiledFn fn = encode_fn_attn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hq, (cuuint64_t)positions};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)row_stride_elems * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)G, (cuuint32_t)pos_rows};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int D>
 bool launch_tc(const AttnArgs& a, cudaStream_t s) {
   static bool attr_set[64] = {};
+  static int n_sm[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
@@ -372,22 +619,41 @@ bool launch_tc(const AttnArgs& a, cudaStream_t s) {
       set_error("cudaFuncSetAttribute(attn_tc_kernel) failed");
       return false;
     }
+    cudaDeviceGetAttribute(&n_sm[dev], cudaDevAttrMultiProcessorCount, dev);
     attr_set[dev] = true;
   }
   TcMaps maps;
   const long pool_rows = (long)a.num_pages * a.page_size;
   bool ok = make_kv_map(&maps.k, a.k_pool, pool_rows, a.Hkv, D, (long)a.Hkv * D, 16) &&
-            make_kv_map(&maps.v, a.v_pool, pool_rows, a.Hkv, D, (long)a.Hkv * D, 16) &&
+            make_kv_map4(&maps.v, a.v_pool, pool_rows, a.Hkv, D, (long)a.Hkv * D) &&
             make_kv_map(&maps.kb, a.kb, (long)a.C * a.K, a.Hkv, D, a.kb_rs, TT) &&
-            make_kv_map(&maps.vb, a.vb, (long)a.C * a.K, a.Hkv, D, a.vb_rs, TT);
+            make_kv_map4(&maps.vb, a.vb, (long)a.C * a.K, a.Hkv, D, a.vb_rs);
+  // Q as [C*K positions][Hq heads][D]: a box holds G heads x (16 / G or 128 / G) positions
+  const int G = a.Hq / a.Hkv;
+  const int Rq = a.K * G;
+  ok = ok && make_q_map(&maps.q, a.q, (long)a.C * a.K, a.Hq, D, a.q_rs, G, Rq <= 64 ? 16 / G : ROWS / G);
   if (!ok) {
     set_error("cuTensorMapEncodeTiled failed for the attention K/V maps");
     return false;
   }
   const int R = a.K * (a.Hq / a.Hkv);
   const int n_rb = (R + ROWS - 1) / ROWS;
+  if (a.sub_splits != 2) {
+    set_error("tensor-core attention writes two partials per split");
+    return false;
+  }
+  // after the partials: the work counter and unit count (256 bytes), then the unit list
+  const size_t pairs = (size_t)a.C * a.Hkv * a.n_splits * 2 * R;
+  int* sched = (int*)(a.ws_ml + pairs * 2);
+  int2* units = (int2*)(sched + 64);
+  attn_sched_kernel<<<1, 1024, 0, s>>>(a.ctx_lens, a.C, a.split_tokens, (long)a.max_pages * a.page_size, sched,
+                                       units, a.err);
+  note_launch();
+  const long max_items = (long)a.C * a.n_splits * n_rb * a.Hkv;
+  const int sms = dev < 64 && n_sm[dev] > 0 ? n_sm[dev] : 148;
+  const int grid = max_items < sms ? (int)max_items : sms;
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
-  attn_tc_kernel<D><<<dim3(a.n_splits, a.Hkv, a.C * n_rb), THREADS, Lay<D>::SMEM, s>>>(maps, a, scale_log2, n_rb);
+  attn_tc_kernel<D><<<grid, THREADS, Lay<D>::SMEM, s>>>(maps, a, scale_log2, n_rb, sched, units);
   note_launch();
   return true;
 }
@@ -398,6 +664,8 @@ bool attn_tc_supported(const AttnArgs& a, const char** why) {
   if (a.D != 64 && a.D != 128) return *why = "head_dim must be 64 or 128", false;
   if (a.page_size % 16) return *why = "page_size must be a multiple of 16", false;
   if (a.K > 64) return *why = "K must be <= 64", false;
+  const int G = a.Hq / a.Hkv;
+  if (G > 16 || (G & (G - 1))) return *why = "the GQA group Hq/Hkv must be a power of two <= 16", false;
   if ((a.q_rs % 8) || (a.kb_rs % 8) || (a.vb_rs % 8))
     return *why = "q / k_blk / v_blk row strides must be multiples of 8 elements", false;
   const uintptr_t any = (uintptr_t)a.q | (uintptr_t)a.kb | (uintptr_t)a.vb | (uintptr_t)a.k_pool | (uintptr_t)a.v_pool;

@@ -180,7 +180,8 @@ AttnPlan attn_plan(const hspec_cfg* c, int C, int K, int max_pages) {
   const int max_ctx = max_pages * c->page_size;
   p.split_tokens = attn_split_tokens(c->dtype, C, c->n_kv_heads, K, max_ctx, c->attn_split_tokens);
   p.n_splits = attn_num_splits(c->dtype, K, max_ctx, p.split_tokens);
-  p.ws = align256(attn_ws_bytes(C, c->n_kv_heads, K, c->n_q_heads / c->n_kv_heads, c->head_dim, p.n_splits));
+  p.ws = align256(attn_ws_bytes(C, c->n_kv_heads, K, c->n_q_heads / c->n_kv_heads, c->head_dim, p.n_splits,
+                                attn_sub_splits(c->dtype)));
   return p;
 }
 
@@ -204,7 +205,8 @@ AttnArgs attn_args(const hspec_cfg* c, const AttnPlan& p, const hspec_kv_view* k
   a.n_splits = p.n_splits;
   a.causal_block = (c->flags & HSPEC_FLAG_CAUSAL_BLOCK) != 0;
   a.block_in_last_split = c->dtype == HSPEC_DTYPE_BF16;
-  const size_t rows = (size_t)C * a.Hkv * p.n_splits * K * (a.Hq / a.Hkv);
+  a.sub_splits = attn_sub_splits(c->dtype);
+  const size_t rows = (size_t)C * a.Hkv * p.n_splits * a.sub_splits * K * (a.Hq / a.Hkv);
   a.ws_acc = (float*)ws;
   a.ws_ml = a.ws_acc + rows * a.D;
   a.err = device_error_word();

@@ -68,6 +68,7 @@ size_t ssd_smem_bytes(int P, int N, int Q);
 void ssd_scan(int dtype, const SsdArgs& a, cudaStream_t s);
 
 // ------------------------------------------------------------ attn.cu
+constexpr int kAttnTcTile = 64;  // keys per tile of the tensor-core attention path
 struct AttnArgs {
   int C, K, Hq, Hkv, D;
   const void* q; long q_rs;              // token row stride; head h at column h*D
@@ -81,13 +82,15 @@ struct AttnArgs {
   int n_splits;                          // splits per (request, kv head) upper bound
   bool causal_block;
   bool block_in_last_split;              // tensor-core path: block keys ride with the last context split
+  int sub_splits;                        // partials per split (tensor-core path: one per softmax warpgroup)
   float* ws_acc; float* ws_ml;           // split partials
   int* err;
 };
 // Split policy (tokens per split, splits per request) and workspace bytes.
 int attn_split_tokens(int dtype, int C, int Hkv, int K, int max_ctx, int requested);
 int attn_num_splits(int dtype, int K, int max_ctx, int split_tokens);
-size_t attn_ws_bytes(int C, int Hkv, int K, int G, int D, int n_splits);
+size_t attn_ws_bytes(int C, int Hkv, int K, int G, int D, int n_splits, int sub_splits);
+int attn_sub_splits(int dtype);
 bool attn_supported(int dtype, int K, int G, int D, const char** why);
 // Checks the pointer / stride requirements of the tensor-core path (bf16).
 bool attn_tc_supported(const AttnArgs& a, const char** why);

@@ -36,7 +36,7 @@ EXPORTS = ("hspec_inject_state", "hspec_ssd_block_scan", "hspec_attn_workspace_s
            "hspec_step_workspace_size", "hspec_draft_step", "hspec_sync_status",
            "hspec_status_string", "hspec_last_error", "hspec_launch_count", "hspec_version",
            "hspec_profile_enable", "hspec_profile_read", "hspec_attn_paged_block_noalloc")
-HSPEC_NOALLOC_SCRATCH_BYTES = 32 << 20
+HSPEC_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
 class HspecError(RuntimeError):

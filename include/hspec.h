@@ -188,7 +188,7 @@ HSPEC_API hspec_status hspec_attn_paged_block(const hspec_cfg* cfg, const void* 
  *    reads.  Calls that overlap on the GPU (different streams, or different host
  *    threads on one device) race on the array; serialise them.
  *  - Calls no cudaMalloc, cudaFree or other allocating routine. */
-#define HSPEC_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+#define HSPEC_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
 HSPEC_API hspec_status hspec_attn_paged_block_noalloc(const hspec_cfg* cfg, const void* q,
                                                       const hspec_kv_view* kv, const int32_t* ctx_lens,
                                                       const void* k_blk, const void* v_blk, int C, int K,

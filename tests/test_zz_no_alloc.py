@@ -41,9 +41,13 @@ def without_workspace(H, cfg, inp, K):
     return out
 
 
-@pytest.mark.parametrize("name", ["llama_c32", "tiny"])
+# Llama-3-8B shapes with 16 requests of up to 8k context fit the 64 MiB scratch
+LLAMA_C16 = I.Workload("llama_c16", I.LLAMA, C=16, K=16, ctx_lo=512, ctx_hi=8192, seed=5)
+
+
+@pytest.mark.parametrize("name", ["llama_c16", "tiny"])
 def test_noalloc_attention_matches_workspace_attention_twice(H, cuda, name):
-    wl = I.WORKLOADS[name]
+    wl = LLAMA_C16 if name == "llama_c16" else I.WORKLOADS[name]
     sh = wl.shapes
     cfg = H.make_cfg(sh)
     for call, seed in enumerate((31, 32)):  # two calls in a row through the shared scratch
