@@ -159,34 +159,66 @@ __global__ void attn_merge_kernel(AttnArgs a) {
   const size_t base0 = (((size_t)c * a.Hkv + g) * a.n_splits * a.sub_splits) * R + row;
   // Partial q exists when its split has keys for it: on the tensor-core path half h of
   // split s holds the split's tiles of parity h, so it exists iff the split has more
-  // than h tiles (the rest of the workspace is never written and never read); a
-  // partial with l = 0 saw no key and is skipped.
+  // than h tiles (a missing partial is never written, and its weight is 0); a partial
+  // with l = 0 saw no key and is skipped.
   const int n_units = ns / a.sub_splits;
   auto has = [&](int q) -> bool {
     if (!a.block_in_last_split) return true;
     const int sp = q / a.sub_splits, h = q % a.sub_splits;
     const int b = sp * a.split_tokens, e = min(ctx, b + a.split_tokens);
-    const int tiles = (e > b ? (e - b + kAttnTcTile - 1) / kAttnTcTile : 0) + (sp == n_units - 1 ? 1 : 0);
+    const int nbt = (a.K + kAttnTcTile - 1) / kAttnTcTile;  // tiles of the block's own keys
+    const int tiles = (e > b ? (e - b + kAttnTcTile - 1) / kAttnTcTile : 0) + (sp == n_units - 1 ? nbt : 0);
     return tiles > h;
   };
+  // (m, l) of partial q: lanes take q = lane, lane + 32, ... (independent loads)
+  auto ml_of = [&](int q) -> float2 { return *(const float2*)(a.ws_ml + (base0 + (size_t)q * R) * 2); };
   float M = -INFINITY;
-  for (int q = 0; q < ns; ++q) {
-    const float* ml = a.ws_ml + (base0 + (size_t)q * R) * 2;
-    if (has(q) && ml[1] > 0.f) M = fmaxf(M, ml[0]);
-  }
-  float L = 0.f;
-  for (int q = 0; q < ns; ++q) {
-    const float* ml = a.ws_ml + (base0 + (size_t)q * R) * 2;
-    if (has(q) && ml[1] > 0.f) L += exp2f(ml[0] - M) * ml[1];
-  }
-  const float inv = L > 0.f ? 1.f / L : 0.f;
-  for (int e = lane; e < a.D; e += 32) {
-    float o = 0.f;
-    for (int q = 0; q < ns; ++q) {
-      const float* ml = a.ws_ml + (base0 + (size_t)q * R) * 2;
-      if (has(q) && ml[1] > 0.f) o = fmaf(exp2f(ml[0] - M), a.ws_acc[(base0 + (size_t)q * R) * a.D + e], o);
+  for (int q = lane; q < ns; q += 32)
+    if (has(q)) {
+      const float2 ml = ml_of(q);
+      if (ml.y > 0.f) M = fmaxf(M, ml.x);
     }
-    out[e] = from_f<T>(o * inv);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  float L = 0.f;
+  for (int q = lane; q < ns; q += 32)
+    if (has(q)) {
+      const float2 ml = ml_of(q);
+      if (ml.y > 0.f) L += exp2f(ml.x - M) * ml.y;
+    }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  // o = sum_q w_q acc_q with w_q = 2^(m_q - M) (0 for a missing partial): lane holds
+  // elements lane + 32 i; the acc loads do not depend on the weights, so the loads of
+  // several partials are in flight together (a missing partial is read but not used)
+  constexpr int EPL = 4;  // elements per lane (head_dim <= 128)
+  float o[EPL] = {0.f, 0.f, 0.f, 0.f};
+  for (int q0 = 0; q0 < ns; q0 += 32) {
+    float w_l = 0.f;
+    if (q0 + lane < ns && has(q0 + lane)) {
+      const float2 ml = ml_of(q0 + lane);
+      if (ml.y > 0.f) w_l = exp2f(ml.x - M);
+    }
+    const int cnt = min(32, ns - q0);
+#pragma unroll 4
+    for (int k = 0; k < cnt; ++k) {
+      const float w = __shfl_sync(0xffffffffu, w_l, k);
+      const float* accp = a.ws_acc + (base0 + (size_t)(q0 + k) * R) * a.D;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        if (e < a.D) {
+          const float x = accp[e];
+          o[i] = w != 0.f ? fmaf(w, x, o[i]) : o[i];
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    const int e = lane + 32 * i;
+    if (e < a.D) out[e] = from_f<T>(o[i] * inv);
   }
 }
 

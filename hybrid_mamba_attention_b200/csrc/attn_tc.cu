@@ -50,10 +50,12 @@ int* device_error_word();
 namespace {
 
 constexpr int TT = kAttnTcTile;  // tokens per tile
-constexpr int NS = 5;         // K/V ring stages
-constexpr int THREADS = 320;
+constexpr int PPT = TT / 16;     // 16-token pages per tile
+constexpr int NS = TT == 64 ? 5 : 10;   // K/V ring stages (160 KB)
+constexpr int NSB = TT == 64 ? 4 : 8;   // S buffers in TMEM (half the columns)
+constexpr int NPW = 4;           // producer warps
+constexpr int THREADS = 32 * (NPW + 2 + 8);  // producers, 2 MMA warps, 2 softmax warpgroups
 constexpr int ROWS = 128;     // MMA M
-constexpr int NSB = 4;        // S buffers in TMEM, two per softmax warpgroup
 constexpr int kLenBuckets = 256;  // schedule: units sorted by tile count (capped)
 
 struct TileMeta {  // written by the producer before the stage's barrier arrive
@@ -64,7 +66,7 @@ struct TileMeta {  // written by the producer before the stage's barrier arrive
   int block;       // 1: the block's own keys
   int qslot, qseq; // Q buffer of the item and the item's use count of that buffer
   int end;         // 1: no more work
-  int pad;
+  int bt;          // block tiles: index among the block's tiles
 };
 
 template <int D>
@@ -72,19 +74,19 @@ struct Lay {
   static constexpr int DB = D / 64;                     // 64-element column blocks
   static constexpr int Q_BLK = ROWS * 128;              // 16 KB per Q column block
   static constexpr int Q_BYTES = DB * Q_BLK;
-  static constexpr int KV_BLK = TT * 128;               // 8 KB per K column block
-  static constexpr int K_BYTES = DB * KV_BLK;           // K: [column block][64 tokens][128 B]
+  static constexpr int KV_BLK = TT * 128;               // per K column block
+  static constexpr int K_BYTES = DB * KV_BLK;           // K: [column block][TT tokens][128 B]
   static constexpr int V_PAGE = DB * 2048;              // V: [page][column block][16 tokens][128 B]
   static constexpr int STAGE = 2 * K_BYTES;             // K then V
   static constexpr int OFF_Q = 0;                       // two Q buffers
   static constexpr int OFF_KV = 2 * Q_BYTES;
   static constexpr int OFF_META = OFF_KV + NS * STAGE;
   static constexpr int OFF_BAR = OFF_META + 64 * NS;
-  static constexpr int SMEM = OFF_BAR + 256 + 1024;
-  // TMEM columns: S_b [64b, 64b+64) for b < 4 (P of the tile, bf16 packed, overwrites
-  // its first 32 columns), O_w [256 + 128w, 256 + 128w + D)
+  static constexpr int SMEM = OFF_BAR + 512 + 1024;
+  // TMEM columns: S_b [TT b, TT b + TT) for b < NSB (P of the tile, bf16 packed,
+  // overwrites its first TT / 2 columns), O_w [256 + 128w, 256 + 128w + D)
   static constexpr uint32_t TMEM_COLS = 512;
-  __host__ __device__ static constexpr uint32_t S_COL(int b) { return (uint32_t)(b * 64); }
+  __host__ __device__ static constexpr uint32_t S_COL(int b) { return (uint32_t)(b * TT); }
   __host__ __device__ static constexpr uint32_t O_COL(int w) { return (uint32_t)(256 + w * 128); }
 };
 
@@ -100,18 +102,19 @@ __device__ __forceinline__ int row_of_lane(int lane128, bool spread) {
   return l < 16 ? q * 16 + l : -1;
 }
 
-// Tiles (64-token tiles, plus the block tile in a request's last split) of unit
-// (ctx, split sp of n).
-__host__ __device__ inline int unit_tiles(int ctx, int sp, int n, int split_tokens) {
+// Tiles (TT-token context tiles, plus the block's own keys, nbt tiles, in a request's
+// last split) of unit (ctx, split sp of n).
+__host__ __device__ inline int unit_tiles(int ctx, int sp, int n, int split_tokens, int nbt) {
   const int b = sp * split_tokens, e = min(ctx, b + split_tokens);
-  return (e > b ? (e - b + TT - 1) / TT : 0) + (sp == n - 1 ? 1 : 0);
+  return (e > b ? (e - b + TT - 1) / TT : 0) + (sp == n - 1 ? nbt : 0);
 }
 
 // One CTA: lists the (request, split) units longest first into `units` and resets the
 // work counter; sched[1] = number of units.  Requests with an invalid context length
 // get no unit (their output rows are written as zeros by the merge).
 __global__ void __launch_bounds__(1024) attn_sched_kernel(const int32_t* ctx_lens, int C, int split_tokens,
-                                                          long max_ctx, int* sched, int2* units, int* err) {
+                                                          long max_ctx, int nbt, int* sched, int2* units,
+                                                          int* err) {
   __shared__ int hist[kLenBuckets];
   for (int b = threadIdx.x; b < kLenBuckets; b += blockDim.x) hist[b] = 0;
   __syncthreads();
@@ -122,7 +125,7 @@ __global__ void __launch_bounds__(1024) attn_sched_kernel(const int32_t* ctx_len
       continue;
     }
     const int n = ctx > 0 ? (ctx + split_tokens - 1) / split_tokens : 1;
-    for (int sp = 0; sp < n; ++sp) atomicAdd(&hist[min(unit_tiles(ctx, sp, n, split_tokens), kLenBuckets - 1)], 1);
+    for (int sp = 0; sp < n; ++sp) atomicAdd(&hist[min(unit_tiles(ctx, sp, n, split_tokens, nbt), kLenBuckets - 1)], 1);
   }
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -141,7 +144,7 @@ __global__ void __launch_bounds__(1024) attn_sched_kernel(const int32_t* ctx_len
     if (ctx < 0 || ctx > max_ctx) continue;
     const int n = ctx > 0 ? (ctx + split_tokens - 1) / split_tokens : 1;
     for (int sp = 0; sp < n; ++sp) {
-      const int pos = atomicAdd(&hist[min(unit_tiles(ctx, sp, n, split_tokens), kLenBuckets - 1)], 1);
+      const int pos = atomicAdd(&hist[min(unit_tiles(ctx, sp, n, split_tokens, nbt), kLenBuckets - 1)], 1);
       units[pos] = make_int2(c, sp);
     }
   }
@@ -158,7 +161,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint8_t* sQ = smem + L::OFF_Q;
   uint8_t* sKV = smem + L::OFF_KV;
   volatile TileMeta* meta = (volatile TileMeta*)(smem + L::OFF_META);
-  uint64_t* kv_full = (uint64_t*)(smem + L::OFF_BAR);
+  uint64_t* kv_full = (uint64_t*)(smem + L::OFF_BAR);  // one arrival per producer warp
   uint64_t* kv_empty = kv_full + NS;
   uint64_t* s_full = kv_empty + NS;   // [NSB] S_b written by Q.K^T
   uint64_t* s_free = s_full + NSB;    // [NSB] P.V of S_b's tile finished (S_b / P free)
@@ -169,18 +172,21 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* pv_done = p_full + NSB;   // [2]   group w's P.V finished (O_w quiescent)
   uint64_t* q_full = pv_done + 2;     // [2]
   uint64_t* q_empty = q_full + 2;     // [2]
-  uint64_t* drain = q_empty + 2;      // every MMA (and its barrier arrivals) finished
-  uint32_t* tmem_slot = (uint32_t*)(drain + 1);
+  uint64_t* drain = q_empty + 2;      // [2] every MMA of an issuer (and its arrivals) finished
+  uint32_t* tmem_slot = (uint32_t*)(drain + 2);
   volatile int* end_tile = (volatile int*)(tmem_slot + 1);
+  volatile int* s_item = end_tile + 1;  // [2] next work item, published by producer warp 0
+  volatile int* s_stop = s_item + 2;    // a producer warp gave up waiting
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = a.Hq / a.Hkv, R = a.K * G;
   const bool spread = R <= 64;
   int* err = a.err;
+  constexpr int QK_WARP = NPW, PV_WARP = NPW + 1, SM_WARP0 = NPW + 2;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
-      tc::mbar_init(&kv_full[s], 1);
+      tc::mbar_init(&kv_full[s], NPW);
       tc::mbar_init(&kv_empty[s], 1);
     }
     for (int b = 0; b < NSB; ++b) {
@@ -193,11 +199,13 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc::mbar_init(&q_full[w], 1);
       tc::mbar_init(&q_empty[w], 1);
     }
-    tc::mbar_init(drain, 1);
+    tc::mbar_init(&drain[0], 1);
+    tc::mbar_init(&drain[1], 1);
     *end_tile = 0x7fffffff;
+    *s_stop = 0;
     tc::fence_mbar_init();
   }
-  if (warp == 1) tc::tmem_alloc(tmem_slot, L::TMEM_COLS);
+  if (warp == QK_WARP) tc::tmem_alloc(tmem_slot, L::TMEM_COLS);
   // Q rows without a query are never written by TMA: zero both Q buffers once
   for (int e = threadIdx.x; e < 2 * L::Q_BYTES / 16; e += THREADS) ((uint4*)sQ)[e] = make_uint4(0, 0, 0, 0);
   tc::fence_proxy_async();
@@ -206,9 +214,22 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
+  if (warp < NPW) {
+    // ------------------------------------------------------------ producers
+    // A tile's TMA boxes are spread over the NPW producer warps (the issue of one box
+    // takes a warp tens of nanoseconds; in parallel the boxes keep up with HBM):
+    // box bx < KB is K page bx / DB, column block bx % DB (16 tokens x 64 dims of head
+    // g, 128-byte swizzle); box KB + q is V page q (one 4-D box, both column blocks).
+    // Box bx is issued by lane bx / NPW of warp bx % NPW.  All producer warps walk the
+    // same tiles; warp 0 takes the work items and loads the Q tiles.
+    constexpr int KB = PPT * L::DB, NBX = KB + PPT;
+    const int pw = warp;
+    const int bx = pw + NPW * lane;
+    const bool has_box = bx < NBX;
+    const bool k_box = bx < KB;
+    const int q16 = k_box ? bx / L::DB : bx - KB;  // page of the tile
+    const int bk = k_box ? bx % L::DB : 0;
+    if (threadIdx.x == 0) {
       tc::tma_prefetch_desc(&maps.k);
       tc::tma_prefetch_desc(&maps.v);
       tc::tma_prefetch_desc(&maps.kb);
@@ -221,14 +242,19 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int q_pos = spread ? 16 / G : ROWS / G;
     const int per_unit = a.Hkv * n_rb;
     const int n_items = sched[1] * per_unit;
+    const int nbt = (a.K + TT - 1) / TT;  // tiles of the block's own keys
+    const int pshift = (a.page_size & (a.page_size - 1)) == 0 ? __ffs(a.page_size) - 1 : -1;
     int tile_i = 0;
     bool ok = true;
-    int it_next = lane == 0 ? atomicAdd(sched, 1) : 0;  // the following item's index, in flight
-    for (int seq = 0; ok; ++seq) {
-      int item = lane == 0 ? it_next : 0;
-      item = __shfl_sync(0xffffffffu, item, 0);
-      if (item >= n_items) break;
-      if (lane == 0) it_next = atomicAdd(sched, 1);  // prefetch: used by the next item
+    int it_next = threadIdx.x == 0 ? atomicAdd(sched, 1) : 0;  // the following item, in flight
+    // Every producer warp passes the same item barriers: the loop ends only after one,
+    // when the work is done or a producer has given up waiting.
+    for (int seq = 0;; ++seq) {
+      if (threadIdx.x == 0) s_item[seq & 1] = it_next;
+      asm volatile("bar.sync 1, %0;" ::"n"(32 * NPW) : "memory");
+      const int item = s_item[seq & 1];
+      if (item >= n_items || *s_stop) break;
+      if (threadIdx.x == 0) it_next = atomicAdd(sched, 1);  // prefetch: used by the next item
       const int u = item / per_unit, g = item % a.Hkv, rb = (item % per_unit) / a.Hkv;
       const int2 cu = units[u];
       const int c = cu.x, split = cu.y;
@@ -237,34 +263,34 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int c_begin = split * a.split_tokens;
       const int c_end = min(ctx, c_begin + a.split_tokens);
       const int n_ctx_tiles = c_end > c_begin ? (c_end - c_begin + TT - 1) / TT : 0;
-      const int n_tiles = n_ctx_tiles + (split == n_ctx_splits - 1 ? 1 : 0);
+      const int n_tiles = n_ctx_tiles + (split == n_ctx_splits - 1 ? nbt : 0);
       const int slot = seq & 1;
 
       // Q tile of the item into Q buffer `slot` once the item two back is done with it
-      if (lane == 0) ok = tc::mbar_wait(&q_empty[slot], ((seq >> 1) & 1) ^ 1, err);
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-      if (!ok) break;
-      uint8_t* qbuf = sQ + slot * L::Q_BYTES;
-      if (lane == 0) tc::mbar_arrive_expect_tx(&q_full[slot], (uint32_t)(q_boxes * L::DB * q_pos * G * 128));
-      __syncwarp();
-      if (lane < q_boxes * L::DB) {
-        const int qb = lane / L::DB, bk = lane % L::DB;
-        const int pos0 = c * a.K + (spread ? qb * q_pos : rb * q_pos);
-        tc::tma_load_3d(qbuf + bk * L::Q_BLK + qb * 32 * 128, &maps.q, &q_full[slot], bk * 64, g * G, pos0);
+      if (pw == 0) {
+        if (lane == 0) ok = tc::mbar_wait(&q_empty[slot], ((seq >> 1) & 1) ^ 1, err);
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (ok) {
+          uint8_t* qbuf = sQ + slot * L::Q_BYTES;
+          if (lane == 0)
+            tc::mbar_arrive_expect_tx(&q_full[slot], (uint32_t)(q_boxes * L::DB * q_pos * G * 128));
+          __syncwarp();
+          if (lane < q_boxes * L::DB) {
+            const int qb = lane / L::DB, qk = lane % L::DB;
+            const int pos0 = c * a.K + (spread ? qb * q_pos : rb * q_pos);
+            tc::tma_load_3d(qbuf + qk * L::Q_BLK + qb * 32 * 128, &maps.q, &q_full[slot], qk * 64, g * G, pos0);
+          }
+          __syncwarp();
+        }
       }
-      __syncwarp();
 
-      // Page ids: lane L holds the id of page q16 = L % 4 of the tile (a 64-token tile
-      // spans four 16-token pages) for the current tile and the next two.  K boxes are
-      // issued by lanes 0 .. 4 DB - 1 (column block L / 4), V boxes by lanes 16..19.
-      // The table reads are unconditional (the index is clamped into the request's
-      // row of the table) and their values are used two tiles later, so nothing waits
-      // for them; ids of tokens past the split's end are never used.
+      // page id of this lane's page, read two tiles ahead into registers
+      // (unconditionally, the index clamped into the request's row of the table, so
+      // that nothing waits for it; ids past the split's end are never used)
       const int32_t* table = a.page_table + (size_t)c * a.max_pages;
-      const int q16 = lane & 3, lj = lane >> 2;
-      const bool k_lane = lj < L::DB, v_lane = lj == 4;
       auto page_of = [&](int local) -> int {
-        const int idx = (c_begin + local * TT + 16 * q16) / a.page_size;
+        const int t = c_begin + local * TT + 16 * q16;
+        const int idx = pshift >= 0 ? t >> pshift : t / a.page_size;
         return table[idx < a.max_pages ? idx : a.max_pages - 1];
       };
       int pid0 = page_of(0), pid1 = page_of(1);
@@ -280,66 +306,107 @@ __global__ void __launch_bounds__(THREADS, 1)
         uint8_t* kd = sKV + s * L::STAGE;
         uint8_t* vd = kd + L::K_BYTES;
         const bool block = local >= n_ctx_tiles;
+        const int bt = local - n_ctx_tiles;  // block tiles: keys [bt TT, bt TT + TT) of the block
         const int t0 = c_begin + local * TT;
-        const int valid = block ? a.K : min(TT, c_end - t0);
-        if (lane == 0) {
+        const int valid = block ? min(TT, a.K - bt * TT) : min(TT, c_end - t0);
+        const int groups = (valid + 15) / 16;  // 16-row boxes with keys
+        if (pw == 0 && lane == 0) {
           volatile TileMeta& m = meta[s];
           m.c = c, m.g = g, m.split = split, m.rb = rb, m.valid = valid, m.local = local;
           m.n_tiles = n_tiles, m.block = block ? 1 : 0, m.qslot = slot, m.qseq = seq, m.end = 0;
+          m.bt = block ? bt : 0;
         }
-        if (!block) {
-          const int groups = (valid + 15) / 16;
-          if (lane == 0) tc::mbar_arrive_expect_tx(&kv_full[s], (uint32_t)(groups * L::DB * 2048 * 2));
-          __syncwarp();
-          if ((k_lane || v_lane) && q16 < groups) {
-            const int t = t0 + 16 * q16;
+        // this lane's box: what it loads and how many bytes
+        uint32_t bytes = 0;
+        if (has_box && q16 < groups) {
+          if (!block) bytes = k_box ? 2048u : (uint32_t)L::V_PAGE;
+          else if (k_box ? q16 == 0 : true) bytes = k_box ? (uint32_t)(16 * 128) * PPT : (uint32_t)L::V_PAGE;
+        }
+        // block tiles: K of column block bk is one TT-row box (lanes with q16 == 0)
+        const uint32_t warp_bytes = __reduce_add_sync(0xffffffffu, bytes);
+        if (lane == 0) tc::mbar_arrive_expect_tx(&kv_full[s], warp_bytes);  // also this warp's arrival
+        __syncwarp();
+        if (bytes) {
+          if (!block) {
             int pg = pid;
             if (pg < 0 || pg >= a.num_pages) {
               flag_error(err, kErrPageOOB);
               pg = 0;  // keep the copy in bounds; the request's output is flagged as invalid
             }
-            const int z = pg * a.page_size + t % a.page_size;
-            if (k_lane) {
-              const int bk = lj;
+            const int tt = t0 + 16 * q16;
+            const int z = pg * a.page_size + (pshift >= 0 ? (tt & (a.page_size - 1)) : tt % a.page_size);
+            if (k_box)
               tc::tma_load_3d(kd + bk * L::KV_BLK + q16 * 2048, &maps.k, &kv_full[s], bk * 64, g, z);
-            } else {
+            else
               tc::tma_load_4d(vd + q16 * L::V_PAGE, &maps.v, &kv_full[s], 0, z, g, 0);
-            }
-          }
-        } else {
-          const int nq = (a.K + 15) / 16;
-          if (lane == 0) tc::mbar_arrive_expect_tx(&kv_full[s], (uint32_t)(L::DB * L::KV_BLK + nq * L::V_PAGE));
-          __syncwarp();
-          if (lane < L::DB) {
-            tc::tma_load_3d(kd + lane * L::KV_BLK, &maps.kb, &kv_full[s], lane * 64, g, c * a.K);
-          } else if (lane >= 16 && lane < 16 + nq) {
-            tc::tma_load_4d(vd + (lane - 16) * L::V_PAGE, &maps.vb, &kv_full[s], 0, c * a.K + 16 * (lane - 16), g, 0);
+          } else {
+            const int row0 = c * a.K + bt * TT;
+            if (k_box)
+              tc::tma_load_3d(kd + bk * L::KV_BLK, &maps.kb, &kv_full[s], bk * 64, g, row0);
+            else
+              tc::tma_load_4d(vd + q16 * L::V_PAGE, &maps.vb, &kv_full[s], 0, row0 + 16 * q16, g, 0);
           }
         }
         __syncwarp();
       }
+      if (!ok) *s_stop = 1;
     }
     // sentinel stage: no more work
-    if (ok && lane == 0) {
+    if (!*s_stop) {
       const int s = tile_i % NS;
-      if (tc::mbar_wait(&kv_empty[s], ((tile_i / NS) & 1) ^ 1, err)) {
-        meta[s].end = 1;
+      bool fine = true;
+      if (lane == 0) fine = tc::mbar_wait(&kv_empty[s], ((tile_i / NS) & 1) ^ 1, err);
+      if (lane == 0 && fine) {
+        if (pw == 0) meta[s].end = 1;
         tc::mbar_arrive(&kv_full[s]);
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == QK_WARP) {
     if (lane == 0) {
-      // ---------------------------------------------------------- MMA issuer
+      // ---------------------------------------------------------- Q.K^T issuer
+      // S_b = Q . K_i^T into S buffer b = i % NSB once tile i has landed, S_b is free
+      // (the P.V of tile i - NSB has read its P) and the item's Q is loaded.  Issuing
+      // P.V from another thread keeps either kind of MMA from waiting behind the other.
       constexpr uint32_t idesc_qk = tc::idesc_bf16_f32(ROWS, TT);
-      constexpr uint32_t idesc_pv = tc::idesc_bf16_f32(ROWS, D) | (1u << 16);  // B (= V) MN-major
       int q_seen[2] = {-1, -1};
-      int qk = 0, pv = 0, end_at = 0x7fffffff;
+      for (int qk = 0;; ++qk) {
+        const int s = qk % NS, b = qk & (NSB - 1);
+        if (qk >= NSB && !tc::mbar_wait(&s_free[b], ((qk / NSB) - 1) & 1, err)) break;
+        if (!tc::mbar_wait(&kv_full[s], (qk / NS) & 1, err)) break;
+        if (meta[s].end) {
+          *end_tile = qk;
+          break;
+        }
+        const int slot = meta[s].qslot, seq = meta[s].qseq;
+        if (seq > q_seen[slot]) {
+          if (!tc::mbar_wait(&q_full[slot], (seq >> 1) & 1, err)) break;
+          q_seen[slot] = seq;
+        }
+        tc::tc_fence_after();
+        const uint32_t q = tc::smem_u32(sQ + slot * L::Q_BYTES), k = tc::smem_u32(sKV + s * L::STAGE);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          tc::mma_bf16(tmem + L::S_COL(b), tc::sdesc_k128(q + (kk / 4) * L::Q_BLK + (kk % 4) * 32),
+                       tc::sdesc_k128(k + (kk / 4) * L::KV_BLK + (kk % 4) * 32), idesc_qk, kk > 0);
+        tc::mma_commit(&s_full[b]);
+        if (meta[s].local == meta[s].n_tiles - 1) tc::mma_commit(&q_empty[slot]);  // item's last QK
+      }
+      // no MMA or commit arrival may land after the CTA has finished
+      tc::mma_commit(&drain[0]);
+      tc::mbar_wait(&drain[0], 0, err);
+    }
+  } else if (warp == PV_WARP) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- P.V issuer
+      // O_w += P_i . V_i as soon as the P of tile i is in TMEM (group w = i % 2).  Tile
+      // i's Q.K^T finished before its softmax began, so the commit after P.V frees the
+      // whole stage.
+      constexpr uint32_t idesc_pv = tc::idesc_bf16_f32(ROWS, D) | (1u << 16);  // B (= V) MN-major
       bool ok = true;
+      int pv = 0;
       uint64_t idle_since = 0;
-      while (pv < end_at) {
-        bool progress = false;
-        // P.V of the oldest tile whose P is in shared memory
-        if (pv < qk && tc::mbar_test_wait(&p_full[pv & (NSB - 1)], (pv / NSB) & 1)) {
+      while (pv < *end_tile) {
+        if (tc::mbar_test_wait(&p_full[pv & (NSB - 1)], (pv / NSB) & 1)) {
           tc::tc_fence_after();
           const int w = pv & 1, s = pv % NS;
           const bool first = meta[s].local < 2;  // this group's first tile of the item
@@ -347,43 +414,13 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint32_t v = tc::smem_u32(sKV + s * L::STAGE + L::K_BYTES);
           // K slice kk = the 16 keys of page kk: V [column block][16 tokens] blocks 2 KB apart
 #pragma unroll
-          for (int kk = 0; kk < TT / 16; ++kk)
+          for (int kk = 0; kk < PPT; ++kk)
             tc::mma_bf16_ts(tmem + L::O_COL(w), pt + kk * 8, tc::sdesc_mn128(v + kk * L::V_PAGE, 2048), idesc_pv,
                             (kk > 0 || !first) ? 1u : 0u);
           tc::mma_commit(&kv_empty[s]);
           tc::mma_commit(&pv_done[w]);
-          tc::mma_commit(&s_free[pv & (NSB - 1)]);  // P read: S buffer free for tile pv + 4
+          tc::mma_commit(&s_free[pv & (NSB - 1)]);  // P read: S buffer free for tile pv + NSB
           ++pv;
-          progress = true;
-        }
-        // Q.K^T of the next tile once it has landed, its S buffer is free (the P.V of the
-        // tile four back has read its P) and its Q is loaded
-        if (qk < end_at) {
-          const int s = qk % NS, b = qk & (NSB - 1);
-          if ((qk < NSB || tc::mbar_test_wait(&s_free[b], ((qk / NSB) - 1) & 1)) &&
-              tc::mbar_test_wait(&kv_full[s], (qk / NS) & 1)) {
-            if (meta[s].end) {
-              end_at = qk;
-              progress = true;
-            } else {
-              const int slot = meta[s].qslot, seq = meta[s].qseq;
-              if (seq <= q_seen[slot] || tc::mbar_test_wait(&q_full[slot], (seq >> 1) & 1)) {
-                q_seen[slot] = seq > q_seen[slot] ? seq : q_seen[slot];
-                tc::tc_fence_after();
-                const uint32_t q = tc::smem_u32(sQ + slot * L::Q_BYTES), k = tc::smem_u32(sKV + s * L::STAGE);
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                  tc::mma_bf16(tmem + L::S_COL(b), tc::sdesc_k128(q + (kk / 4) * L::Q_BLK + (kk % 4) * 32),
-                               tc::sdesc_k128(k + (kk / 4) * L::KV_BLK + (kk % 4) * 32), idesc_qk, kk > 0);
-                tc::mma_commit(&s_full[b]);
-                if (meta[s].local == meta[s].n_tiles - 1) tc::mma_commit(&q_empty[slot]);  // item's last QK
-                ++qk;
-                progress = true;
-              }
-            }
-          }
-        }
-        if (progress) {
           idle_since = 0;
         } else {
           const uint64_t t = tc::global_ns();
@@ -397,23 +434,25 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
       if (ok) {
-        // wake both softmax groups: their next tiles are end_at and end_at + 1
-        *end_tile = end_at;
+        // wake both softmax groups: their next tiles are end_at and end_at + 1 (every
+        // earlier tile's softmax is done, so those S buffers' earlier phases are complete)
+        const int end_at = pv;
+        *end_tile = end_at;  // (again, by this thread, before its arrivals release it)
         tc::mbar_arrive(&s_full[end_at & (NSB - 1)]);
         tc::mbar_arrive(&s_full[(end_at + 1) & (NSB - 1)]);
       }
-      // no MMA or commit arrival may land after the CTA has finished
-      tc::mma_commit(drain);
-      tc::mbar_wait(drain, 0, err);
+      tc::mma_commit(&drain[1]);
+      tc::mbar_wait(&drain[1], 0, err);
     }
   } else {
     // ------------------------------------------------------------ softmax warpgroups
-    const int wg = (warp - 2) >> 2;         // 0: warps 2..5, 1: warps 6..9
+    const int wg = (warp - SM_WARP0) >> 2;  // 0: first four softmax warps, 1: the next four
     const int quarter = warp & 3;           // TMEM lanes this warp may access
     const int lane128 = quarter * 32 + lane;
     const int r_local = row_of_lane(lane128, spread);
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const uint32_t tOw = tmem + lane_off + L::O_COL(wg);
+    const int gthread = (warp - SM_WARP0 - 4 * wg) * 32 + lane;  // 0..127 within the group
 
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
@@ -431,6 +470,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int c = meta[s].c, g = meta[s].g, split = meta[s].split, rb = meta[s].rb;
       const int local = meta[s].local, n_tiles = meta[s].n_tiles, valid = meta[s].valid;
       const bool block_tile = meta[s].block != 0;
+      const int bt = meta[s].bt;
       const int gr = rb * ROWS + (r_local < 0 ? 0 : r_local);
       const bool active = r_local >= 0 && gr < R;
       const int jq = active ? gr / G : 0;
@@ -439,7 +479,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         l = 0.f;
       }
       float sv[TT];
-      tc::tmem_ld64(tmem + lane_off + L::S_COL(b), sv);
+      tc::tmem_ld(tmem + lane_off + L::S_COL(b), sv);
       float mx = -INFINITY;
       if (valid == TT && !(block_tile && a.causal_block)) {
 #pragma unroll
@@ -448,7 +488,8 @@ __global__ void __launch_bounds__(THREADS, 1)
           mx = fmaxf(mx, sv[j]);
         }
       } else {
-        const int vis_end = (block_tile && a.causal_block) ? min(valid, jq + 1) : valid;
+        // causal block: query position jq sees the block keys 0..jq
+        const int vis_end = (block_tile && a.causal_block) ? min(valid, jq + 1 - bt * TT) : valid;
 #pragma unroll
         for (int j = 0; j < TT; ++j) {
           sv[j] = j < vis_end ? sv[j] * scale_log2 : -INFINITY;
@@ -479,12 +520,19 @@ __global__ void __launch_bounds__(THREADS, 1)
         pk[j / 2] = *reinterpret_cast<uint32_t*>(&h2);
       }
       l += psum;
-      tc::tmem_st32u(tmem + lane_off + L::S_COL(b), pk);  // P over the first half of S_b
-      if (__any_sync(0xffffffffu, rescale)) {
-        // O_w holds this group's earlier tiles of the item; their P.V must be done
+      // P over the first half of S_b
+      tc::tmem_stu(tmem + lane_off + L::S_COL(b), pk);
+      // The group's previous P.V (before O_w may be rescaled).  It is waited for at
+      // every tile, not only before a rescale: softmax may run several tiles ahead of
+      // the P.V's, and a parity wait is only unambiguous while its waiter is at most
+      // one phase behind the barrier.
+      if (n >= 1) {
         ok = __all_sync(0xffffffffu, tc::mbar_wait(&pv_done[wg], (n - 1) & 1, err));
         if (!ok) break;
         tc::tc_fence_after();
+      }
+      if (__any_sync(0xffffffffu, rescale)) {
+        // O_w holds this group's earlier tiles of the item
 #pragma unroll
         for (int cb = 0; cb < D / 32; ++cb) {
           float v[32];
@@ -498,10 +546,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         // V rows past the last valid token may hold stale data: zero them (P is 0 there)
         uint8_t* vbase = sKV + s * L::STAGE + L::K_BYTES;
         const int n_chunks = (TT - valid) * L::DB * 8;
-        for (int e = (warp - 2 - 4 * wg) * 32 + lane; e < n_chunks; e += 128) {
+        for (int e = gthread; e < n_chunks; e += 128) {
           const int r2 = valid + e / (L::DB * 8), rest = e % (L::DB * 8);
-          const int bk = rest / 8, cc = rest % 8, rr = r2 & 15;
-          *(uint4*)(vbase + (r2 >> 4) * L::V_PAGE + bk * 2048 + rr * 128 + ((cc ^ (rr & 7)) << 4)) =
+          const int ck = rest / 8, cc = rest % 8, rr = r2 & 15;
+          *(uint4*)(vbase + (r2 >> 4) * L::V_PAGE + ck * 2048 + rr * 128 + ((cc ^ (rr & 7)) << 4)) =
               make_uint4(0, 0, 0, 0);
         }
         tc::fence_proxy_async();
@@ -537,7 +585,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   }
   __syncthreads();
-  if (warp == 1) {
+  if (warp == QK_WARP) {
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, L::TMEM_COLS);
   }
@@ -646,8 +694,8 @@ bool launch_tc(const AttnArgs& a, cudaStream_t s) {
   const size_t pairs = (size_t)a.C * a.Hkv * a.n_splits * 2 * R;
   int* sched = (int*)(a.ws_ml + pairs * 2);
   int2* units = (int2*)(sched + 64);
-  attn_sched_kernel<<<1, 1024, 0, s>>>(a.ctx_lens, a.C, a.split_tokens, (long)a.max_pages * a.page_size, sched,
-                                       units, a.err);
+  attn_sched_kernel<<<1, 1024, 0, s>>>(a.ctx_lens, a.C, a.split_tokens, (long)a.max_pages * a.page_size,
+                                       (a.K + TT - 1) / TT, sched, units, a.err);
   note_launch();
   const long max_items = (long)a.C * a.n_splits * n_rb * a.Hkv;
   const int sms = dev < 64 && n_sm[dev] > 0 ? n_sm[dev] : 148;

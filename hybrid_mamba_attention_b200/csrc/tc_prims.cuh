@@ -194,6 +194,16 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// Stores 16 consecutive 32-bit columns of this thread's TMEM lane (warp-collective)
+// and waits for the store to complete.
+__device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n\t"
+      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+
 // Stores 32 consecutive 32-bit columns of this thread's TMEM lane (warp-collective)
 // and waits for the store to complete.
 __device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t (&v)[32]) {
@@ -202,6 +212,12 @@ __device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t (&v)[3
   for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v[i]);
   tmem_st32(taddr, f);
 }
+
+// Loads / stores by width (overloads on the array size).
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, float (&v)[32]) { tmem_ld32(taddr, v); }
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, float (&v)[64]) { tmem_ld64(taddr, v); }
+__device__ __forceinline__ void tmem_stu(uint32_t taddr, const uint32_t (&v)[16]) { tmem_st16u(taddr, v); }
+__device__ __forceinline__ void tmem_stu(uint32_t taddr, const uint32_t (&v)[32]) { tmem_st32u(taddr, v); }
 
 // ---------------------------------------------------------------- MMA
 // D[tmem] (+)= A[smem] . B[smem]^T, bf16 inputs, fp32 accumulate, cta_group::1.

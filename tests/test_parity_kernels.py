@@ -255,10 +255,10 @@ def test_context_longer_than_page_table_is_reported(H, cuda):
 
 # ------------------------------------------- tensor-core attention edge shapes
 
-@pytest.mark.parametrize("K,lens", [(1, [0, 1, 15, 16, 63, 64, 65, 4097]), (3, [0, 7, 130, 2000]),
-                                    (16, [64, 128, 4096, 4100, 8191])])
+@pytest.mark.parametrize("K,lens", [(1, [0, 1, 15, 16, 31, 32, 33, 63, 64, 65, 4097]), (3, [0, 7, 97, 130, 2000]),
+                                    (16, [64, 96, 128, 4096, 4100, 8191])])
 def test_bf16_attention_ragged_tiles(H, cuda, K, lens):
-    # contexts that end inside a page, on a page, on a 64-token tile and past a split
+    # contexts that end inside a page, on a page, on a key tile and past a split
     sh = I.LLAMA
     lens_t = torch.tensor(lens, dtype=torch.int32)
     inp = I.make_attn_inputs(sh, lens_t, K, 21, cuda)
@@ -275,6 +275,18 @@ def test_bf16_attention_more_than_128_query_rows(H, cuda):
     out = run_attn(H, sh, inp, 32)
     assert H.hspec_sync_status() == 0
     compare_attn(to_np(out), oracle_attn(inp, [0, 1]), sh, "attn 256 rows")
+
+
+@pytest.mark.parametrize("K", [33, 40, 64])
+def test_bf16_attention_block_keys_span_two_tiles(H, cuda, K):
+    # K > 32: the block's own keys take two key tiles; causal masking crosses them
+    sh = I.LLAMA
+    lens = torch.tensor([0, 17, 1000], dtype=torch.int32)
+    inp = I.make_attn_inputs(sh, lens, K, 24, cuda)
+    for causal in (False, True):
+        out = run_attn(H, sh, inp, K, causal=causal)
+        assert H.hspec_sync_status() == 0
+        compare_attn(to_np(out), oracle_attn(inp, [0, 1, 2], causal=causal), sh, f"attn K={K} causal={causal}")
 
 
 def test_bf16_attention_head_dim_64(H, cuda):
