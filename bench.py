@@ -122,12 +122,29 @@ def barrier(world):
 
 
 def max_over_ranks(v: float, world: int) -> float:
+    """The slowest rank's value: every rank takes the same collective step (one
+    all-reduce of one float64) on the process group's device (CUDA under NCCL, host
+    memory under gloo)."""
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_workload(I, wl, rank: int):
+    """Rank r's batch: the same shapes and context-length range, its own seed (the
+    requests of different replicas are different requests)."""
+    return I.Workload(wl.name, wl.shapes, wl.C, wl.K, wl.ctx_lo, wl.ctx_hi, seed=wl.seed + 1000 * rank)
+
+
+def replica_throughput(tokens_per_rank: int, ms_per_rank: float, world: int):
+    """Whole-job tokens/s of `world` replicas: all ranks' tokens over the slowest
+    rank's step time (max over ranks)."""
+    ms_max = max_over_ranks(ms_per_rank, world)
+    return ms_max, tokens_per_rank * world / (ms_max / 1e3)
 
 
 # ---------------------------------------------------------------- algorithmic work
@@ -284,17 +301,14 @@ def run_ours(args, rank, world, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     peaks = load_peaks()
-    wl = I.full_workload(args.C, args.K)
-    wl = I.Workload(wl.name, wl.shapes, wl.C, wl.K, wl.ctx_lo, wl.ctx_hi, seed=wl.seed + 1000 * rank)
+    wl = replica_workload(I, I.full_workload(args.C, args.K), rank)
     runner = StepRunner(H, I, wl, dev)
 
     clocks = ClockSampler(local)
     clocks.start()
     ms, launches, prof = time_steps(runner, args.steps, args.warmup, world, profile=True)
     clk = clocks.stop()
-    ms_max = max_over_ranks(ms, world)
-    tokens = wl.C * wl.K * world
-    value = tokens / (ms_max / 1e3)
+    ms_max, value = replica_throughput(wl.C * wl.K, ms, world)
 
     # roofline: per kernel group, from the events recorded on the step's stream
     work = step_work(wl.shapes, wl.C, wl.K, runner.st["ctx_lens"].cpu())
@@ -314,8 +328,8 @@ def run_ours(args, rank, world, local):
     attn_roof = kernels.get("attn_paged", {}).get("roofline")
 
     e2e_ms, e2e_wall_ms, h2d, d2h = time_e2e(runner, args.steps)
-    e2e_ms = max_over_ranks(e2e_ms, world)
-    e2e = {"value": round(tokens / (e2e_ms / 1e3), 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
+    e2e_ms, e2e_value = replica_throughput(wl.C * wl.K, e2e_ms, world)
+    e2e = {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4), "wall_ms_per_step": round(e2e_wall_ms, 4)}
 
     sweep = None
