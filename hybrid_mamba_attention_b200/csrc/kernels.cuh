@@ -66,6 +66,10 @@ struct SsdArgs {
 };
 size_t ssd_smem_bytes(int P, int N, int Q);
 void ssd_scan(int dtype, const SsdArgs& a, cudaStream_t s);
+// Tensor-core state readout (ssd_tc.cu): bf16, h0 given, no final state, one chunk,
+// K <= 16, d_state 128, 64 <= P <= 128 dividing 128.
+bool ssd_tc_supported(int dtype, const SsdArgs& a);
+bool ssd_tc_launch(const SsdArgs& a, cudaStream_t s);
 
 // ------------------------------------------------------------ attn.cu
 constexpr int kAttnTcTile = 64;  // keys per tile of the tensor-core attention path

@@ -245,6 +245,8 @@ void launch(const SsdArgs& a, cudaStream_t s) {
 size_t ssd_smem_bytes(int P, int N, int Q) { return (size_t)ssd_layout(P, N, Q).total * sizeof(float); }
 
 void ssd_scan(int dtype, const SsdArgs& a, cudaStream_t s) {
+  // bf16 drafter, one chunk, no final state: the state readout on the tensor cores
+  if (ssd_tc_supported(dtype, a) && ssd_tc_launch(a, s)) return;
   if (dtype == HSPEC_DTYPE_BF16) {
     if (a.dt_bias) launch<bf16, bf16>(a, s);
     else launch<bf16, float>(a, s);

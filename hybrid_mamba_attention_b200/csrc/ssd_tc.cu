@@ -1,0 +1,511 @@
+// Mamba-2 SSD block scan from an injected state, readout on the 5th-generation tensor
+// cores (bf16 drafter, one chunk of K <= 16 positions, no final state requested).
+// H-Spec (arXiv 2609.24197) Abstract: each Mamba layer starts from the projected
+// last-token hidden state and the block is evaluated in parallel; the chunked
+// "state-space dual" form of Dao & Gu (2024) gives, for head h and position t,
+//
+//   y_t[p] = exp(cum_t) sum_n C_t[n] S[p][n]                      (the injected state)
+//          + sum_{s<=t} (C_t . B_s) exp(cum_t - cum_s) dt_s x_s[p]  (inside the block)
+//          + D_h x_t[p],                    cum_t = sum_{r<=t} dt_r A_h,
+//
+// the same sum as the step-by-step recurrence.  The state S = h0 of one request is
+// H*P rows of N fp32 values: 2 MB per request and layer at Llama shapes, the only large
+// operand, read once.  Its readout C . S^T is a dense contraction (K x N by N x H*P)
+// and runs on tcgen05 as kind::tf32 with M = 128 state rows (heads x P), N = 16
+// positions, K = 8 per instruction, the accumulator in TMEM.  So that the product is
+// as exact as fp32, each state tile is split into hi = tf32(S), rounded in place in
+// shared memory, and lo = S - hi, written to TMEM and read by the MMA from there (C is
+// exact in tf32: it comes from bf16); tf32 x tf32 products are exact and accumulate in
+// fp32.
+//
+// Persistent kernel, one CTA per SM, a static range of (request, 128-row tile) items:
+//   warp 0      TMA producer: the fp32 state tile (N / 32 boxes of 128 rows x 128 B,
+//               128-byte swizzle) into one of three stages.
+//   warp 1      TMEM owner and MMA issuer: 2 (hi from shared memory, lo from TMEM) x
+//               N / 8 MMAs per tile into one of two TMEM accumulators.
+//   warps 2..5  transform group 0 (tiles k even), warps 6..9 group 1 (k odd); per tile,
+//               one state row (= TMEM lane) per thread: round the row to tf32 in place
+//               and write its lo to the group's TMEM buffer; for a new request the C^T
+//               operand (bf16 -> fp32, swizzled) and C . B^T; the tile's dt, cumulative
+//               decay, the in-block matrix L and x; then, once the tile's MMAs are done,
+//               its epilogue.  The tile's global loads are issued before its waits, and
+//               the two groups overlap each other's latencies.
+// Every wait gives up after a time bound and sets the device error word.
+#include <stdint.h>
+
+#include "../../include/hspec.h"
+#include "common.cuh"
+#include "kernels.cuh"
+#include "tc_prims.cuh"
+
+namespace hspec {
+
+int* device_error_word();
+
+namespace {
+
+constexpr int THREADS = 320;  // producer, MMA, 2 transform warpgroups
+constexpr int ROWS = 128;    // MMA M: state rows (head, p) per tile
+constexpr int NT = 16;       // MMA N: positions (K <= 16, rows past K are zero)
+constexpr int KMAX = 16;
+constexpr int NMAX = 128;    // d_state
+constexpr int TILE_BYTES = ROWS * NMAX * 4;  // 64 KB
+constexpr int HPT_MAX = 2;   // heads per tile (P >= 64)
+constexpr int NSTAGE = 3;    // state-tile stages
+// TMEM columns: lo of tile k in [128 (k % 2), +128), accumulator of tile k at 256 + 16 (k % 2)
+constexpr uint32_t TMEM_COLS = 512;
+
+struct SsdTcLay {
+  static constexpr int OFF_A = 0;                          // stages of the state tile (hi)
+  static constexpr int OFF_B = OFF_A + NSTAGE * TILE_BYTES;  // C^T: [n/32][16 positions][128 B]
+  static constexpr int B_BYTES = NMAX / 32 * NT * 128;     // 8 KB
+  // per transform group g: x, L^T, exp(cum) and D, C . B^T, dt and cum
+  static constexpr int OFF_X = OFF_B + B_BYTES;            // x: [2][KMAX][ROWS] fp32
+  static constexpr int X_BYTES = KMAX * ROWS * 4;
+  static constexpr int OFF_L = OFF_X + 2 * X_BYTES;        // L^T: [2][HPT_MAX][KMAX (s)][KMAX (t)]
+  static constexpr int L_BYTES = HPT_MAX * KMAX * KMAX * 4;
+  static constexpr int OFF_E = OFF_L + 2 * L_BYTES;        // exp(cum): [2][HPT_MAX][KMAX], D_h: [2][HPT_MAX]
+  static constexpr int E_BYTES = HPT_MAX * (KMAX + 1) * 4;
+  static constexpr int OFF_CB = OFF_E + 2 * E_BYTES;       // C . B^T: [2][KMAX][KMAX]
+  static constexpr int OFF_DT = OFF_CB + 2 * KMAX * KMAX * 4;  // dt, then cum: [2][2][HPT_MAX][KMAX]
+  static constexpr int OFF_BAR = OFF_DT + 4 * HPT_MAX * KMAX * 4;
+  static constexpr int SMEM = OFF_BAR + 256 + 1024;
+};
+
+struct SsdTcArgs {
+  SsdArgs a;
+  int* err;       // device error word
+  int hpt;        // heads per tile = 128 / P
+  int n_tiles;    // tiles per request = H / hpt
+  int n_items;    // C * n_tiles
+};
+
+// hi: the value with its 13 low mantissa bits cleared (a tf32 value, whatever rounding
+// the tensor core applies to it); lo = v - hi is exact in fp32 and below 2^-10 |v|.
+__device__ __forceinline__ uint32_t tf32_hi(uint32_t bits) { return bits & 0xFFFFE000u; }
+
+// Loads issued where they stand (volatile: not moved towards their first use), so
+// their latency overlaps the waits that follow.
+__device__ __forceinline__ uint16_t ldg_u16(const void* p) {
+  uint16_t v;
+  asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
+  return v;
+}
+__device__ __forceinline__ uint32_t ldg_u32(const void* p) {
+  uint32_t v;
+  asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+
+// Instruction descriptor of kind::tf32: fp32 accumulator, tf32 A and B (K-major).
+__host__ __device__ constexpr uint32_t idesc_tf32(int M, int N) {
+  return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// A from TMEM (row i in lane i, one tf32 per 32-bit column)
+__device__ __forceinline__ void mma_tf32_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_tf32(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+template <typename TDT>
+__global__ void __launch_bounds__(THREADS, 1) ssd_tc_kernel(const __grid_constant__ CUtensorMap h0_map, SsdTcArgs t) {
+  using L = SsdTcLay;
+  const SsdArgs& a = t.a;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = tc::smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw + 1023) & ~1023u) - raw);
+  uint8_t* sA = smem + L::OFF_A;
+  uint8_t* sB = smem + L::OFF_B;
+  float* sX = (float*)(smem + L::OFF_X);
+  float* sL = (float*)(smem + L::OFF_L);
+  float* sE = (float*)(smem + L::OFF_E);
+  float* sCB = (float*)(smem + L::OFF_CB);
+  float* sDt = (float*)(smem + L::OFF_DT);
+  uint64_t* a_full = (uint64_t*)(smem + L::OFF_BAR);  // [NSTAGE]
+  uint64_t* a_empty = a_full + NSTAGE;                 // [NSTAGE]
+  // [2] tile k: hi rounded, lo in TMEM buffer k % 2, operands ready (one barrier per lo
+  // buffer: the transform may finish tile k + 1 before the MMA thread has taken tile k,
+  // and the phases of one barrier must not run two ahead of its waiter)
+  uint64_t* lo_full = a_empty + NSTAGE;
+  uint64_t* acc_full = lo_full + 2;                    // [2] MMAs of the accumulator's tile done
+  uint64_t* d_free = acc_full + 2;                     // [2] epilogue has read the accumulator
+  uint64_t* drain = d_free + 2;
+  uint32_t* tmem_slot = (uint32_t*)(drain + 1);
+  volatile int* s_fail = (volatile int*)(tmem_slot + 1);  // a transform thread gave up waiting
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int P = a.P, N = a.N, K = a.K, hpt = t.hpt;
+  const int nblk = N / 32;  // 128-byte column blocks of a state row
+  int* err = t.err;
+  const int i0 = (int)((long)blockIdx.x * t.n_items / gridDim.x);
+  const int i1 = (int)((long)(blockIdx.x + 1) * t.n_items / gridDim.x);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NSTAGE; ++s) {
+      tc::mbar_init(&a_full[s], 1);
+      tc::mbar_init(&a_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      tc::mbar_init(&acc_full[s], 1);
+      tc::mbar_init(&d_free[s], 4);
+    }
+    tc::mbar_init(&lo_full[0], 4);
+    tc::mbar_init(&lo_full[1], 4);
+    tc::mbar_init(drain, 1);
+    *s_fail = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == 1) tc::tmem_alloc(tmem_slot, TMEM_COLS);
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tc::tma_prefetch_desc(&h0_map);
+      for (int i = i0; i < i1; ++i) {
+        const int k = i - i0, st = k % NSTAGE;
+        if (!tc::mbar_wait(&a_empty[st], ((k / NSTAGE) & 1) ^ 1, err)) break;
+        const int c = i / t.n_tiles, j = i % t.n_tiles;
+        const int row0 = (c * a.H + j * hpt) * P;
+        tc::mbar_arrive_expect_tx(&a_full[st], (uint32_t)(nblk * ROWS * 128));
+        for (int b = 0; b < nblk; ++b)
+          tc::tma_load_2d(sA + st * TILE_BYTES + b * ROWS * 128, &h0_map, &a_full[st], b * 32, row0);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
+      const uint32_t idesc = idesc_tf32(ROWS, NT);
+      const uint32_t b_base = tc::smem_u32(sB);
+      for (int i = i0; i < i1; ++i) {
+        const int k = i - i0, st = k % NSTAGE, db = k & 1;
+        // accumulator db is free once the epilogue of tile k - 2 has read it
+        if (k >= 2 && !tc::mbar_wait(&d_free[db], ((k >> 1) - 1) & 1, err)) break;
+        if (!tc::mbar_wait(&lo_full[k & 1], (k >> 1) & 1, err)) break;
+        tc::tc_fence_after();
+        const uint32_t hi = tc::smem_u32(sA + st * TILE_BYTES);
+        const uint32_t lo = tmem + (uint32_t)(128 * (k & 1));
+        const uint32_t d = tmem + 256u + (uint32_t)(db * NT);
+#pragma unroll
+        for (int kb = 0; kb < NMAX / 8; ++kb) {
+          const uint32_t aoff = (uint32_t)((kb >> 2) * ROWS * 128 + (kb & 3) * 32);
+          const uint64_t bdesc = tc::sdesc_k128(b_base + (uint32_t)((kb >> 2) * NT * 128 + (kb & 3) * 32));
+          mma_tf32(d, tc::sdesc_k128(hi + aoff), bdesc, idesc, kb > 0);
+          mma_tf32_ts(d, lo + (uint32_t)(kb * 8), bdesc, idesc, 1u);
+        }
+        tc::mma_commit(&acc_full[db]);
+        tc::mma_commit(&a_empty[st]);
+      }
+      tc::mma_commit(drain);
+      tc::mbar_wait(drain, 0, err);
+    }
+  } else {
+    // ------------------------------------------------------------ transform groups
+    const int g = (warp - 2) >> 2;              // group: tiles k with k % 2 == g
+    const int tid = threadIdx.x - 64 - 128 * g; // 0..127 within the group
+    const int quarter = warp & 3;                // TMEM lanes of this warp
+    const int row = quarter * 32 + lane;         // the state row (TMEM lane) of this thread
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const int hl = row / P, p = row % P;
+    const int gw = (warp - 2) & 3;               // warp within the group
+    const TDT* dtp = (const TDT*)a.dt;
+    const bf16* xg = (const bf16*)a.x;
+    const bf16* Bg = (const bf16*)a.B;
+    const bf16* Cg = (const bf16*)a.Cm;
+    float* gX = sX + g * KMAX * ROWS;
+    float* gL = sL + g * HPT_MAX * KMAX * KMAX;  // [head][s][t]
+    float* gE = sE + g * HPT_MAX * (KMAX + 1);
+    float* gCB = sCB + g * KMAX * KMAX;
+    float* gDt = sDt + g * 2 * HPT_MAX * KMAX;   // dt [head][t], then cum [head][t]
+    int c_prev = -1;
+    auto gsync = [&]() {
+      if (g == 0) asm volatile("bar.sync 1, 128;" ::: "memory");
+      else asm volatile("bar.sync 2, 128;" ::: "memory");
+    };
+
+    // The group's warps pass the same named barriers in the same order; a wait that
+    // gives up sets s_fail, and the group leaves the loop after its next barrier.
+    for (int i = i0 + g; i < i1; i += 2) {
+      const int k = i - i0, st = k % NSTAGE;
+      const int c = i / t.n_tiles, j = i % t.n_tiles;
+      const bool new_req = c != c_prev;
+      // the tile's global loads first: x of this thread's row at every position (rows
+      // past K re-read row K - 1 and are zeroed below), and (first warp, lane hh * 16 +
+      // tt) dt of head hh at position tt
+      uint16_t xv[KMAX];
+      {
+        const bf16* xr = xg + (size_t)c * K * a.x_rs + (size_t)(j * hpt) * P + row;
+#pragma unroll
+        for (int tt = 0; tt < KMAX; ++tt) xv[tt] = ldg_u16(xr + (size_t)(tt < K ? tt : K - 1) * a.x_rs);
+      }
+      const int dh = tid >> 4, dtt = tid & 15;
+      const bool dlive = tid < 32 && dh < hpt && dtt < K;
+      const int dhead = j * hpt + (dh < hpt ? dh : 0);
+      uint32_t draw_bits = 0, dA_bits = 0, dD_bits = 0, dbias_bits = 0;
+      if (dlive) {
+        const TDT* dp = dtp + (size_t)(c * K + dtt) * a.dt_rs + dhead;
+        draw_bits = sizeof(TDT) == 2 ? (uint32_t)ldg_u16(dp) : ldg_u32(dp);
+        dA_bits = ldg_u32(a.A + dhead);
+        dD_bits = ldg_u32(a.D + dhead);
+        if (a.dt_bias) dbias_bits = ldg_u32(a.dt_bias + dhead);
+      }
+      // the state tile has landed; for a new request also the MMAs of the previous tile
+      // (the last reader of the C^T operand) are done
+      bool ok = tc::mbar_wait(&a_full[st], (k / NSTAGE) & 1, err);
+      if (ok && new_req && k >= 1) ok = tc::mbar_wait(&acc_full[(k - 1) & 1], ((k - 1) >> 1) & 1, err);
+      if (!ok) *s_fail = 1;
+      gsync();
+      if (*s_fail) break;
+      tc::tc_fence_after();
+      if (new_req) {
+        // C^T operand: row tt (position) of 128-byte column blocks, zero past K
+        constexpr int PER = NT * NMAX / 4 / 128;  // float4 entries per thread
+        uint2 rw[PER];
+#pragma unroll
+        for (int q = 0; q < PER; ++q) {
+          const int e = tid + 128 * q, tt = e / (NMAX / 4), n4 = (e % (NMAX / 4)) * 4;
+          rw[q] = tt < K ? *(const uint2*)(Cg + (size_t)(c * K + tt) * a.bc_rs + n4) : make_uint2(0u, 0u);
+        }
+#pragma unroll
+        for (int q = 0; q < PER; ++q) {
+          const int e = tid + 128 * q, tt = e / (NMAX / 4), n4 = (e % (NMAX / 4)) * 4;
+          const float2 lo2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&rw[q].x));
+          const float2 hi2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&rw[q].y));
+          const int ch = (n4 & 31) >> 2;
+          *(float4*)(sB + (n4 >> 5) * NT * 128 + tt * 128 + ((ch ^ (tt & 7)) << 4)) =
+              make_float4(lo2.x, lo2.y, hi2.x, hi2.y);
+        }
+        c_prev = c;
+      }
+      // this thread's state row: round to tf32 in place (hi), lo = S - hi into the
+      // group's TMEM buffer (free: the group's previous tile finished its MMAs)
+      {
+        uint8_t* rowp = sA + st * TILE_BYTES + row * 128;
+#pragma unroll
+        for (int cb = 0; cb < NMAX / 32; ++cb) {
+          uint4 v[8];
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) v[ch] = *(const uint4*)(rowp + cb * ROWS * 128 + ((ch ^ (row & 7)) << 4));
+          uint32_t lo[32];
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) {
+            const uint32_t h0 = tf32_hi(v[ch].x), h1 = tf32_hi(v[ch].y);
+            const uint32_t h2 = tf32_hi(v[ch].z), h3 = tf32_hi(v[ch].w);
+            lo[4 * ch + 0] = __float_as_uint(__uint_as_float(v[ch].x) - __uint_as_float(h0));
+            lo[4 * ch + 1] = __float_as_uint(__uint_as_float(v[ch].y) - __uint_as_float(h1));
+            lo[4 * ch + 2] = __float_as_uint(__uint_as_float(v[ch].z) - __uint_as_float(h2));
+            lo[4 * ch + 3] = __float_as_uint(__uint_as_float(v[ch].w) - __uint_as_float(h3));
+            v[ch] = make_uint4(h0, h1, h2, h3);
+          }
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) *(uint4*)(rowp + cb * ROWS * 128 + ((ch ^ (row & 7)) << 4)) = v[ch];
+          tc::tmem_st32_nowait(tmem + lane_off + (uint32_t)(128 * g + 32 * cb), lo);
+        }
+        tc::tmem_wait_st();
+      }
+      gsync();  // the C^T operand of a new request is complete
+      if (new_req) {
+        // C . B^T of the request (entries s <= t): warp gw takes s = gw mod 4; lane l
+        // holds n = 4l .. 4l + 3 of B_s (registers) and reads those of C_t
+        for (int ss = gw; ss < K; ss += 4) {
+          const uint2 r = *(const uint2*)(Bg + (size_t)(c * K + ss) * a.bc_rs + 4 * lane);
+          const float2 b01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.x));
+          const float2 b23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.y));
+          const int n4 = 4 * lane, ch = (n4 & 31) >> 2;
+          for (int tt = ss; tt < K; ++tt) {
+            const float4 cv = *(const float4*)(sB + (n4 >> 5) * NT * 128 + tt * 128 + ((ch ^ (tt & 7)) << 4));
+            float v = cv.x * b01.x;
+            v = fmaf(cv.y, b01.y, v);
+            v = fmaf(cv.z, b23.x, v);
+            v = fmaf(cv.w, b23.y, v);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+            if (lane == 0) gCB[tt * KMAX + ss] = v;
+          }
+        }
+      }
+      // the tile's heads: dt, cum = inclusive scan of dt A_h (segmented, 16 lanes), exp(cum)
+      if (tid < 32) {
+        float d = sizeof(TDT) == 2 ? __bfloat162float(__ushort_as_bfloat16((unsigned short)draw_bits))
+                                   : __uint_as_float(draw_bits);
+        if (dlive && a.dt_bias) d = softplus(d + __uint_as_float(dbias_bits));
+        const float dA = __uint_as_float(dA_bits), dD = __uint_as_float(dD_bits);
+        float cum = dlive ? d * dA : 0.f;
+#pragma unroll
+        for (int o = 1; o < 16; o <<= 1) {
+          const float v = __shfl_up_sync(0xffffffffu, cum, o, 16);
+          if (dtt >= o) cum += v;
+        }
+        if (dlive) {
+          gDt[dh * KMAX + dtt] = d;
+          gDt[(HPT_MAX + dh) * KMAX + dtt] = cum;
+          gE[dh * (KMAX + 1) + dtt] = expf(cum);
+          if (dtt == 0) gE[dh * (KMAX + 1) + KMAX] = dD;
+        }
+      }
+      // x of this thread's row (zero past K)
+#pragma unroll
+      for (int tt = 0; tt < KMAX; ++tt)
+        gX[tt * ROWS + row] = tt < K ? __bfloat162float(__ushort_as_bfloat16((unsigned short)xv[tt])) : 0.f;
+      gsync();
+      // L^T[s][t] = (C_t . B_s) exp(cum_t - cum_s) dt_s for s <= t, else 0: entry
+      // e = (head, t, s) of a 2 x 16 x 16 grid, four per thread, loads first
+      {
+        constexpr int PER = HPT_MAX * KMAX * KMAX / 128;
+        float cb[PER], ct[PER], cs[PER], dts[PER];
+        bool live[PER];
+#pragma unroll
+        for (int q = 0; q < PER; ++q) {
+          const int e = tid + 128 * q, hh = e >> 8, tt = (e >> 4) & 15, ss = e & 15;
+          live[q] = hh < hpt && tt < K && ss <= tt;
+          cb[q] = gCB[tt * KMAX + ss];
+          ct[q] = gDt[(HPT_MAX + hh) * KMAX + tt];
+          cs[q] = gDt[(HPT_MAX + hh) * KMAX + ss];
+          dts[q] = gDt[hh * KMAX + ss];
+        }
+#pragma unroll
+        for (int q = 0; q < PER; ++q) {
+          const int e = tid + 128 * q, hh = e >> 8, tt = (e >> 4) & 15, ss = e & 15;
+          gL[(hh * KMAX + ss) * KMAX + tt] = live[q] ? cb[q] * expf(ct[q] - cs[q]) * dts[q] : 0.f;
+        }
+      }
+      // hi and C^T were written by threads and lo by tcgen05.st; the MMA reads them
+      tc::fence_proxy_async();
+      tc::tc_fence_before();
+      gsync();
+      if (lane == 0) tc::mbar_arrive(&lo_full[g]);
+
+      // epilogue, once the tile's MMAs are done:
+      // y_t = exp(cum_t) (C S^T)_t + sum_{s<=t} L_ts x_s + D_h x_t
+      ok = tc::mbar_wait(&acc_full[g], (k >> 1) & 1, err);
+      if (!ok) {
+        *s_fail = 1;
+        continue;  // the group leaves after its next barrier
+      }
+      tc::tc_fence_after();
+      float dv[NT];
+      tc::tmem_ld16(tmem + lane_off + 256u + (uint32_t)(g * NT), dv);
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&d_free[g]);
+      const int h = j * hpt + hl;
+      const float* LTh = gL + hl * KMAX * KMAX;  // [s][t]
+      const float* Eh = gE + hl * (KMAX + 1);
+      float xs[KMAX], acc[KMAX];
+#pragma unroll
+      for (int s2 = 0; s2 < KMAX; ++s2) xs[s2] = gX[s2 * ROWS + row];
+#pragma unroll
+      for (int tt = 0; tt < KMAX; ++tt) acc[tt] = fmaf(Eh[tt], dv[tt], Eh[KMAX] * xs[tt]);
+#pragma unroll
+      for (int s2 = 0; s2 < KMAX; ++s2)
+#pragma unroll
+        for (int t4 = (s2 & ~3); t4 < KMAX; t4 += 4) {
+          const float4 l4 = *(const float4*)(LTh + s2 * KMAX + t4);  // zero above the diagonal
+          acc[t4 + 0] = fmaf(l4.x, xs[s2], acc[t4 + 0]);
+          acc[t4 + 1] = fmaf(l4.y, xs[s2], acc[t4 + 1]);
+          acc[t4 + 2] = fmaf(l4.z, xs[s2], acc[t4 + 2]);
+          acc[t4 + 3] = fmaf(l4.w, xs[s2], acc[t4 + 3]);
+        }
+      float* yr = a.y + (size_t)c * K * a.y_rs + (size_t)h * P + p;
+#pragma unroll
+      for (int tt = 0; tt < KMAX; ++tt)
+        if (tt < K) yr[(size_t)tt * a.y_rs] = acc[tt];
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn_ssd() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)p;
+    tried = true;
+  }
+  return fn;
+}
+
+template <typename TDT>
+bool launch_ssd_tc(const SsdArgs& a, cudaStream_t s) {
+  static bool attr_set[64] = {};
+  static int n_sm[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    if (cudaFuncSetAttribute(ssd_tc_kernel<TDT>, cudaFuncAttributeMaxDynamicSharedMemorySize, SsdTcLay::SMEM) !=
+        cudaSuccess)
+      return false;
+    cudaDeviceGetAttribute(&n_sm[dev], cudaDevAttrMultiProcessorCount, dev);
+    attr_set[dev] = true;
+  }
+  EncodeTiledFn fn = encode_fn_ssd();
+  if (!fn) return false;
+  CUtensorMap map;
+  cuuint64_t dims[2] = {(cuuint64_t)a.N, (cuuint64_t)a.C * a.H * a.P};
+  cuuint64_t strides[1] = {(cuuint64_t)a.N * 4};
+  cuuint32_t box[2] = {32, ROWS};
+  cuuint32_t estr[2] = {1, 1};
+  if (fn(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(a.h0), dims, strides, box, estr,
+         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  SsdTcArgs t;
+  t.a = a;
+  t.err = device_error_word();
+  t.hpt = ROWS / a.P;
+  t.n_tiles = a.H / t.hpt;
+  t.n_items = a.C * t.n_tiles;
+  const int sms = dev < 64 && n_sm[dev] > 0 ? n_sm[dev] : 148;
+  const int grid = t.n_items < sms ? t.n_items : sms;
+  ssd_tc_kernel<TDT><<<grid, THREADS, SsdTcLay::SMEM, s>>>(map, t);
+  note_launch();
+  return true;
+}
+
+}  // namespace
+
+bool ssd_tc_supported(int dtype, const SsdArgs& a) {
+  if (dtype != HSPEC_DTYPE_BF16 || !a.h0 || a.hK || a.Q != a.K) return false;
+  if (a.K < 1 || a.K > KMAX || a.N != NMAX || a.C < 1) return false;
+  if (a.P < ROWS / HPT_MAX || ROWS % a.P || a.H % (ROWS / a.P)) return false;
+  if (((uintptr_t)a.h0 & 15) || (long)a.C * a.H * a.P > 0x7fffffffL) return false;
+  if (((uintptr_t)a.B & 7) || ((uintptr_t)a.Cm & 7) || (a.bc_rs & 3)) return false;  // 8-byte loads
+  return true;
+}
+
+bool ssd_tc_launch(const SsdArgs& a, cudaStream_t s) {
+  return a.dt_bias ? launch_ssd_tc<bf16>(a, s) : launch_ssd_tc<float>(a, s);
+}
+
+}  // namespace hspec

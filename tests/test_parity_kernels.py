@@ -84,6 +84,21 @@ def test_ssd_scan_matches_sequential_recurrence(H, cuda, name):
     assert_close(to_np(hK), ref_h, "f32", f"ssd hK {name}")
 
 
+@pytest.mark.parametrize("name,C,K", [("llama_c32", 8, 16), ("qwen_c128", 3, 16), ("llama_c32", 160, 16),
+                                     ("llama_c32", 5, 7), ("qwen_c128", 2, 1)])
+def test_ssd_scan_readout_without_final_state(H, cuda, name, C, K):
+    # Without the final state, one bf16 chunk of K <= 16 positions is evaluated with the
+    # state readout on the tensor cores (tf32 hi + lo split of the fp32 state): it must
+    # still meet the fp32 bound against the sequential recurrence.
+    sh = I.WORKLOADS[name].shapes
+    inp = I.make_ssd_inputs(sh, C, K, 31 + C, cuda)
+    y, _ = run_ssd(H, sh, inp, K, want_state=False)
+    rows = sample_requests(C, min(C, 6), seed=C)
+    ref_y = oracle.ssd_scan(host(inp["x"])[rows], host(inp["dt"])[rows], host(inp["A"]), host(inp["B"])[rows],
+                               host(inp["Cm"])[rows], host(inp["D"]), host(inp["h0"])[rows], want_state=False)
+    assert_close(to_np(y[rows]), ref_y, "f32", f"ssd readout {name} C={C} K={K}")
+
+
 @pytest.mark.parametrize("K,chunks", [(16, (1, 4, 5, 8, 16)), (32, (8, 16, 32)), (7, (3, 7)), (1, (1,))])
 def test_ssd_chunk_length_is_only_an_evaluation_order(H, cuda, K, chunks):
     sh = I.LLAMA
