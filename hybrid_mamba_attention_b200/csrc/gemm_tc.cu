@@ -1,18 +1,22 @@
 // bf16 GEMM on the 5th-generation tensor cores: out = epi(A . B^T), A [M,K] and
 // B [N,K] row-major (K-major) bf16, fp32 accumulation in tensor memory.
 //
-// One CTA computes a 128 x 256 output tile (SwiGLU: 128 x 128 outputs from a
-// 128 x (128 gate + 128 up) accumulator) with three roles:
+// Persistent kernel, one CTA per SM; the output is cut into 128 x 256 tiles (SwiGLU:
+// 128 x 128 outputs from a 128 x (128 gate + 128 up) accumulator), numbered M-tile
+// fastest, and CTA b takes tiles b, b + grid, ... so that the CTAs working on one
+// weight tile at a time are resident together and the weight is read from HBM once.
+// Three roles:
 //   warp 0      TMA producer: streams 128x64 A and 256x64 B tiles (128-byte
-//               swizzle) through a 4-stage shared-memory ring of mbarriers;
-//   warp 1      allocates 256 TMEM columns; one lane issues tcgen05.mma
-//               (M=128, N=256, K=16, four per 64-wide stage) and commits each
-//               stage back to the producer, then the finished accumulator;
-//   warps 2..5  epilogue: tcgen05.ld of their 32-lane quarter of TMEM, then the
-//               fused epilogue (store, residual add, SwiGLU, per-row argmax).
+//               swizzle) through a 4-stage shared-memory ring of mbarriers, on
+//               from one output tile to the next;
+//   warp 1      allocates 512 TMEM columns (two 256-column accumulators); one lane
+//               issues tcgen05.mma (M=128, N=256, K=16, four per 64-wide stage),
+//               commits each stage back to the producer and each finished
+//               accumulator to the epilogue;
+//   warps 2..5  epilogue: tcgen05.ld of their 32-lane quarter of TMEM, then the fused
+//               epilogue (store, residual add, SwiGLU, per-row argmax), while the
+//               next tile accumulates into the other TMEM buffer.
 // Rows/columns beyond M/N are zero-filled by TMA and skipped by the epilogue.
-// Grids run M-tiles fastest so that the CTAs sharing one weight tile are resident
-// together and the weight is read from HBM once.
 #include <mutex>
 #include <stdint.h>
 
@@ -31,7 +35,7 @@ constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2, B_BYTES = BN * BK * 2, STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 constexpr int THREADS = 192;
-constexpr uint32_t TMEM_COLS = 256;
+constexpr uint32_t TMEM_COLS = 512;  // two accumulators of BN columns
 
 template <int EPI>
 __global__ void __launch_bounds__(THREADS, 1)
@@ -42,13 +46,14 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint8_t* smem = smem_raw + (((raw + 1023) & ~1023u) - raw);
   uint64_t* full = (uint64_t*)(smem + STAGES * STAGE_BYTES);
   uint64_t* empty = full + STAGES;
-  uint64_t* acc_full = empty + STAGES;
-  uint32_t* tmem_slot = (uint32_t*)(acc_full + 1);
+  uint64_t* acc_full = empty + STAGES;   // [2] accumulator b holds a finished tile
+  uint64_t* acc_empty = acc_full + 2;    // [2] the epilogue has read accumulator b
+  uint32_t* tmem_slot = (uint32_t*)(acc_empty + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * BM;
   const int ncols_out = (EPI == kEpiSwiGLU) ? BN / 2 : BN;
-  const int n0 = blockIdx.y * ncols_out;
+  const int n_mt = (g.M + BM - 1) / BM;
+  const int n_tiles = n_mt * ((g.N + ncols_out - 1) / ncols_out);
   const int num_k = (g.K + BK - 1) / BK;
 
   if (threadIdx.x == 0) {
@@ -56,7 +61,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc::mbar_init(&full[s], 1);
       tc::mbar_init(&empty[s], 1);
     }
-    tc::mbar_init(acc_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(&acc_full[b], 1);
+      tc::mbar_init(&acc_empty[b], 4);
+    }
     tc::fence_mbar_init();
   }
   if (warp == 1) tc::tmem_alloc(tmem_slot, TMEM_COLS);
@@ -70,116 +78,134 @@ __global__ void __launch_bounds__(THREADS, 1)
     tc::tma_prefetch_desc(&tmA);
     tc::tma_prefetch_desc(&tmB);
     if (EPI == kEpiSwiGLU) tc::tma_prefetch_desc(&tmB2);
-    for (int kt = 0; kt < num_k; ++kt) {
-      const int s = kt % STAGES;
-      const uint32_t ph = (kt / STAGES) & 1;
-      if (!tc::mbar_wait(&empty[s], ph ^ 1, err)) break;
-      uint8_t* sa = smem + s * STAGE_BYTES;
-      uint8_t* sb = sa + A_BYTES;
-      tc::mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
-      tc::tma_load_2d(sa, &tmA, &full[s], kt * BK, m0);
-      if (EPI == kEpiSwiGLU) {
-        tc::tma_load_2d(sb, &tmB, &full[s], kt * BK, n0);
-        tc::tma_load_2d(sb + B_BYTES / 2, &tmB2, &full[s], kt * BK, n0);
-      } else {
-        tc::tma_load_2d(sb, &tmB, &full[s], kt * BK, n0);
+    int it = 0;  // stage-ring position, continued across tiles
+    bool ok = true;
+    for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+      const int m0 = (t % n_mt) * BM, n0 = (t / n_mt) * ncols_out;
+      for (int kt = 0; kt < num_k; ++kt, ++it) {
+        const int s = it % STAGES;
+        if (!(ok = tc::mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, err))) break;
+        uint8_t* sa = smem + s * STAGE_BYTES;
+        uint8_t* sb = sa + A_BYTES;
+        tc::mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
+        tc::tma_load_2d(sa, &tmA, &full[s], kt * BK, m0);
+        if (EPI == kEpiSwiGLU) {
+          tc::tma_load_2d(sb, &tmB, &full[s], kt * BK, n0);
+          tc::tma_load_2d(sb + B_BYTES / 2, &tmB2, &full[s], kt * BK, n0);
+        } else {
+          tc::tma_load_2d(sb, &tmB, &full[s], kt * BK, n0);
+        }
       }
     }
   } else if (warp == 1 && lane == 0) {
     // ---------------------------------------------------------- MMA issuer
     constexpr uint32_t idesc = tc::idesc_bf16_f32(BM, BN);
     bool ok = true;
-    for (int kt = 0; kt < num_k && ok; ++kt) {
-      const int s = kt % STAGES;
-      const uint32_t ph = (kt / STAGES) & 1;
-      ok = tc::mbar_wait(&full[s], ph, err);
-      if (!ok) break;
+    int it = 0, lt = 0;
+    for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++lt) {
+      const int b = lt & 1;
+      // accumulator b is free once the epilogue has read the tile two back
+      if (!(ok = tc::mbar_wait(&acc_empty[b], ((lt >> 1) & 1) ^ 1, err))) break;
       tc::tc_fence_after();
-      const uint32_t sa = tc::smem_u32(smem + s * STAGE_BYTES);
-      const uint32_t sb = sa + A_BYTES;
+      const uint32_t d = tmem + (uint32_t)(b * BN);
+      for (int kt = 0; kt < num_k; ++kt, ++it) {
+        const int s = it % STAGES;
+        if (!(ok = tc::mbar_wait(&full[s], (it / STAGES) & 1, err))) break;
+        tc::tc_fence_after();
+        const uint32_t sa = tc::smem_u32(smem + s * STAGE_BYTES);
+        const uint32_t sb = sa + A_BYTES;
 #pragma unroll
-      for (int k = 0; k < BK / 16; ++k) {
-        tc::mma_bf16(tmem, tc::sdesc_k128(sa + k * 32), tc::sdesc_k128(sb + k * 32), idesc,
-                     (kt | k) != 0);
+        for (int k = 0; k < BK / 16; ++k) {
+          tc::mma_bf16(d, tc::sdesc_k128(sa + k * 32), tc::sdesc_k128(sb + k * 32), idesc, (kt | k) != 0);
+        }
+        tc::mma_commit(&empty[s]);
       }
-      tc::mma_commit(&empty[s]);
+      tc::mma_commit(&acc_full[b]);
     }
-    tc::mma_commit(acc_full);
   } else if (warp >= 2) {
     // ---------------------------------------------------------- epilogue
     const int quarter = warp & 3;  // TMEM lanes this warp may access
     const int row = quarter * 32 + lane;
-    const int m = m0 + row;
-    const bool ok = tc::mbar_wait(acc_full, 0, err);
-    __syncwarp();
-    tc::tc_fence_after();
-    const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16);
-    float v[32], u[32];
-    if (EPI == kEpiArgmax) {
-      float best = -INFINITY;
-      int bidx = 0x7fffffff;
-      for (int c = 0; c < BN; c += 32) {
-        tc::tmem_ld32(taddr + c, v);
+    int lt = 0;
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++lt) {
+      const int b = lt & 1;
+      const int m0 = (t % n_mt) * BM, n0 = (t / n_mt) * ncols_out, ntile = t / n_mt;
+      const int m = m0 + row;
+      const bool ok = tc::mbar_wait(&acc_full[b], (lt >> 1) & 1, err);
+      __syncwarp();
+      tc::tc_fence_after();
+      const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(b * BN);
+      float v[32], u[32];
+      if (EPI == kEpiArgmax) {
+        float best = -INFINITY;
+        int bidx = 0x7fffffff;
+        for (int c = 0; c < BN; c += 32) {
+          tc::tmem_ld32(taddr + c, v);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int n = n0 + c + i;
-          if (n < g.N && v[i] > best) best = v[i], bidx = n;
-        }
-      }
-      if (ok && m < g.M) {
-        g.pval[(size_t)m * g.n_parts + blockIdx.y] = best;
-        g.pidx[(size_t)m * g.n_parts + blockIdx.y] = bidx;
-      }
-    } else {
-      for (int c = 0; c < ncols_out; c += 32) {
-        tc::tmem_ld32(taddr + c, v);
-        if (EPI == kEpiSwiGLU) tc::tmem_ld32(taddr + BN / 2 + c, u);
-        if (!ok || m >= g.M) continue;
-        const int nb = n0 + c;
-        if (EPI == kEpiStore && g.out_f32) {
-          float* o = (float*)g.out + (size_t)m * g.ldo + nb;
-          if (nb + 32 <= g.N && (((uintptr_t)o) & 15) == 0) {
-#pragma unroll
-            for (int i = 0; i < 32; i += 4) *(float4*)(o + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-          } else {
-            for (int i = 0; i < 32; ++i)
-              if (nb + i < g.N) o[i] = v[i];
-          }
-        } else if (EPI == kEpiResid) {
-          float* o = (float*)g.out + (size_t)m * g.ldo + nb;
-          if (nb + 32 <= g.N && (((uintptr_t)o) & 15) == 0) {
-#pragma unroll
-            for (int i = 0; i < 32; i += 4) {
-              float4 x = *(float4*)(o + i);
-              x.x += v[i], x.y += v[i + 1], x.z += v[i + 2], x.w += v[i + 3];
-              *(float4*)(o + i) = x;
-            }
-          } else {
-            for (int i = 0; i < 32; ++i)
-              if (nb + i < g.N) o[i] += v[i];
-          }
-        } else {
-          if (EPI == kEpiSwiGLU) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = silu(v[i]) * u[i];
-          }
-          bf16* o = (bf16*)g.out + (size_t)m * g.ldo + nb;
-          if (nb + 32 <= g.N && (((uintptr_t)o) & 15) == 0) {
-#pragma unroll
-            for (int i = 0; i < 32; i += 8) {
-              __align__(16) bf16 t[8];
-#pragma unroll
-              for (int k = 0; k < 8; ++k) t[k] = __float2bfloat16_rn(v[i + k]);
-              *(uint4*)(o + i) = *(uint4*)t;
-            }
-          } else {
-            for (int i = 0; i < 32; ++i)
-              if (nb + i < g.N) o[i] = __float2bfloat16_rn(v[i]);
+          for (int i = 0; i < 32; ++i) {
+            const int n = n0 + c + i;
+            if (n < g.N && v[i] > best) best = v[i], bidx = n;
           }
         }
+        if (ok && m < g.M) {
+          g.pval[(size_t)m * g.n_parts + ntile] = best;
+          g.pidx[(size_t)m * g.n_parts + ntile] = bidx;
+        }
+      } else {
+        for (int c = 0; c < ncols_out; c += 32) {
+          tc::tmem_ld32(taddr + c, v);
+          if (EPI == kEpiSwiGLU) tc::tmem_ld32(taddr + BN / 2 + c, u);
+          if (!ok || m >= g.M) continue;
+          const int nb = n0 + c;
+          if (EPI == kEpiStore && g.out_f32) {
+            float* o = (float*)g.out + (size_t)m * g.ldo + nb;
+            if (nb + 32 <= g.N && (((uintptr_t)o) & 15) == 0) {
+#pragma unroll
+              for (int i = 0; i < 32; i += 4) *(float4*)(o + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+            } else {
+              for (int i = 0; i < 32; ++i)
+                if (nb + i < g.N) o[i] = v[i];
+            }
+          } else if (EPI == kEpiResid) {
+            float* o = (float*)g.out + (size_t)m * g.ldo + nb;
+            if (nb + 32 <= g.N && (((uintptr_t)o) & 15) == 0) {
+#pragma unroll
+              for (int i = 0; i < 32; i += 4) {
+                float4 x = *(float4*)(o + i);
+                x.x += v[i], x.y += v[i + 1], x.z += v[i + 2], x.w += v[i + 3];
+                *(float4*)(o + i) = x;
+              }
+            } else {
+              for (int i = 0; i < 32; ++i)
+                if (nb + i < g.N) o[i] += v[i];
+            }
+          } else {
+            if (EPI == kEpiSwiGLU) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) v[i] = silu(v[i]) * u[i];
+            }
+            bf16* o = (bf16*)g.out + (size_t)m * g.ldo + nb;
+            if (nb + 32 <= g.N && (((uintptr_t)o) & 15) == 0) {
+#pragma unroll
+              for (int i = 0; i < 32; i += 8) {
+                __align__(16) bf16 t8[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) t8[k] = __float2bfloat16_rn(v[i + k]);
+                *(uint4*)(o + i) = *(uint4*)t8;
+              }
+            } else {
+              for (int i = 0; i < 32; ++i)
+                if (nb + i < g.N) o[i] = __float2bfloat16_rn(v[i]);
+            }
+          }
+        }
       }
+      // accumulator b may take the tile after next
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&acc_empty[b]);
+      if (!ok) break;
     }
-    tc::tc_fence_before();
   }
   __syncthreads();
   if (warp == 1) {
@@ -224,6 +250,7 @@ bool make_map(CUtensorMap* m, const void* base, long rows, long cols, long ld, i
 template <int EPI>
 bool launch_tc(const GemmArgs& g, cudaStream_t s, int* err) {
   static bool attr_set[64] = {};
+  static int n_sm[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
@@ -232,6 +259,7 @@ bool launch_tc(const GemmArgs& g, cudaStream_t s, int* err) {
       set_error("cudaFuncSetAttribute(gemm_tc_kernel) failed");
       return false;
     }
+    cudaDeviceGetAttribute(&n_sm[dev], cudaDevAttrMultiProcessorCount, dev);
     attr_set[dev] = true;
   }
   CUtensorMap ta, tb, tb2;
@@ -244,7 +272,9 @@ bool launch_tc(const GemmArgs& g, cudaStream_t s, int* err) {
     return false;
   }
   const int ncols_out = (EPI == kEpiSwiGLU) ? BN / 2 : BN;
-  dim3 grid(cdiv(g.M, BM), cdiv(g.N, ncols_out));
+  const long n_tiles = (long)cdiv(g.M, BM) * cdiv(g.N, ncols_out);
+  const int sms = dev < 64 && n_sm[dev] > 0 ? n_sm[dev] : 148;
+  const int grid = n_tiles < sms ? (int)n_tiles : sms;
   gemm_tc_kernel<EPI><<<grid, THREADS, SMEM_BYTES, s>>>(ta, tb, tb2, g, err);
   note_launch();
   return true;
