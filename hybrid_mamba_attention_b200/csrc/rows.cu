@@ -42,6 +42,117 @@ __global__ void rmsnorm_kernel(const float* __restrict__ x, const float* __restr
   for (int i = threadIdx.x; i < n; i += blockDim.x) o[i] = from_f<T>(row[i] * inv * w[i]);
 }
 
+// Vectorised forms for rows of n <= 4 * kRowThreads * kV4 values, n % 4 == 0: one
+// pass over global memory, the row held in registers (float4 loads, 8- or 16-byte
+// stores).  Same arithmetic per element as the scalar kernels above.
+constexpr int kV4 = 8;
+
+__device__ __forceinline__ void store4(bf16* o, float a, float b, float c, float d) {
+  __nv_bfloat162 lo = __floats2bfloat162_rn(a, b), hi = __floats2bfloat162_rn(c, d);
+  uint2 u;
+  u.x = *reinterpret_cast<uint32_t*>(&lo);
+  u.y = *reinterpret_cast<uint32_t*>(&hi);
+  *(uint2*)o = u;
+}
+__device__ __forceinline__ void store4(float* o, float a, float b, float c, float d) {
+  *(float4*)o = make_float4(a, b, c, d);
+}
+__device__ __forceinline__ float4 load4(const bf16* p) {
+  const uint2 u = *(const uint2*)p;
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+__device__ __forceinline__ float4 load4(const float* p) { return *(const float4*)p; }
+
+template <typename T>
+__global__ void __launch_bounds__(kRowThreads) rmsnorm_v4_kernel(const float* __restrict__ x,
+                                                                 const float* __restrict__ w,
+                                                                 T* __restrict__ out, int n, float eps) {
+  __shared__ float red[32];
+  const int n4 = n / 4;
+  const float4* row = (const float4*)(x + (size_t)blockIdx.x * n);
+  float4 v[kV4];
+  float ss = 0.f;
+#pragma unroll
+  for (int k = 0; k < kV4; ++k) {
+    const int i = threadIdx.x + k * kRowThreads;
+    v[k] = i < n4 ? row[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+    ss += v[k].x * v[k].x + v[k].y * v[k].y + v[k].z * v[k].z + v[k].w * v[k].w;
+  }
+  ss = block_sum(ss, red);
+  const float inv = 1.f / sqrtf(ss / n + eps);  // correctly rounded: fewer bf16 rounding flips
+  T* o = out + (size_t)blockIdx.x * n;
+#pragma unroll
+  for (int k = 0; k < kV4; ++k) {
+    const int i = threadIdx.x + k * kRowThreads;
+    if (i < n4) {
+      const float4 ww = ((const float4*)w)[i];
+      store4(o + 4 * i, v[k].x * inv * ww.x, v[k].y * inv * ww.y, v[k].z * inv * ww.z, v[k].w * inv * ww.w);
+    }
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kRowThreads) gated_rmsnorm_v4_kernel(const float* __restrict__ y,
+                                                                       const T* __restrict__ z, long z_stride,
+                                                                       const float* __restrict__ w,
+                                                                       T* __restrict__ out, int n, float eps) {
+  __shared__ float red[32];
+  const int n4 = n / 4;
+  const float* yr = y + (size_t)blockIdx.x * n;
+  const T* zr = z + (size_t)blockIdx.x * z_stride;
+  float4 gv[kV4];
+  float ss = 0.f;
+#pragma unroll
+  for (int k = 0; k < kV4; ++k) {
+    const int i = threadIdx.x + k * kRowThreads;
+    if (i < n4) {
+      const float4 yy = ((const float4*)yr)[i];
+      const float4 zz = load4(zr + 4 * i);
+      gv[k] = make_float4(yy.x * silu(zz.x), yy.y * silu(zz.y), yy.z * silu(zz.z), yy.w * silu(zz.w));
+    } else {
+      gv[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    ss += gv[k].x * gv[k].x + gv[k].y * gv[k].y + gv[k].z * gv[k].z + gv[k].w * gv[k].w;
+  }
+  ss = block_sum(ss, red);
+  const float inv = 1.f / sqrtf(ss / n + eps);
+  T* o = out + (size_t)blockIdx.x * n;
+#pragma unroll
+  for (int k = 0; k < kV4; ++k) {
+    const int i = threadIdx.x + k * kRowThreads;
+    if (i < n4) {
+      const float4 ww = ((const float4*)w)[i];
+      store4(o + 4 * i, gv[k].x * inv * ww.x, gv[k].y * inv * ww.y, gv[k].z * inv * ww.z, gv[k].w * inv * ww.w);
+    }
+  }
+}
+
+// Rotate-half RoPE in place with one angle per (row, pair i), shared by all heads:
+// CTA = row; thread t takes pair i = t % (D/2) of heads t / (D/2), + groups, ....
+template <typename T>
+__global__ void __launch_bounds__(kRowThreads) rope_rows_kernel(T* __restrict__ qkv, long row_stride,
+                                                                const int32_t* __restrict__ ctx_lens, int K,
+                                                                int n_heads, int D, double log_theta) {
+  const int half = D / 2, groups = kRowThreads / half;
+  const int t = threadIdx.x, i = t % half, hg = t / half;
+  if (hg >= groups) return;
+  const long m = blockIdx.x;
+  const int c = (int)(m / K), j = (int)(m % K);
+  const double pos = (double)ctx_lens[c] + j;
+  const double ang = pos * exp(-2.0 * i / D * log_theta);
+  double sn, cs;
+  sincos(ang, &sn, &cs);
+  T* row = qkv + m * row_stride;
+  for (int h = hg; h < n_heads; h += groups) {
+    T* v = row + (long)h * D;
+    const double a = to_f(v[i]), b = to_f(v[i + half]);
+    v[i] = from_f<T>((float)(a * cs - b * sn));
+    v[i + half] = from_f<T>((float)(a * sn + b * cs));
+  }
+}
+
 // Mamba-2 output gate: g = y * silu(z), then RMSNorm over the H*P features.
 template <typename T>
 __global__ void gated_rmsnorm_kernel(const float* __restrict__ y, const T* __restrict__ z, long z_stride,
@@ -139,7 +250,11 @@ void rows_to_f32(int dtype, const void* in, float* x, long n, cudaStream_t s) {
 
 void rmsnorm_rows(int dtype, const float* x, const float* w, void* out, int M, int n, float eps,
                   cudaStream_t s) {
-  if (dtype == HSPEC_DTYPE_BF16)
+  const bool v4 = n % 4 == 0 && n <= 4 * kRowThreads * kV4 && !(((uintptr_t)x | (uintptr_t)w | (uintptr_t)out) & 15);
+  if (v4) {
+    if (dtype == HSPEC_DTYPE_BF16) rmsnorm_v4_kernel<bf16><<<M, kRowThreads, 0, s>>>(x, w, (bf16*)out, n, eps);
+    else rmsnorm_v4_kernel<float><<<M, kRowThreads, 0, s>>>(x, w, (float*)out, n, eps);
+  } else if (dtype == HSPEC_DTYPE_BF16)
     rmsnorm_kernel<bf16><<<M, kRowThreads, 0, s>>>(x, w, (bf16*)out, n, eps);
   else
     rmsnorm_kernel<float><<<M, kRowThreads, 0, s>>>(x, w, (float*)out, n, eps);
@@ -148,7 +263,16 @@ void rmsnorm_rows(int dtype, const float* x, const float* w, void* out, int M, i
 
 void gated_rmsnorm_rows(int dtype, const float* y, const void* z, long z_stride, const float* w,
                         void* out, int M, int n, float eps, bool gate, cudaStream_t s) {
-  if (dtype == HSPEC_DTYPE_BF16)
+  const int zb = dtype == HSPEC_DTYPE_BF16 ? 2 : 4;
+  const bool v4 = gate && n % 4 == 0 && n <= 4 * kRowThreads * kV4 && (z_stride * zb) % 16 == 0 &&
+                  !(((uintptr_t)y | (uintptr_t)w | (uintptr_t)out) & 15) && !(((uintptr_t)z) & 7);
+  if (v4) {
+    if (dtype == HSPEC_DTYPE_BF16)
+      gated_rmsnorm_v4_kernel<bf16><<<M, kRowThreads, 0, s>>>(y, (const bf16*)z, z_stride, w, (bf16*)out, n, eps);
+    else
+      gated_rmsnorm_v4_kernel<float><<<M, kRowThreads, 0, s>>>(y, (const float*)z, z_stride, w, (float*)out, n,
+                                                               eps);
+  } else if (dtype == HSPEC_DTYPE_BF16)
     gated_rmsnorm_kernel<bf16><<<M, kRowThreads, 0, s>>>(y, (const bf16*)z, z_stride, w, (bf16*)out, n,
                                                          eps, gate);
   else
@@ -162,7 +286,12 @@ void rope_rows(int dtype, void* qkv, long row_stride, const int32_t* ctx_lens, i
   const long total = (long)C * K * n_heads * (D / 2);
   const int grid = (int)((total + kRowThreads - 1) / kRowThreads);
   const double lt = log((double)theta);
-  if (dtype == HSPEC_DTYPE_BF16)
+  if (D % 2 == 0 && D / 2 <= kRowThreads) {
+    if (dtype == HSPEC_DTYPE_BF16)
+      rope_rows_kernel<bf16><<<C * K, kRowThreads, 0, s>>>((bf16*)qkv, row_stride, ctx_lens, K, n_heads, D, lt);
+    else
+      rope_rows_kernel<float><<<C * K, kRowThreads, 0, s>>>((float*)qkv, row_stride, ctx_lens, K, n_heads, D, lt);
+  } else if (dtype == HSPEC_DTYPE_BF16)
     rope_kernel<bf16><<<grid, kRowThreads, 0, s>>>((bf16*)qkv, row_stride, ctx_lens, K, n_heads, D, lt,
                                                    total);
   else
