@@ -406,7 +406,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       int pv = 0;
       uint64_t idle_since = 0;
       while (pv < *end_tile) {
-        if (tc::mbar_test_wait(&p_full[pv & (NSB - 1)], (pv / NSB) & 1)) {
+        // try_wait suspends the thread until the phase completes or a short time passes
+        // (no busy polling against the softmax warps' issue slots), then end_tile is
+        // checked again
+        if (tc::mbar_try_wait(&p_full[pv & (NSB - 1)], (pv / NSB) & 1)) {
           tc::tc_fence_after();
           const int w = pv & 1, s = pv % NS;
           const bool first = meta[s].local < 2;  // this group's first tile of the item
@@ -480,23 +483,21 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       float sv[TT];
       tc::tmem_ld(tmem + lane_off + L::S_COL(b), sv);
+      // raw scores; the scale (> 0) is applied inside the exponent below
       float mx = -INFINITY;
       if (valid == TT && !(block_tile && a.causal_block)) {
 #pragma unroll
-        for (int j = 0; j < TT; ++j) {
-          sv[j] *= scale_log2;
-          mx = fmaxf(mx, sv[j]);
-        }
+        for (int j = 0; j < TT; ++j) mx = fmaxf(mx, sv[j]);
       } else {
         // causal block: query position jq sees the block keys 0..jq
         const int vis_end = (block_tile && a.causal_block) ? min(valid, jq + 1 - bt * TT) : valid;
 #pragma unroll
         for (int j = 0; j < TT; ++j) {
-          sv[j] = j < vis_end ? sv[j] * scale_log2 : -INFINITY;
+          sv[j] = j < vis_end ? sv[j] : -INFINITY;
           mx = fmaxf(mx, sv[j]);
         }
       }
-      const float m_new = fmaxf(m_used, mx);
+      const float m_new = fmaxf(m_used, mx * scale_log2);  // running max in the exp2 domain
       float alpha = 1.f;
       bool rescale = false;
       if (m_new > m_used + 8.f) {
@@ -513,8 +514,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint32_t pk[TT / 2];
 #pragma unroll
       for (int j = 0; j < TT; j += 2) {
-        const float p0 = exp2f(sv[j] - mu);  // exp2(-inf) = 0 for masked columns
-        const float p1 = exp2f(sv[j + 1] - mu);
+        // p = 2^(s scale - m), one FFMA and one ex2 (flushing results below 2^-126 to
+        // zero); 2^(-inf) = 0 for masked columns
+        const float p0 = tc::ex2_ftz(fmaf(sv[j], scale_log2, -mu));
+        const float p1 = tc::ex2_ftz(fmaf(sv[j + 1], scale_log2, -mu));
         psum += p0 + p1;
         __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
         pk[j / 2] = *reinterpret_cast<uint32_t*>(&h2);
