@@ -510,19 +510,20 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       // with no visible key yet (m = -inf) every s is -inf: subtract 0 so p = 0, not NaN
       const float mu = m_used == -INFINITY ? 0.f : m_used;
-      float psum = 0.f;
+      float2 psum = make_float2(0.f, 0.f);
       uint32_t pk[TT / 2];
+      const float2 sc2 = make_float2(scale_log2, scale_log2), nm2 = make_float2(-mu, -mu);
 #pragma unroll
       for (int j = 0; j < TT; j += 2) {
-        // p = 2^(s scale - m), one FFMA and one ex2 (flushing results below 2^-126 to
-        // zero); 2^(-inf) = 0 for masked columns
-        const float p0 = tc::ex2_ftz(fmaf(sv[j], scale_log2, -mu));
-        const float p1 = tc::ex2_ftz(fmaf(sv[j + 1], scale_log2, -mu));
-        psum += p0 + p1;
-        __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+        // p = 2^(s scale - m): the exponents of a pair in one packed FFMA, then one ex2
+        // each (flushing results below 2^-126 to zero); 2^(-inf) = 0 for masked columns
+        const float2 e = tc::ffma2(make_float2(sv[j], sv[j + 1]), sc2, nm2);
+        const float2 pp = make_float2(tc::ex2_ftz(e.x), tc::ex2_ftz(e.y));
+        psum = tc::fadd2(psum, pp);
+        __nv_bfloat162 h2 = __floats2bfloat162_rn(pp.x, pp.y);
         pk[j / 2] = *reinterpret_cast<uint32_t*>(&h2);
       }
-      l += psum;
+      l += psum.x + psum.y;
       // P over the first half of S_b
       tc::tmem_stu(tmem + lane_off + L::S_COL(b), pk);
       // The group's previous P.V (before O_w may be rescaled).  It is waited for at
