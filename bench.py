@@ -49,7 +49,9 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+    """nvidia-smi clocks and throttle reasons sampled every 50 ms; the summary keeps the
+    samples taken inside the timed region (window()), started early so that nvidia-smi
+    is already sampling when the region begins."""
     FIELDS = ["index", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
               "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
               "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
@@ -58,6 +60,7 @@ class ClockSampler:
         self.dev = device_index
         self.proc = None
         self.lines = []
+        self.t0 = self.t1 = None
 
     def start(self):
         try:
@@ -65,7 +68,7 @@ class ClockSampler:
             target = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={','.join(self.FIELDS)}", "--format=csv,noheader,nounits",
-                 "-lms", "200", "-i", target], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "50", "-i", target], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
         except Exception:
@@ -73,7 +76,10 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.monotonic(), line.strip()))
+
+    def window(self, t0, t1):
+        self.t0, self.t1 = t0, t1
 
     def stop(self):
         if not self.proc:
@@ -86,7 +92,8 @@ class ClockSampler:
         self.thread.join(timeout=2)
         sm, smax, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        inside = [ln for t, ln in self.lines if self.t0 is not None and self.t0 <= t <= self.t1 + 0.05]
+        for ln in inside if inside else [ln for _, ln in self.lines]:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 9:
                 continue
@@ -99,7 +106,7 @@ class ClockSampler:
                 if v.lower().startswith("active"):
                     reasons.add(nm)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "in_timed_region": bool(inside)}
 
 
 def dist_setup(n_gpus: int):
@@ -181,6 +188,15 @@ def step_work(sh, C, K, ctx_lens):
     return w
 
 
+# DRAM bytes (read + write) per algorithmic byte of the paged-attention kernel, from
+# one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum) of the current
+# attn_tc_kernel at Llama-3-8B shapes, C=32, ctx U[512,8192] (682.8 MB for 656.2 MB of
+# K/V; the excess is the split partials).  The step's attention launch is too large
+# to capture; its traffic is this ratio times its algorithmic bytes (traffic grows
+# with the K/V read).  Set to None whenever the kernel changes until re-captured.
+ATTN_TRAFFIC_PER_BYTE = 1.0405
+
+
 def roofline_of(name, work, avg_ms, peaks, traffic=None, sustained=True):
     """hbm- or tensor-bound roofline fraction of one kernel group."""
     fl, by = work["flops"], work["bytes"]
@@ -226,7 +242,7 @@ class StepRunner:
         self.dr.close()
 
 
-def time_steps(runner, steps, warmup, world, profile=False):
+def time_steps(runner, steps, warmup, world, profile=False, clocks=None):
     H = runner.H
     for _ in range(warmup):
         runner.step()
@@ -238,11 +254,14 @@ def time_steps(runner, steps, warmup, world, profile=False):
     n0 = H.hspec_launch_count()
     barrier(world)
     torch.cuda.synchronize()
+    t0 = time.monotonic()
     e0.record(stream)
     for _ in range(steps):
         runner.step()
     e1.record(stream)
     torch.cuda.synchronize()
+    if clocks is not None:
+        clocks.window(t0, time.monotonic())
     barrier(world)
     launches = H.hspec_launch_count() - n0
     prof = H.hspec_profile_read() if profile else {}
@@ -302,11 +321,10 @@ def run_ours(args, rank, world, local):
     torch.cuda.set_device(dev)
     peaks = load_peaks()
     wl = replica_workload(I, I.full_workload(args.C, args.K), rank)
-    runner = StepRunner(H, I, wl, dev)
-
     clocks = ClockSampler(local)
-    clocks.start()
-    ms, launches, prof = time_steps(runner, args.steps, args.warmup, world, profile=True)
+    clocks.start()  # before the inputs are built: sampling by the time the steps run
+    runner = StepRunner(H, I, wl, dev)
+    ms, launches, prof = time_steps(runner, args.steps, args.warmup, world, profile=True, clocks=clocks)
     clk = clocks.stop()
     ms_max, value = replica_throughput(wl.C * wl.K, ms, world)
 
@@ -318,7 +336,10 @@ def run_ours(args, rank, world, local):
         ent = {"avg_ms": round(avg, 4), "launches_per_step": cnt / args.steps,
                "share": round(tot / (ms * args.steps), 4)}
         if name in work:
-            ent["roofline"] = roofline_of(name, work[name], avg, peaks)
+            traffic = None
+            if name == "attn_paged" and ATTN_TRAFFIC_PER_BYTE is not None:
+                traffic = round(ATTN_TRAFFIC_PER_BYTE * work[name]["bytes"])
+            ent["roofline"] = roofline_of(name, work[name], avg, peaks, traffic=traffic)
         kernels[name] = ent
     dominant = max(kernels, key=lambda k: kernels[k]["share"]) if kernels else None
     roof = dict(kernels[dominant]["roofline"]) if dominant and "roofline" in kernels[dominant] else None
@@ -421,11 +442,13 @@ def run_kernel(args, rank, world, local):
     clocks = ClockSampler(local)
     clocks.start()
     torch.cuda.synchronize()
+    t0 = time.monotonic()
     e0.record(stream)
     for _ in range(args.steps):
         call()
     e1.record(stream)
     torch.cuda.synchronize()
+    clocks.window(t0, time.monotonic())
     clk = clocks.stop()
     if H.hspec_sync_status() != 0:
         raise RuntimeError(H.hspec_last_error())
