@@ -18,6 +18,7 @@ from __future__ import annotations
 
 import argparse
 import json
+import re
 import math
 import os
 import statistics
@@ -188,13 +189,37 @@ def step_work(sh, C, K, ctx_lens):
     return w
 
 
+def step_roofline_ms(sh, C, K, ctx_lens, peaks):
+    """Lower bound of one draft step: every kernel group at its own roofline (the
+    slower of its algorithmic bytes at measured HBM bandwidth and its flops at the
+    sustained bf16 peak), summed over the step's launches; the row kernels
+    (RMSNorms, RoPE, embedding) as HBM traffic."""
+    w = step_work(sh, C, K, ctx_lens)
+    nM, nA = sh.layers.count("M"), sh.layers.count("A")
+    nL = len(sh.layers)
+    count = {"in_proj": nM, "inject": nM, "ssd_scan": nM, "out_proj": nM,
+             "qkv_proj": nA, "attn_paged": nA, "o_proj": nA}
+    if sh.d_ff:
+        count.update(mlp_gate_up=nL, mlp_down=nL)
+    if sh.vocab:
+        count["lm_head_argmax"] = 1
+    hbm, tf = peaks["hbm_gbs"] * 1e9, peaks["bf16_tflops_sustained"] * 1e12
+    sec = sum(n * max(w[g]["bytes"] / hbm, w[g]["flops"] / tf) for g, n in count.items() if g in w)
+    M, E = C * K, (2 if sh.dtype == "bf16" else 4)
+    row_bytes = (nL * (2 if sh.d_ff else 1) + 1) * M * sh.d * (4 + E)          # RMSNorms
+    row_bytes += nM * M * sh.H * sh.P * (4 + 2 * E)                          # gated RMSNorm
+    row_bytes += nA * M * (sh.Hq + sh.Hkv) * sh.D * 2 * E                    # RoPE
+    row_bytes += M * sh.d * (E + 4) if sh.vocab else 0                       # embedding
+    return (sec + row_bytes / hbm) * 1e3
+
+
 # DRAM bytes (read + write) per algorithmic byte of the paged-attention kernel, from
 # one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum) of the current
 # attn_tc_kernel at Llama-3-8B shapes, C=32, ctx U[512,8192] (682.8 MB for 656.2 MB of
 # K/V; the excess is the split partials).  The step's attention launch is too large
 # to capture; its traffic is this ratio times its algorithmic bytes (traffic grows
 # with the K/V read).  Set to None whenever the kernel changes until re-captured.
-ATTN_TRAFFIC_PER_BYTE = 1.0405
+ATTN_TRAFFIC_PER_BYTE = None
 
 
 def roofline_of(name, work, avg_ms, peaks, traffic=None, sustained=True):
@@ -353,19 +378,26 @@ def run_ours(args, rank, world, local):
     e2e = {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4), "wall_ms_per_step": round(e2e_wall_ms, 4)}
 
-    sweep = None
-    if args.sweep:
-        sweep = []
-        for K in I.FULL_SWEEP_K:
-            for C in I.FULL_SWEEP_C:
+    # concurrency sweep: draft-step latency and drafted tokens/s at C = 1 .. 128 (K = 16;
+    # with --sweep also K = 8 and 32), each against the step's roofline.  The main
+    # measurement above is the C = 128, K = 16 point.
+    sweep = []
+    for K in (I.FULL_SWEEP_K if args.sweep else (args.K,)):
+        for C in I.FULL_SWEEP_C:
+            if C == wl.C and K == wl.K:
+                m2, lens2 = ms_max, runner.st["ctx_lens"].cpu()
+            else:
                 w2 = I.full_workload(C, K)
                 r2 = StepRunner(H, I, w2, dev, weights=runner.st["weights"])
-                m2, _, _ = time_steps(r2, max(3, args.steps // 2), 2, 1)
-                sweep.append({"C": C, "K": K, "us_per_step": round(m2 * 1e3, 1),
-                              "tokens_per_s": round(C * K / (m2 / 1e3), 1)})
+                m2, _, _ = time_steps(r2, max(5, args.steps // 2), 3, 1)
+                lens2 = r2.st["ctx_lens"].cpu()
                 r2.close()
                 del r2
                 torch.cuda.empty_cache()
+            roof_ms = step_roofline_ms(wl.shapes, C, K, lens2, peaks)
+            sweep.append({"C": C, "K": K, "us_per_step": round(m2 * 1e3, 1),
+                          "tokens_per_s": round(C * K / (m2 / 1e3), 1),
+                          "roofline_us": round(roof_ms * 1e3, 1), "frac_of_roofline": round(roof_ms / m2, 4)})
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -401,7 +433,8 @@ def run_kernel(args, rank, world, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     peaks = load_peaks()
-    wl = I.WORKLOADS[args.workload]
+    m = re.fullmatch(r"full_C(\d+)_K(\d+)", args.workload)
+    wl = I.full_workload(int(m.group(1)), int(m.group(2))) if m else I.WORKLOADS[args.workload]
     sh, C, K = wl.shapes, wl.C, wl.K
     cfg = H.make_cfg(sh)
     E = 2 if sh.dtype == "bf16" else 4
@@ -512,7 +545,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel", choices=["step", "attn", "inject", "ssd"], default="step",
                     help="time one C-ABI call on --workload instead of the full draft step")
-    ap.add_argument("--workload", default="llama_c32", help="kernel-level workload (tiny, llama_c1, llama_c32, qwen_c128)")
+    ap.add_argument("--workload", default="llama_c32", help="kernel-level workload (tiny, llama_c1, llama_c32, qwen_c128, or full_C<C>_K<K>: one layer of the full step)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

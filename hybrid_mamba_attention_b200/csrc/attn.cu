@@ -138,87 +138,160 @@ __global__ void __launch_bounds__(kThreads) attn_split_kernel(AttnArgs a, float 
   }
 }
 
-template <typename T>
-__global__ void attn_merge_kernel(AttnArgs a) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+// Combines the split partials of one output row (request c, block position j, query
+// head h): o = sum_q 2^(m_q - M) acc_q / sum_q 2^(m_q - M) l_q, M = max m_q.  W warps
+// share a row, warp w taking partials q = w, w + W, ... (with few rows the partial
+// loads of a row then spread over W warps); the warps' (M_w, L_w, o_w) are combined in
+// warp order, so the result does not depend on timing.  V4: a lane holds elements
+// 4 lane .. 4 lane + 3 (float4 loads); else lane + 32 i.
+template <typename T, int W, bool V4>
+__global__ void __launch_bounds__(256) attn_merge_kernel(AttnArgs a) {
+  constexpr int RPC = 8 / W;  // rows per CTA
+  __shared__ float s_acc[W > 1 ? 8 : 1][128];
+  __shared__ float s_ml[8][2];
+  const int wib = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int wq = wib % W, rl = wib / W;
   const int G = a.Hq / a.Hkv, R = a.K * G;
   const long rows = (long)a.C * a.K * a.Hq;
-  if (warp >= rows) return;
-  const int h = warp % a.Hq;
-  const int j = (warp / a.Hq) % a.K;
-  const int c = warp / (a.Hq * a.K);
+  const long row_id = (long)blockIdx.x * RPC + rl;
+  const bool live = row_id < rows;
+  const int rid = live ? (int)row_id : 0;
+  const int h = rid % a.Hq;
+  const int j = (rid / a.Hq) % a.K;
+  const int c = rid / (a.Hq * a.K);
   const int g = h / G, row = j * G + h % G;
   const int ctx = a.ctx_lens[c];
-  T* out = (T*)a.out + (size_t)(c * a.K + j) * a.o_rs + (size_t)h * a.D;
-  if (ctx < 0 || ctx > a.max_pages * a.page_size) {
-    for (int e = lane; e < a.D; e += 32) out[e] = from_f<T>(0.f);
-    return;
+  const bool valid = live && ctx >= 0 && ctx <= a.max_pages * a.page_size;
+  // Partials of the row: q = 0 .. ns - 1 at rows base0 + q * stride.
+  //   fp32 path: one per split of (c, g).
+  //   tensor-core path: the sequence (c, rb, g) holds t_seq tiles from tile s0 of the
+  //   line cut into chunks of Z tiles; its piece p in chunk k0 + p has slot
+  //   c * spr + rb * Hkv + g + k0 + p, two halves each, so q = 2 p + half.  Half h of
+  //   a piece holds its tiles of parity h: it exists iff the piece has more than h
+  //   tiles (a missing partial is never written, and its weight is 0).
+  // A partial with l = 0 saw no key and is skipped.
+  int ns = 0, s0 = 0, k0 = 0, t_seq = 0, Z = 1;
+  size_t base0 = 0, stride = R;
+  if (a.block_in_last_split) {
+    const int* off = a.sched + 64;
+    const int n_rb = (R + kAttnTcRows - 1) / kAttnTcRows, spr = a.Hkv * n_rb;
+    const int rb = row / kAttnTcRows, rr = row % kAttnTcRows;
+    const int r = rb * a.Hkv + g;
+    Z = a.sched[2];
+    stride = R < kAttnTcRows ? R : kAttnTcRows;
+    if (valid) {
+      t_seq = (off[c + 1] - off[c]) / spr;
+      s0 = off[c] + r * t_seq;
+      k0 = s0 / Z;
+      ns = t_seq > 0 ? 2 * ((s0 + t_seq - 1) / Z - k0 + 1) : 0;
+    }
+    base0 = ((size_t)c * spr + r + k0) * 2 * stride + rr;
+  } else {
+    ns = valid ? (ctx + a.K + a.split_tokens - 1) / a.split_tokens * a.sub_splits : 0;
+    base0 = (((size_t)c * a.Hkv + g) * a.n_splits * a.sub_splits) * R + row;
   }
-  const int ns = (a.block_in_last_split ? max(1, (ctx + a.split_tokens - 1) / a.split_tokens)
-                                       : (ctx + a.K + a.split_tokens - 1) / a.split_tokens) * a.sub_splits;
-  const size_t base0 = (((size_t)c * a.Hkv + g) * a.n_splits * a.sub_splits) * R + row;
-  // Partial q exists when its split has keys for it: on the tensor-core path half h of
-  // split s holds the split's tiles of parity h, so it exists iff the split has more
-  // than h tiles (a missing partial is never written, and its weight is 0); a partial
-  // with l = 0 saw no key and is skipped.
-  const int n_units = ns / a.sub_splits;
   auto has = [&](int q) -> bool {
     if (!a.block_in_last_split) return true;
-    const int sp = q / a.sub_splits, h = q % a.sub_splits;
-    const int b = sp * a.split_tokens, e = min(ctx, b + a.split_tokens);
-    const int nbt = (a.K + kAttnTcTile - 1) / kAttnTcTile;  // tiles of the block's own keys
-    const int tiles = (e > b ? (e - b + kAttnTcTile - 1) / kAttnTcTile : 0) + (sp == n_units - 1 ? nbt : 0);
-    return tiles > h;
+    const int p = q >> 1, hh = q & 1;
+    const int lo = max(s0, (k0 + p) * Z), hi = min(s0 + t_seq, (k0 + p + 1) * Z);
+    return hi - lo > hh;
   };
-  // (m, l) of partial q: lanes take q = lane, lane + 32, ... (independent loads)
-  auto ml_of = [&](int q) -> float2 { return *(const float2*)(a.ws_ml + (base0 + (size_t)q * R) * 2); };
+  auto ml_of = [&](int q) -> float2 { return *(const float2*)(a.ws_ml + (base0 + (size_t)q * stride) * 2); };
+  // this warp's partials: q = wq + W k
+  const int nk = ns > wq ? (ns - wq + W - 1) / W : 0;
   float M = -INFINITY;
-  for (int q = lane; q < ns; q += 32)
+  for (int k = lane; k < nk; k += 32) {
+    const int q = wq + W * k;
     if (has(q)) {
       const float2 ml = ml_of(q);
       if (ml.y > 0.f) M = fmaxf(M, ml.x);
     }
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   float L = 0.f;
-  for (int q = lane; q < ns; q += 32)
+  for (int k = lane; k < nk; k += 32) {
+    const int q = wq + W * k;
     if (has(q)) {
       const float2 ml = ml_of(q);
       if (ml.y > 0.f) L += exp2f(ml.x - M) * ml.y;
     }
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-  const float inv = L > 0.f ? 1.f / L : 0.f;
-  // o = sum_q w_q acc_q with w_q = 2^(m_q - M) (0 for a missing partial): lane holds
-  // elements lane + 32 i; the acc loads do not depend on the weights, so the loads of
-  // several partials are in flight together (a missing partial is read but not used)
-  constexpr int EPL = 4;  // elements per lane (head_dim <= 128)
-  float o[EPL] = {0.f, 0.f, 0.f, 0.f};
-  for (int q0 = 0; q0 < ns; q0 += 32) {
+  // o_w = sum_q 2^(m_q - M_w) acc_q: the acc loads do not depend on the weights, so the
+  // loads of several partials are in flight together (a missing partial is read but
+  // not used)
+  float o[4] = {0.f, 0.f, 0.f, 0.f};
+  const bool v4_lane = V4 && 4 * lane < a.D;
+  for (int kk0 = 0; kk0 < nk; kk0 += 32) {
     float w_l = 0.f;
-    if (q0 + lane < ns && has(q0 + lane)) {
-      const float2 ml = ml_of(q0 + lane);
+    if (kk0 + lane < nk && has(wq + W * (kk0 + lane))) {
+      const float2 ml = ml_of(wq + W * (kk0 + lane));
       if (ml.y > 0.f) w_l = exp2f(ml.x - M);
     }
-    const int cnt = min(32, ns - q0);
-#pragma unroll 4
+    const int cnt = min(32, nk - kk0);
+#pragma unroll 8
     for (int k = 0; k < cnt; ++k) {
       const float w = __shfl_sync(0xffffffffu, w_l, k);
-      const float* accp = a.ws_acc + (base0 + (size_t)(q0 + k) * R) * a.D;
+      const float* accp = a.ws_acc + (base0 + (size_t)(wq + W * (kk0 + k)) * stride) * a.D;
+      if (V4) {
+        if (v4_lane) {
+          const float4 x = *(const float4*)(accp + 4 * lane);
+          o[0] = w != 0.f ? fmaf(w, x.x, o[0]) : o[0];
+          o[1] = w != 0.f ? fmaf(w, x.y, o[1]) : o[1];
+          o[2] = w != 0.f ? fmaf(w, x.z, o[2]) : o[2];
+          o[3] = w != 0.f ? fmaf(w, x.w, o[3]) : o[3];
+        }
+      } else {
 #pragma unroll
-      for (int i = 0; i < EPL; ++i) {
-        const int e = lane + 32 * i;
-        if (e < a.D) {
-          const float x = accp[e];
-          o[i] = w != 0.f ? fmaf(w, x, o[i]) : o[i];
+        for (int i = 0; i < 4; ++i) {
+          const int e = lane + 32 * i;
+          if (e < a.D) {
+            const float x = accp[e];
+            o[i] = w != 0.f ? fmaf(w, x, o[i]) : o[i];
+          }
         }
       }
     }
   }
+  T* out = (T*)a.out + (size_t)(c * a.K + j) * a.o_rs + (size_t)h * a.D;
+  auto store = [&](const float* v, float inv) {
+    if (V4) {
+      if (v4_lane)
 #pragma unroll
-  for (int i = 0; i < EPL; ++i) {
-    const int e = lane + 32 * i;
-    if (e < a.D) out[e] = from_f<T>(o[i] * inv);
+        for (int i = 0; i < 4; ++i) out[4 * lane + i] = from_f<T>(v[i] * inv);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (lane + 32 * i < a.D) out[lane + 32 * i] = from_f<T>(v[i] * inv);
+    }
+  };
+  if constexpr (W == 1) {
+    if (live) store(o, L > 0.f ? 1.f / L : 0.f);
+  } else {
+    // the W warps of the row: (M_w, L_w, o_w) through shared memory, combined in order
+#pragma unroll
+    for (int i = 0; i < 4; ++i) s_acc[wib][V4 ? 4 * lane + i : lane + 32 * i] = o[i];
+    if (lane == 0) s_ml[wib][0] = M, s_ml[wib][1] = L;
+    __syncthreads();
+    if (wq == 0 && live) {
+      float Mx = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < W; ++w)
+        if (s_ml[rl * W + w][1] > 0.f) Mx = fmaxf(Mx, s_ml[rl * W + w][0]);
+      float Lt = 0.f, ot[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int w = 0; w < W; ++w) {
+        const int src = rl * W + w;
+        if (!(s_ml[src][1] > 0.f)) continue;
+        const float sc = exp2f(s_ml[src][0] - Mx);
+        Lt += sc * s_ml[src][1];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) ot[i] = fmaf(sc, s_acc[src][V4 ? 4 * lane + i : lane + 32 * i], ot[i]);
+      }
+      store(ot, Lt > 0.f ? 1.f / Lt : 0.f);
+    }
   }
 }
 
@@ -246,11 +319,26 @@ void launch_simt(const AttnArgs& a, cudaStream_t s) {
   }
 }
 
+template <typename T, int W>
+void launch_merge_w(const AttnArgs& a, long rows, cudaStream_t s) {
+  const int grid = (int)((rows + 8 / W - 1) / (8 / W));
+  if (a.D % 4 == 0) attn_merge_kernel<T, W, true><<<grid, 256, 0, s>>>(a);
+  else attn_merge_kernel<T, W, false><<<grid, 256, 0, s>>>(a);
+  note_launch();
+}
+
 template <typename T>
 void launch_merge(const AttnArgs& a, cudaStream_t s) {
+  // warps per output row: enough warps in all for about 32 per SM
   const long rows = (long)a.C * a.K * a.Hq;
-  attn_merge_kernel<T><<<(int)((rows + 7) / 8), 256, 0, s>>>(a);
-  note_launch();
+  int W = 1;
+  while (W < 8 && rows * W < 148L * 32) W *= 2;
+  switch (W) {
+    case 1: launch_merge_w<T, 1>(a, rows, s); break;
+    case 2: launch_merge_w<T, 2>(a, rows, s); break;
+    case 4: launch_merge_w<T, 4>(a, rows, s); break;
+    default: launch_merge_w<T, 8>(a, rows, s); break;
+  }
 }
 
 }  // namespace
@@ -273,19 +361,9 @@ bool attn_supported(int dtype, int K, int G, int D, const char** why) {
 }
 
 int attn_split_tokens(int dtype, int C, int Hkv, int K, int max_ctx, int requested) {
-  if (dtype == HSPEC_DTYPE_BF16) {
-    // tensor-core path: 64-token tiles; long splits amortise the partial write, but
-    // at least ~2 CTAs per SM over the grid
-    // the persistent kernel balances items dynamically: splits only need to spread
-    // long requests over several SMs (about 4 items per SM), and long splits keep the
-    // partial traffic (two halves of R x D fp32 per split) small against the K/V read
-    if (requested > 0) return ((requested + 63) / 64) * 64;
-    long per = ((long)C * Hkv * max_ctx + 4L * 148 - 1) / (4L * 148);
-    per = ((per + 63) / 64) * 64;
-    if (per < 256) per = 256;
-    if (per > 8192) per = 8192;
-    return (int)per;
-  }
+  // tensor-core path: the requested chunk length in tokens (whole 64-token tiles), or 0
+  // for one chunk per SM, chosen on the device from the actual context lengths
+  if (dtype == HSPEC_DTYPE_BF16) return requested > 0 ? ((requested + 63) / 64) * 64 : 0;
   if (requested > 0) return requested;
   const long target_ctas = 148L * 16;
   long per = ((long)C * Hkv * (max_ctx + K) + target_ctas - 1) / target_ctas;
@@ -295,16 +373,28 @@ int attn_split_tokens(int dtype, int C, int Hkv, int K, int max_ctx, int request
 }
 
 int attn_num_splits(int dtype, int K, int max_ctx, int split_tokens) {
-  if (dtype == HSPEC_DTYPE_BF16) return max(1, (max_ctx + split_tokens - 1) / split_tokens);
+  if (dtype == HSPEC_DTYPE_BF16) return 0;
   return (max_ctx + K + split_tokens - 1) / split_tokens;
 }
 
 int attn_sub_splits(int dtype) { return dtype == HSPEC_DTYPE_BF16 ? 2 : 1; }
 
-size_t attn_ws_bytes(int C, int Hkv, int K, int G, int D, int n_splits, int sub_splits) {
-  const size_t rows = (size_t)C * Hkv * n_splits * sub_splits * K * G;
-  // + work counter and unit count, + unit list of the tensor-core path
-  return rows * D * sizeof(float) + rows * 2 * sizeof(float) + 256 + (size_t)C * n_splits * 2 * sizeof(int);
+size_t attn_partial_rows(int dtype, int C, int Hkv, int K, int G, int n_splits, int max_chunks) {
+  const int R = K * G;
+  if (dtype == HSPEC_DTYPE_BF16) {
+    // a slot per (sequence, chunk) piece: at most C * Hkv * n_rb + chunks slots, two
+    // halves of a row block each
+    const int n_rb = (R + kAttnTcRows - 1) / kAttnTcRows;
+    const size_t slots = (size_t)C * Hkv * n_rb + max_chunks;
+    return slots * 2 * (R < kAttnTcRows ? R : kAttnTcRows);
+  }
+  return (size_t)C * Hkv * n_splits * R;
+}
+
+size_t attn_ws_bytes(int dtype, int C, int Hkv, int K, int G, int D, int n_splits, int max_chunks) {
+  const size_t rows = attn_partial_rows(dtype, C, Hkv, K, G, n_splits, max_chunks);
+  // + the schedule words (256 bytes) and the requests' tile offsets (C + 1)
+  return rows * D * sizeof(float) + rows * 2 * sizeof(float) + 256 + (size_t)(C + 1) * sizeof(int);
 }
 
 bool attn_paged(int dtype, const AttnArgs& a, cudaStream_t s) {

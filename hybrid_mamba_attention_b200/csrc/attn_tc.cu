@@ -3,24 +3,29 @@
 // the target KVs in place -- here the K/V pages are streamed by TMA straight out of
 // the target's pool through the page table, never copied to a drafter-side cache.
 //
-// Work units are (request, context split) pairs; a unit expands into one item per
-// (row block, kv head g).  A one-CTA schedule kernel lists the units longest first
-// (counting sort on the unit's tile count), so that the short units are the last
-// ones taken and the SMs finish together.  The persistent kernel (one CTA per SM)
-// takes items from an atomic counter, the heads of one unit adjacent so that
-// concurrent CTAs read the same pages.  The R = K*G queries of kv head g (block
+// Work partition (stream-K over the tile space): each (request c, row block rb, kv
+// head g) is a sequence of t_c 64-token tiles (the context's, then the block's own
+// keys), and the sequences are laid end to end, request by request.  A one-CTA
+// schedule kernel sums them (T tiles) and cuts the line into chunks of Z = ceil(T /
+// grid) tiles, one per CTA of the persistent kernel (or of a requested length, CTA b
+// then taking chunks b, b + grid, ...), so that every SM streams the same number of
+// tiles whatever the mix of context lengths.  A CTA walks its chunk as pieces, one
+// per sequence it crosses; the piece of sequence q in chunk k writes its partial to
+// slot q + k (distinct for every piece: a later sequence never starts in an earlier
+// chunk), and the merge kernel finds the pieces of a sequence from T, Z and the
+// request's tile offset.  The R = K*G queries of kv head g (block
 // position j, query head g*G + i) form the rows of a 128-row Q tile, so every K/V
 // byte read from HBM feeds all R queries; with R <= 64 the rows are spread 16 per
 // 32-lane TMEM quarter so that all four SM sub-partitions share the softmax work;
 // rows without a query are zero.
 // Warp roles (320 threads):
-//   warp 0      producer: takes the next item, loads its Q tile (TMA) into one of
+//   warp 0      producer: walks the CTA's pieces, loads each one's Q tile (TMA) into one of
 //               two Q buffers, reads page ids two tiles ahead, and streams its
 //               64-token K/V tiles through a 4-stage ring -- per tile one 3-D TMA box
 //               of 16 tokens x 64 dims of head g per page and column block (128-byte
 //               swizzle), all boxes of a tile issued at once, one lane each -- and
-//               writes the tile's description next to it.  The last context split
-//               of a request also streams the block's own keys as one more tile.
+//               writes the tile's description next to it.  A sequence's last tiles
+//               are the block's own keys (one more tile for K <= 64).
 //   warp 1      TMEM owner and single-thread MMA issuer, driven by readiness rather
 //               than by a fixed order: it issues O_w += P_w . V_i (M=128, N=D, K=64)
 //               as soon as the P of tile i is in shared memory, and S_b = Q . K_i^T
@@ -31,10 +36,10 @@
 //               one TMEM lane (query row) per thread; mask, running max in the exp2
 //               domain, P = exp2(s - m) to shared memory as bf16; O_w is rescaled in
 //               TMEM only when the running max grows by more than 8.  Each group
-//               keeps its own (m, l, O) per item and writes its own partial when its
-//               last tile of the item is done -- the half of the split made of the
-//               item's even (or odd) tiles, so the arithmetic does not depend on
-//               scheduling; the merge kernel combines the halves and the splits.
+//               keeps its own (m, l, O) per piece and writes its own partial when its
+//               last tile of the piece is done -- the half of the piece made of its
+//               even (or odd) tiles, so the arithmetic does not depend on timing;
+//               the merge kernel combines the halves and the pieces.
 // Every wait gives up after a time bound and sets the device error word.
 #include <stdint.h>
 
@@ -51,28 +56,31 @@ namespace {
 
 constexpr int TT = kAttnTcTile;  // tokens per tile
 constexpr int PPT = TT / 16;     // 16-token pages per tile
-constexpr int NS = TT == 64 ? 5 : 10;   // K/V ring stages (160 KB)
 constexpr int NSB = TT == 64 ? 4 : 8;   // S buffers in TMEM (half the columns)
 constexpr int NPW = 4;           // producer warps
 constexpr int THREADS = 32 * (NPW + 2 + 8);  // producers, 2 MMA warps, 2 softmax warpgroups
 constexpr int ROWS = 128;     // MMA M
-constexpr int kLenBuckets = 256;  // schedule: units sorted by tile count (capped)
 
 struct TileMeta {  // written by the producer before the stage's barrier arrive
-  int c, g, split, rb;
+  int c, g, slot, rb;  // slot: the partial slot of the piece
   int valid;       // keys in the tile
-  int local;       // tile index within the item
-  int n_tiles;     // tiles of the item
+  int local;       // tile index within the piece
+  int n_tiles;     // tiles of the piece
   int block;       // 1: the block's own keys
-  int qslot, qseq; // Q buffer of the item and the item's use count of that buffer
+  int qslot, qseq; // Q buffer of the piece and the piece's use count of that buffer
   int end;         // 1: no more work
   int bt;          // block tiles: index among the block's tiles
 };
 
-template <int D>
+// SP: the R <= 64 queries of a kv head in an M = 64 tile (rows 16 per TMEM lane
+// quarter, lanes 0..15); else an M = 128 tile.  The 64-row Q buffers leave room for a
+// sixth K/V stage.
+template <int D, bool SP>
 struct Lay {
+  static constexpr int MR = SP ? 64 : ROWS;             // MMA M (rows of the Q tile)
+  static constexpr int NS = SP ? 6 : 5;                 // K/V ring stages (TT = 64)
   static constexpr int DB = D / 64;                     // 64-element column blocks
-  static constexpr int Q_BLK = ROWS * 128;              // 16 KB per Q column block
+  static constexpr int Q_BLK = MR * 128;                // per Q column block
   static constexpr int Q_BYTES = DB * Q_BLK;
   static constexpr int KV_BLK = TT * 128;               // per K column block
   static constexpr int K_BYTES = DB * KV_BLK;           // K: [column block][TT tokens][128 B]
@@ -94,67 +102,57 @@ struct TcMaps {
   CUtensorMap k, v, kb, vb, q;
 };
 
-// TMEM lane (0..127) -> query row of the row block: identity for R > 64; for
-// R <= 64, 16 rows per 32-lane quarter (lanes 0..15 of each quarter), else -1.
-__device__ __forceinline__ int row_of_lane(int lane128, bool spread) {
-  if (!spread) return lane128;
-  const int q = lane128 >> 5, l = lane128 & 31;
-  return l < 16 ? q * 16 + l : -1;
+// Tiles of each sequence of a request: its context tiles and the block's own keys
+// (nbt tiles); none for an invalid context length (the merge writes zero rows).
+__device__ __forceinline__ int seq_tiles(int ctx, long max_ctx, int nbt) {
+  return ctx < 0 || ctx > max_ctx ? 0 : (ctx + TT - 1) / TT + nbt;
 }
 
-// Tiles (TT-token context tiles, plus the block's own keys, nbt tiles, in a request's
-// last split) of unit (ctx, split sp of n).
-__host__ __device__ inline int unit_tiles(int ctx, int sp, int n, int split_tokens, int nbt) {
-  const int b = sp * split_tokens, e = min(ctx, b + split_tokens);
-  return (e > b ? (e - b + TT - 1) / TT : 0) + (sp == n - 1 ? nbt : 0);
-}
-
-// One CTA: lists the (request, split) units longest first into `units` and resets the
-// work counter; sched[1] = number of units.  Requests with an invalid context length
-// get no unit (their output rows are written as zeros by the merge).
-__global__ void __launch_bounds__(1024) attn_sched_kernel(const int32_t* ctx_lens, int C, int split_tokens,
-                                                          long max_ctx, int nbt, int* sched, int2* units,
-                                                          int* err) {
-  __shared__ int hist[kLenBuckets];
-  for (int b = threadIdx.x; b < kLenBuckets; b += blockDim.x) hist[b] = 0;
-  __syncthreads();
-  for (int c = threadIdx.x; c < C; c += blockDim.x) {
+// One CTA: off[c] = tiles of all sequences of requests before c (spr sequences of
+// seq_tiles each per request), off[C] = T; sched[1] = T, sched[2] = Z (the chunk
+// length: ceil(T / grid), or z_req; at least ceil(T / max_chunks)), sched[3] = the
+// number of chunks.
+__global__ void __launch_bounds__(1024) attn_sched_kernel(const int32_t* ctx_lens, int C, long max_ctx, int nbt,
+                                                          int spr, int grid, int z_req, int max_chunks, int* sched,
+                                                          int* off, int* err) {
+  __shared__ int part[1024];
+  const int per = (C + 1023) / 1024;
+  const int c0 = min(C, (int)threadIdx.x * per), c1 = min(C, c0 + per);
+  int sum = 0;
+  for (int c = c0; c < c1; ++c) {
     const int ctx = ctx_lens[c];
-    if (ctx < 0 || ctx > max_ctx) {
-      flag_error(err, kErrCtxOOB);
-      continue;
-    }
-    const int n = ctx > 0 ? (ctx + split_tokens - 1) / split_tokens : 1;
-    for (int sp = 0; sp < n; ++sp) atomicAdd(&hist[min(unit_tiles(ctx, sp, n, split_tokens, nbt), kLenBuckets - 1)], 1);
+    if (ctx < 0 || ctx > max_ctx) flag_error(err, kErrCtxOOB);
+    sum += seq_tiles(ctx, max_ctx, nbt) * spr;
   }
+  part[threadIdx.x] = sum;
   __syncthreads();
-  if (threadIdx.x == 0) {
-    int run = 0;
-    for (int b = kLenBuckets - 1; b >= 0; --b) {
-      const int h = hist[b];
-      hist[b] = run;
-      run += h;
-    }
-    sched[0] = 0;
-    sched[1] = run;
+  for (int o = 1; o < 1024; o <<= 1) {  // inclusive scan of the per-thread sums
+    const int v = threadIdx.x >= (unsigned)o ? part[threadIdx.x - o] : 0;
+    __syncthreads();
+    part[threadIdx.x] += v;
+    __syncthreads();
   }
-  __syncthreads();
-  for (int c = threadIdx.x; c < C; c += blockDim.x) {
-    const int ctx = ctx_lens[c];
-    if (ctx < 0 || ctx > max_ctx) continue;
-    const int n = ctx > 0 ? (ctx + split_tokens - 1) / split_tokens : 1;
-    for (int sp = 0; sp < n; ++sp) {
-      const int pos = atomicAdd(&hist[min(unit_tiles(ctx, sp, n, split_tokens, nbt), kLenBuckets - 1)], 1);
-      units[pos] = make_int2(c, sp);
-    }
+  int run = threadIdx.x > 0 ? part[threadIdx.x - 1] : 0;
+  for (int c = c0; c < c1; ++c) {
+    off[c] = run;
+    run += seq_tiles(ctx_lens[c], max_ctx, nbt) * spr;
+  }
+  if (threadIdx.x == 1023) {
+    const int T = part[1023];
+    int Z = z_req > 0 ? z_req : (T + grid - 1) / grid;
+    Z = max(max(Z, (T + max_chunks - 1) / max_chunks), 1);
+    off[C] = T;
+    sched[1] = T;
+    sched[2] = Z;
+    sched[3] = (T + Z - 1) / Z;
   }
 }
 
-template <int D>
+template <int D, bool SP>
 __global__ void __launch_bounds__(THREADS, 1)
-    attn_tc_kernel(const __grid_constant__ TcMaps maps, AttnArgs a, float scale_log2, int n_rb, int* sched,
-                   const int2* units) {
-  using L = Lay<D>;
+    attn_tc_kernel(const __grid_constant__ TcMaps maps, AttnArgs a, float scale_log2, int n_rb) {
+  using L = Lay<D, SP>;
+  constexpr int NS = L::NS;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = tc::smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023) & ~1023u) - raw);
@@ -175,12 +173,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* drain = q_empty + 2;      // [2] every MMA of an issuer (and its arrivals) finished
   uint32_t* tmem_slot = (uint32_t*)(drain + 2);
   volatile int* end_tile = (volatile int*)(tmem_slot + 1);
-  volatile int* s_item = end_tile + 1;  // [2] next work item, published by producer warp 0
-  volatile int* s_stop = s_item + 2;    // a producer warp gave up waiting
+  volatile int* s_stop = end_tile + 1;  // a producer warp gave up waiting
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = a.Hq / a.Hkv, R = a.K * G;
-  const bool spread = R <= 64;
+  const int RB = R < ROWS ? R : ROWS;  // rows of a row block's partial
+  constexpr bool spread = SP;
   int* err = a.err;
   constexpr int QK_WARP = NPW, PV_WARP = NPW + 1, SM_WARP0 = NPW + 2;
 
@@ -221,7 +219,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     // box bx < KB is K page bx / DB, column block bx % DB (16 tokens x 64 dims of head
     // g, 128-byte swizzle); box KB + q is V page q (one 4-D box, both column blocks).
     // Box bx is issued by lane bx / NPW of warp bx % NPW.  All producer warps walk the
-    // same tiles; warp 0 takes the work items and loads the Q tiles.
+    // same tiles; warp 0 loads the Q tiles.
     constexpr int KB = PPT * L::DB, NBX = KB + PPT;
     const int pw = warp;
     const int bx = pw + NPW * lane;
@@ -240,33 +238,51 @@ __global__ void __launch_bounds__(THREADS, 1)
     // (16 rows); otherwise one holding 128 / G positions (128 rows)
     const int q_boxes = spread ? (R + 15) / 16 : 1;
     const int q_pos = spread ? 16 / G : ROWS / G;
-    const int per_unit = a.Hkv * n_rb;
-    const int n_items = sched[1] * per_unit;
-    const int nbt = (a.K + TT - 1) / TT;  // tiles of the block's own keys
+    const int spr = a.Hkv * n_rb;         // sequences per request
     const int pshift = (a.page_size & (a.page_size - 1)) == 0 ? __ffs(a.page_size) - 1 : -1;
+    const int T = a.sched[1], Z = a.sched[2], n_chunks = a.sched[3];
+    const int* off = a.sched + 64;
+    // the request holding tile p of the line: the last c with off[c] <= p
+    auto locate = [&](int p) -> int {
+      int lo = 0, hi = a.C - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (off[mid] <= p) lo = mid;
+        else hi = mid - 1;
+      }
+      return lo;
+    };
+    int k = blockIdx.x;  // this CTA's chunk
+    int pos = k < n_chunks ? k * Z : 0, end = k < n_chunks ? min(T, pos + Z) : 0;
+    int c = pos < end ? locate(pos) : 0;
     int tile_i = 0;
     bool ok = true;
-    int it_next = threadIdx.x == 0 ? atomicAdd(sched, 1) : 0;  // the following item, in flight
-    // Every producer warp passes the same item barriers: the loop ends only after one,
-    // when the work is done or a producer has given up waiting.
+    // Every producer warp walks the same pieces and passes the same barriers: the loop
+    // ends only after one, when the work is done or a producer has given up waiting.
     for (int seq = 0;; ++seq) {
-      if (threadIdx.x == 0) s_item[seq & 1] = it_next;
       asm volatile("bar.sync 1, %0;" ::"n"(32 * NPW) : "memory");
-      const int item = s_item[seq & 1];
-      if (item >= n_items || *s_stop) break;
-      if (threadIdx.x == 0) it_next = atomicAdd(sched, 1);  // prefetch: used by the next item
-      const int u = item / per_unit, g = item % a.Hkv, rb = (item % per_unit) / a.Hkv;
-      const int2 cu = units[u];
-      const int c = cu.x, split = cu.y;
+      if (*s_stop) break;
+      if (pos >= end) {  // the CTA's next chunk
+        k += gridDim.x;
+        if (k >= n_chunks) break;
+        pos = k * Z;
+        end = min(T, pos + Z);
+        c = locate(pos);
+      }
+      while (off[c + 1] <= pos) ++c;
+      // piece: tiles [lt0, lt0 + n_tiles) of sequence r = rb Hkv + g of request c
+      const int t_seq = (off[c + 1] - off[c]) / spr;
+      const int rel = pos - off[c];
+      const int r = rel / t_seq, lt0 = rel - r * t_seq;
+      const int n_tiles = min(t_seq - lt0, end - pos);
+      const int g = r % a.Hkv, rb = r / a.Hkv;
+      const int pslot = c * spr + r + k;  // partial slot of the piece
+      pos += n_tiles;
       const int ctx = a.ctx_lens[c];
-      const int n_ctx_splits = ctx > 0 ? (ctx + a.split_tokens - 1) / a.split_tokens : 1;
-      const int c_begin = split * a.split_tokens;
-      const int c_end = min(ctx, c_begin + a.split_tokens);
-      const int n_ctx_tiles = c_end > c_begin ? (c_end - c_begin + TT - 1) / TT : 0;
-      const int n_tiles = n_ctx_tiles + (split == n_ctx_splits - 1 ? nbt : 0);
+      const int ct = (ctx + TT - 1) / TT;  // context tiles of the sequence
       const int slot = seq & 1;
 
-      // Q tile of the item into Q buffer `slot` once the item two back is done with it
+      // Q tile of the piece into Q buffer `slot` once the piece two back is done with it
       if (pw == 0) {
         if (lane == 0) ok = tc::mbar_wait(&q_empty[slot], ((seq >> 1) & 1) ^ 1, err);
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -278,7 +294,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (lane < q_boxes * L::DB) {
             const int qb = lane / L::DB, qk = lane % L::DB;
             const int pos0 = c * a.K + (spread ? qb * q_pos : rb * q_pos);
-            tc::tma_load_3d(qbuf + qk * L::Q_BLK + qb * 32 * 128, &maps.q, &q_full[slot], qk * 64, g * G, pos0);
+            tc::tma_load_3d(qbuf + qk * L::Q_BLK + qb * 16 * 128, &maps.q, &q_full[slot], qk * 64, g * G, pos0);
           }
           __syncwarp();
         }
@@ -286,10 +302,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 
       // page id of this lane's page, read two tiles ahead into registers
       // (unconditionally, the index clamped into the request's row of the table, so
-      // that nothing waits for it; ids past the split's end are never used)
+      // that nothing waits for it; ids past the context's end are never used)
       const int32_t* table = a.page_table + (size_t)c * a.max_pages;
       auto page_of = [&](int local) -> int {
-        const int t = c_begin + local * TT + 16 * q16;
+        const int t = (lt0 + local) * TT + 16 * q16;
         const int idx = pshift >= 0 ? t >> pshift : t / a.page_size;
         return table[idx < a.max_pages ? idx : a.max_pages - 1];
       };
@@ -305,14 +321,15 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (!ok) break;
         uint8_t* kd = sKV + s * L::STAGE;
         uint8_t* vd = kd + L::K_BYTES;
-        const bool block = local >= n_ctx_tiles;
-        const int bt = local - n_ctx_tiles;  // block tiles: keys [bt TT, bt TT + TT) of the block
-        const int t0 = c_begin + local * TT;
-        const int valid = block ? min(TT, a.K - bt * TT) : min(TT, c_end - t0);
+        const int st = lt0 + local;  // tile of the sequence
+        const bool block = st >= ct;
+        const int bt = st - ct;      // block tiles: keys [bt TT, bt TT + TT) of the block
+        const int t0 = st * TT;
+        const int valid = block ? min(TT, a.K - bt * TT) : min(TT, ctx - t0);
         const int groups = (valid + 15) / 16;  // 16-row boxes with keys
         if (pw == 0 && lane == 0) {
           volatile TileMeta& m = meta[s];
-          m.c = c, m.g = g, m.split = split, m.rb = rb, m.valid = valid, m.local = local;
+          m.c = c, m.g = g, m.slot = pslot, m.rb = rb, m.valid = valid, m.local = local;
           m.n_tiles = n_tiles, m.block = block ? 1 : 0, m.qslot = slot, m.qseq = seq, m.end = 0;
           m.bt = block ? bt : 0;
         }
@@ -365,9 +382,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (lane == 0) {
       // ---------------------------------------------------------- Q.K^T issuer
       // S_b = Q . K_i^T into S buffer b = i % NSB once tile i has landed, S_b is free
-      // (the P.V of tile i - NSB has read its P) and the item's Q is loaded.  Issuing
+      // (the P.V of tile i - NSB has read its P) and the piece's Q is loaded.  Issuing
       // P.V from another thread keeps either kind of MMA from waiting behind the other.
-      constexpr uint32_t idesc_qk = tc::idesc_bf16_f32(ROWS, TT);
+      constexpr uint32_t idesc_qk = tc::idesc_bf16_f32(L::MR, TT);
       int q_seen[2] = {-1, -1};
       for (int qk = 0;; ++qk) {
         const int s = qk % NS, b = qk & (NSB - 1);
@@ -389,7 +406,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           tc::mma_bf16(tmem + L::S_COL(b), tc::sdesc_k128(q + (kk / 4) * L::Q_BLK + (kk % 4) * 32),
                        tc::sdesc_k128(k + (kk / 4) * L::KV_BLK + (kk % 4) * 32), idesc_qk, kk > 0);
         tc::mma_commit(&s_full[b]);
-        if (meta[s].local == meta[s].n_tiles - 1) tc::mma_commit(&q_empty[slot]);  // item's last QK
+        if (meta[s].local == meta[s].n_tiles - 1) tc::mma_commit(&q_empty[slot]);  // piece's last QK
       }
       // no MMA or commit arrival may land after the CTA has finished
       tc::mma_commit(&drain[0]);
@@ -401,7 +418,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       // O_w += P_i . V_i as soon as the P of tile i is in TMEM (group w = i % 2).  Tile
       // i's Q.K^T finished before its softmax began, so the commit after P.V frees the
       // whole stage.
-      constexpr uint32_t idesc_pv = tc::idesc_bf16_f32(ROWS, D) | (1u << 16);  // B (= V) MN-major
+      constexpr uint32_t idesc_pv = tc::idesc_bf16_f32(L::MR, D) | (1u << 16);  // B (= V) MN-major
       bool ok = true;
       int pv = 0;
       uint64_t idle_since = 0;
@@ -412,7 +429,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (tc::mbar_try_wait(&p_full[pv & (NSB - 1)], (pv / NSB) & 1)) {
           tc::tc_fence_after();
           const int w = pv & 1, s = pv % NS;
-          const bool first = meta[s].local < 2;  // this group's first tile of the item
+          const bool first = meta[s].local < 2;  // this group's first tile of the piece
           const uint32_t pt = tmem + L::S_COL(pv & (NSB - 1));  // P of the tile, in its S buffer
           const uint32_t v = tc::smem_u32(sKV + s * L::STAGE + L::K_BYTES);
           // K slice kk = the 16 keys of page kk: V [column block][16 tokens] blocks 2 KB apart
@@ -451,11 +468,22 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ------------------------------------------------------------ softmax warpgroups
     const int wg = (warp - SM_WARP0) >> 2;  // 0: first four softmax warps, 1: the next four
     const int quarter = warp & 3;           // TMEM lanes this warp may access
-    const int lane128 = quarter * 32 + lane;
-    const int r_local = row_of_lane(lane128, spread);
+    // SP: row quarter * 16 + (lane & 15), the two half-warps taking columns
+    // [0, TT / 2) and [TT / 2, TT) of S (and halves of O); else row quarter * 32 + lane
+    constexpr int CW = SP ? TT / 2 : TT;  // score columns per thread
+    const int hf = SP ? lane >> 4 : 0;    // which half of the row's columns
+    const int r_local = SP ? quarter * 16 + (lane & 15) : quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const uint32_t tOw = tmem + lane_off + L::O_COL(wg);
     const int gthread = (warp - SM_WARP0 - 4 * wg) * 32 + lane;  // 0..127 within the group
+    // the thread's O columns: SP, halves [hf D / 2, hf D / 2 + D / 2) read as 32-column
+    // chunks cb (16x32bx2 with offset D / 2); else all D
+    auto o_ld = [&](int cb, float (&v)[32]) {
+      if constexpr (SP) tc::tmem_ld16x2_32<D / 2>(tOw + cb * 32, v);
+      else tc::tmem_ld32(tOw + cb * 32, v);
+    };
+    constexpr int OCB = SP ? D / 64 : D / 32;  // 32-column chunks of O per thread
+    auto o_col = [&](int cb) { return SP ? hf * (D / 2) + cb * 32 : cb * 32; };
 
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
@@ -470,33 +498,35 @@ __global__ void __launch_bounds__(THREADS, 1)
       // the stage cannot move on before this group's P.V of the tile)
       ok = __all_sync(0xffffffffu, tc::mbar_wait(&kv_full[s], (i / NS) & 1, err));
       if (!ok) break;
-      const int c = meta[s].c, g = meta[s].g, split = meta[s].split, rb = meta[s].rb;
+      const int c = meta[s].c, g = meta[s].g, pslot = meta[s].slot, rb = meta[s].rb;
       const int local = meta[s].local, n_tiles = meta[s].n_tiles, valid = meta[s].valid;
       const bool block_tile = meta[s].block != 0;
       const int bt = meta[s].bt;
-      const int gr = rb * ROWS + (r_local < 0 ? 0 : r_local);
-      const bool active = r_local >= 0 && gr < R;
+      const int gr = rb * ROWS + r_local;
+      const bool active = gr < R;
       const int jq = active ? gr / G : 0;
-      if (local < 2) {  // this group's first tile of a new item
+      if (local < 2) {  // this group's first tile of a new piece
         m_used = -INFINITY;
         l = 0.f;
       }
-      float sv[TT];
-      tc::tmem_ld(tmem + lane_off + L::S_COL(b), sv);
+      float sv[CW];
+      if constexpr (SP) tc::tmem_ld16x2_32<TT / 2>(tmem + lane_off + L::S_COL(b), sv);
+      else tc::tmem_ld(tmem + lane_off + L::S_COL(b), sv);
       // raw scores; the scale (> 0) is applied inside the exponent below
       float mx = -INFINITY;
       if (valid == TT && !(block_tile && a.causal_block)) {
 #pragma unroll
-        for (int j = 0; j < TT; ++j) mx = fmaxf(mx, sv[j]);
+        for (int j = 0; j < CW; ++j) mx = fmaxf(mx, sv[j]);
       } else {
         // causal block: query position jq sees the block keys 0..jq
-        const int vis_end = (block_tile && a.causal_block) ? min(valid, jq + 1 - bt * TT) : valid;
+        const int vis_end = ((block_tile && a.causal_block) ? min(valid, jq + 1 - bt * TT) : valid) - hf * CW;
 #pragma unroll
-        for (int j = 0; j < TT; ++j) {
+        for (int j = 0; j < CW; ++j) {
           sv[j] = j < vis_end ? sv[j] : -INFINITY;
           mx = fmaxf(mx, sv[j]);
         }
       }
+      if constexpr (SP) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
       const float m_new = fmaxf(m_used, mx * scale_log2);  // running max in the exp2 domain
       float alpha = 1.f;
       bool rescale = false;
@@ -511,10 +541,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       // with no visible key yet (m = -inf) every s is -inf: subtract 0 so p = 0, not NaN
       const float mu = m_used == -INFINITY ? 0.f : m_used;
       float2 psum = make_float2(0.f, 0.f);
-      uint32_t pk[TT / 2];
+      uint32_t pk[CW / 2];
       const float2 sc2 = make_float2(scale_log2, scale_log2), nm2 = make_float2(-mu, -mu);
 #pragma unroll
-      for (int j = 0; j < TT; j += 2) {
+      for (int j = 0; j < CW; j += 2) {
         // p = 2^(s scale - m): the exponents of a pair in one packed FFMA, then one ex2
         // each (flushing results below 2^-126 to zero); 2^(-inf) = 0 for masked columns
         const float2 e = tc::ffma2(make_float2(sv[j], sv[j + 1]), sc2, nm2);
@@ -523,9 +553,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         __nv_bfloat162 h2 = __floats2bfloat162_rn(pp.x, pp.y);
         pk[j / 2] = *reinterpret_cast<uint32_t*>(&h2);
       }
-      l += psum.x + psum.y;
-      // P over the first half of S_b
-      tc::tmem_stu(tmem + lane_off + L::S_COL(b), pk);
+      float ps = psum.x + psum.y;
+      if constexpr (SP) ps += __shfl_xor_sync(0xffffffffu, ps, 16);  // the row's other half
+      l += ps;
+      // P over the first half of S_b (bf16 pairs: the row's keys 2c, 2c + 1 in column c)
+      if constexpr (SP) tc::tmem_st16x2_16u<TT / 4>(tmem + lane_off + L::S_COL(b), pk);
+      else tc::tmem_stu(tmem + lane_off + L::S_COL(b), pk);
       // The group's previous P.V (before O_w may be rescaled).  It is waited for at
       // every tile, not only before a rescale: softmax may run several tiles ahead of
       // the P.V's, and a parity wait is only unambiguous while its waiter is at most
@@ -536,14 +569,15 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc::tc_fence_after();
       }
       if (__any_sync(0xffffffffu, rescale)) {
-        // O_w holds this group's earlier tiles of the item
+        // O_w holds this group's earlier tiles of the piece
 #pragma unroll
-        for (int cb = 0; cb < D / 32; ++cb) {
+        for (int cb = 0; cb < OCB; ++cb) {
           float v[32];
-          tc::tmem_ld32(tOw + cb * 32, v);
+          o_ld(cb, v);
 #pragma unroll
           for (int e = 0; e < 32; ++e) v[e] *= alpha;
-          tc::tmem_st32(tOw + cb * 32, v);
+          if constexpr (SP) tc::tmem_st16x2_32<D / 2>(tOw + cb * 32, v);
+          else tc::tmem_st32(tOw + cb * 32, v);
         }
       }
       if (valid < TT) {
@@ -563,24 +597,24 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (lane == 0) tc::mbar_arrive(&p_full[b]);
 
       if (local >= n_tiles - 2) {
-        // this group's last tile of the item: write its partial (half of the split)
+        // this group's last tile of the piece: write its partial (half of the piece)
         ok = __all_sync(0xffffffffu, tc::mbar_wait(&pv_done[wg], n & 1, err));
         if (!ok) break;
         tc::tc_fence_after();
-        // half (local & 1): the item's even or odd tiles, whichever group ran them,
-        // so the result does not depend on how items were scheduled
-        const size_t base = ((((size_t)c * a.Hkv + g) * a.n_splits + split) * 2 + (local & 1)) * R + gr;
+        // half (local & 1): the piece's even or odd tiles, whichever group ran them,
+        // so the result does not depend on timing; rows of the row block
+        const size_t base = ((size_t)pslot * 2 + (local & 1)) * RB + r_local;
 #pragma unroll
-        for (int cb = 0; cb < D / 32; ++cb) {
+        for (int cb = 0; cb < OCB; ++cb) {
           float v[32];
-          tc::tmem_ld32(tOw + cb * 32, v);
+          o_ld(cb, v);
           if (active) {
-            float* o = a.ws_acc + base * D + cb * 32;
+            float* o = a.ws_acc + base * D + o_col(cb);
 #pragma unroll
             for (int e = 0; e < 32; e += 4) *(float4*)(o + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
           }
         }
-        if (active) {
+        if (active && hf == 0) {
           a.ws_ml[base * 2] = m_used;
           a.ws_ml[base * 2 + 1] = l;
         }
@@ -659,14 +693,14 @@ bool make_q_map(CUtensorMap* m, const void* base, long positions, int Hq, int D,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D>
+template <int D, bool SP>
 bool launch_tc(const AttnArgs& a, cudaStream_t s) {
   static bool attr_set[64] = {};
   static int n_sm[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    if (cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay<D>::SMEM) !=
+    if (cudaFuncSetAttribute(attn_tc_kernel<D, SP>, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay<D, SP>::SMEM) !=
         cudaSuccess) {
       set_error("cudaFuncSetAttribute(attn_tc_kernel) failed");
       return false;
@@ -691,21 +725,17 @@ bool launch_tc(const AttnArgs& a, cudaStream_t s) {
   const int R = a.K * (a.Hq / a.Hkv);
   const int n_rb = (R + ROWS - 1) / ROWS;
   if (a.sub_splits != 2) {
-    set_error("tensor-core attention writes two partials per split");
+    set_error("tensor-core attention writes two partials per piece");
     return false;
   }
-  // after the partials: the work counter and unit count (256 bytes), then the unit list
-  const size_t pairs = (size_t)a.C * a.Hkv * a.n_splits * 2 * R;
-  int* sched = (int*)(a.ws_ml + pairs * 2);
-  int2* units = (int2*)(sched + 64);
-  attn_sched_kernel<<<1, 1024, 0, s>>>(a.ctx_lens, a.C, a.split_tokens, (long)a.max_pages * a.page_size,
-                                       (a.K + TT - 1) / TT, sched, units, a.err);
-  note_launch();
-  const long max_items = (long)a.C * a.n_splits * n_rb * a.Hkv;
   const int sms = dev < 64 && n_sm[dev] > 0 ? n_sm[dev] : 148;
-  const int grid = max_items < sms ? (int)max_items : sms;
+  const int grid = min(sms, kAttnMaxChunksAuto);
+  const int z_req = a.split_tokens > 0 ? (a.split_tokens + TT - 1) / TT : 0;
+  attn_sched_kernel<<<1, 1024, 0, s>>>(a.ctx_lens, a.C, (long)a.max_pages * a.page_size, (a.K + TT - 1) / TT,
+                                       a.Hkv * n_rb, grid, z_req, a.max_chunks, a.sched, a.sched + 64, a.err);
+  note_launch();
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
-  attn_tc_kernel<D><<<grid, THREADS, Lay<D>::SMEM, s>>>(maps, a, scale_log2, n_rb, sched, units);
+  attn_tc_kernel<D, SP><<<grid, THREADS, Lay<D, SP>::SMEM, s>>>(maps, a, scale_log2, n_rb);
   note_launch();
   return true;
 }
@@ -723,11 +753,18 @@ bool attn_tc_supported(const AttnArgs& a, const char** why) {
   const uintptr_t any = (uintptr_t)a.q | (uintptr_t)a.kb | (uintptr_t)a.vb | (uintptr_t)a.k_pool | (uintptr_t)a.v_pool;
   if (any & 15) return *why = "q, k_blk, v_blk and the pools must be 16-byte aligned", false;
   if ((long)a.num_pages * a.page_size > 0x7fffffffL) return *why = "pool too large", false;
+  // the tile line (all sequences end to end) is indexed in 32 bits
+  const long n_rb = (a.K * G + ROWS - 1) / ROWS;
+  const long line = (long)a.C * a.Hkv * n_rb * (((long)a.max_pages * a.page_size + TT - 1) / TT + (a.K + TT - 1) / TT);
+  if (line >= (1L << 30)) return *why = "too many context tiles in one call", false;
   return true;
 }
 
 bool attn_tc_launch(const AttnArgs& a, cudaStream_t s) {
-  return a.D == 128 ? launch_tc<128>(a, s) : launch_tc<64>(a, s);
+  // R = K * G query rows per kv head: up to 64 in one M = 64 tile
+  const bool sp = a.K * (a.Hq / a.Hkv) <= 64;
+  if (a.D == 128) return sp ? launch_tc<128, true>(a, s) : launch_tc<128, false>(a, s);
+  return sp ? launch_tc<64, true>(a, s) : launch_tc<64, false>(a, s);
 }
 
 }  // namespace hspec

@@ -171,7 +171,8 @@ hspec_status validate_kv(const hspec_cfg* c, const hspec_kv_view* kv) {
 }
 
 struct AttnPlan {
-  int split_tokens, n_splits;
+  int split_tokens, n_splits, max_chunks;
+  size_t rows;  // partial rows
   size_t ws;
 };
 
@@ -180,8 +181,10 @@ AttnPlan attn_plan(const hspec_cfg* c, int C, int K, int max_pages) {
   const int max_ctx = max_pages * c->page_size;
   p.split_tokens = attn_split_tokens(c->dtype, C, c->n_kv_heads, K, max_ctx, c->attn_split_tokens);
   p.n_splits = attn_num_splits(c->dtype, K, max_ctx, p.split_tokens);
-  p.ws = align256(attn_ws_bytes(C, c->n_kv_heads, K, c->n_q_heads / c->n_kv_heads, c->head_dim, p.n_splits,
-                                attn_sub_splits(c->dtype)));
+  p.max_chunks = p.split_tokens > 0 ? kAttnMaxChunksExplicit : kAttnMaxChunksAuto;
+  const int G = c->n_q_heads / c->n_kv_heads;
+  p.rows = attn_partial_rows(c->dtype, C, c->n_kv_heads, K, G, p.n_splits, p.max_chunks);
+  p.ws = align256(attn_ws_bytes(c->dtype, C, c->n_kv_heads, K, G, c->head_dim, p.n_splits, p.max_chunks));
   return p;
 }
 
@@ -203,21 +206,24 @@ AttnArgs attn_args(const hspec_cfg* c, const AttnPlan& p, const hspec_kv_view* k
   a.ctx_lens = ctx_lens;
   a.split_tokens = p.split_tokens;
   a.n_splits = p.n_splits;
+  a.max_chunks = p.max_chunks;
   a.causal_block = (c->flags & HSPEC_FLAG_CAUSAL_BLOCK) != 0;
   a.block_in_last_split = c->dtype == HSPEC_DTYPE_BF16;
   a.sub_splits = attn_sub_splits(c->dtype);
-  const size_t rows = (size_t)C * a.Hkv * p.n_splits * a.sub_splits * K * (a.Hq / a.Hkv);
   a.ws_acc = (float*)ws;
-  a.ws_ml = a.ws_acc + rows * a.D;
+  a.ws_ml = a.ws_acc + p.rows * a.D;
+  a.sched = (int*)(a.ws_ml + p.rows * 2);
   a.err = device_error_word();
   return a;
 }
 
 // Step workspace layout (all sub-buffers 256-byte aligned).
 struct StepPlan {
-  size_t x, xn, big, y, g, h0, attn, pval, pidx, total;
+  size_t x, xn, big, y, g, h0, attn, pval, pidx, gpart, gcnt, total;
   AttnPlan ap;
   int n_parts;
+  size_t gpart_bytes;  // split-K partials of the projections / MLP GEMMs
+  int gmax_tiles;      // tile counters that follow them
 };
 
 StepPlan step_plan(const hspec_cfg* c, int C, int K, int max_pages) {
@@ -247,6 +253,25 @@ StepPlan step_plan(const hspec_cfg* c, int C, int K, int max_pages) {
   s.n_parts = c->vocab > 0 ? cdiv(c->vocab, argmax_tile_n(c->dtype)) : 0;
   s.pval = off, off += align256(M * s.n_parts * 4);
   s.pidx = off, off += align256(M * s.n_parts * 4);
+  // split-K workspace: the largest need of the step's projection and MLP GEMMs
+  {
+    const int Mi = (int)M;
+    struct Shape { GemmEpi e; int n, k; bool on; } shapes[] = {
+        {kEpiStore, (int)n_in, (int)d, ssm}, {kEpiResid, (int)d, (int)HP, ssm},
+        {kEpiStore, (int)n_qkv, (int)d, att}, {kEpiResid, (int)d, c->n_q_heads * c->head_dim, att},
+        {kEpiSwiGLU, c->d_ff, (int)d, c->d_ff > 0}, {kEpiResid, (int)d, c->d_ff, c->d_ff > 0}};
+    for (const Shape& sh : shapes) {
+      if (!sh.on) continue;
+      const size_t b = gemm_split_bytes(c->dtype, sh.e, Mi, sh.n, sh.k);
+      if (b > s.gpart_bytes) s.gpart_bytes = b;
+      if (b > 0) {
+        const int nt = gemm_tile_count(c->dtype, sh.e, Mi, sh.n);
+        if (nt > s.gmax_tiles) s.gmax_tiles = nt;
+      }
+    }
+  }
+  s.gpart = off, off += align256(s.gpart_bytes);
+  s.gcnt = off, off += align256((size_t)s.gmax_tiles * 4);
   s.total = off;
   return s;
 }
@@ -565,6 +590,14 @@ hspec_status hspec_draft_step(hspec_drafter* dr, const hspec_step_in* in, const 
   uint8_t* g = ws + sp.g;
   float* h0 = (float*)(ws + sp.h0);
   int* err = device_error_word();
+  if (sp.gmax_tiles > 0 && cudaMemsetAsync(ws + sp.gcnt, 0, (size_t)sp.gmax_tiles * 4, s) != cudaSuccess)
+    FAIL(HSPEC_ERR_CUDA, "clearing the GEMM tile counters failed");
+  // the projection and MLP GEMMs may split K over the step workspace
+  auto split = [&](GemmArgs ga) {
+    ga.part = (float*)(ws + sp.gpart), ga.tile_cnt = (int*)(ws + sp.gcnt);
+    ga.part_bytes = sp.gpart_bytes, ga.max_tiles = sp.gmax_tiles;
+    return ga;
+  };
 
   {
     ProfScope p("embed", s);
@@ -583,7 +616,7 @@ hspec_status hspec_draft_step(hspec_drafter* dr, const hspec_step_in* in, const 
       // in_proj -> [z | x | B | C | dt_raw]
       {
         ProfScope p("in_proj", s);
-        if (!gemm(dtype, kEpiStore, gemm_args(M, n_in, d, xn, d, L.W_in, d, big, n_in), s))
+        if (!gemm(dtype, kEpiStore, split(gemm_args(M, n_in, d, xn, d, L.W_in, d, big, n_in)), s))
           return HSPEC_ERR_UNSUPPORTED;
       }
       // injected initial state h0 = W_inj h_last
@@ -610,12 +643,13 @@ hspec_status hspec_draft_step(hspec_drafter* dr, const hspec_step_in* in, const 
       }
       {
         ProfScope p("out_proj", s);
-        if (!gemm(dtype, kEpiResid, gemm_args(M, d, HP, g, HP, L.W_out, HP, x, d), s)) return HSPEC_ERR_UNSUPPORTED;
+        if (!gemm(dtype, kEpiResid, split(gemm_args(M, d, HP, g, HP, L.W_out, HP, x, d)), s))
+          return HSPEC_ERR_UNSUPPORTED;
       }
     } else {
       {
         ProfScope p("qkv_proj", s);
-        if (!gemm(dtype, kEpiStore, gemm_args(M, n_qkv, d, xn, d, L.W_qkv, d, big, n_qkv), s))
+        if (!gemm(dtype, kEpiStore, split(gemm_args(M, n_qkv, d, xn, d, L.W_qkv, d, big, n_qkv)), s))
           return HSPEC_ERR_UNSUPPORTED;
       }
       if (c->flags & HSPEC_FLAG_ROPE) {
@@ -635,7 +669,7 @@ hspec_status hspec_draft_step(hspec_drafter* dr, const hspec_step_in* in, const 
       }
       {
         ProfScope p("o_proj", s);
-        if (!gemm(dtype, kEpiResid, gemm_args(M, d, Hq * Dh, g, (long)Hq * Dh, L.W_o, (long)Hq * Dh, x, d), s))
+        if (!gemm(dtype, kEpiResid, split(gemm_args(M, d, Hq * Dh, g, (long)Hq * Dh, L.W_o, (long)Hq * Dh, x, d)), s))
           return HSPEC_ERR_UNSUPPORTED;
       }
     }
@@ -649,11 +683,12 @@ hspec_status hspec_draft_step(hspec_drafter* dr, const hspec_step_in* in, const 
       gs.B2 = L.W_up;
       {
         ProfScope p("mlp_gate_up", s);
-        if (!gemm(dtype, kEpiSwiGLU, gs, s)) return HSPEC_ERR_UNSUPPORTED;
+        if (!gemm(dtype, kEpiSwiGLU, split(gs), s)) return HSPEC_ERR_UNSUPPORTED;
       }
       {
         ProfScope p("mlp_down", s);
-        if (!gemm(dtype, kEpiResid, gemm_args(M, d, F, big, F, L.W_down, F, x, d), s)) return HSPEC_ERR_UNSUPPORTED;
+        if (!gemm(dtype, kEpiResid, split(gemm_args(M, d, F, big, F, L.W_down, F, x, d)), s))
+          return HSPEC_ERR_UNSUPPORTED;
       }
     }
     if (out->layer_hidden)

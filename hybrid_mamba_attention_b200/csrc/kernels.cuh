@@ -45,7 +45,17 @@ struct GemmArgs {
   bool out_f32;                // kEpiStore: fp32 output instead of dtype
   float* pval; int32_t* pidx;  // kEpiArgmax partials [M, n_parts]
   int n_parts;
+  // Split-K workspace (optional): with fewer output tiles than SMs the K loop is cut into
+  // splits whose fp32 partials go to `part`; the last split of a tile to finish (counter
+  // in `tile_cnt`, zero on entry and left zero) sums them in split order and applies the
+  // epilogue, so the result does not depend on scheduling.
+  float* part; int* tile_cnt; size_t part_bytes; int max_tiles;
 };
+// Splits of the K loop that gemm() uses for this shape (1 = no split), and the workspace
+// bytes (partials) and counters it then needs.
+int gemm_split_count(int dtype, GemmEpi epi, int M, int N, int K);
+size_t gemm_split_bytes(int dtype, GemmEpi epi, int M, int N, int K);
+int gemm_tile_count(int dtype, GemmEpi epi, int M, int N);
 
 // Column tile width of the argmax partials (n_parts = ceil(N / argmax_tile_n(dtype))).
 int argmax_tile_n(int dtype);
@@ -73,6 +83,11 @@ bool ssd_tc_launch(const SsdArgs& a, cudaStream_t s);
 
 // ------------------------------------------------------------ attn.cu
 constexpr int kAttnTcTile = 64;  // keys per tile of the tensor-core attention path
+constexpr int kAttnTcRows = 128; // query rows per row block (MMA M) of that path
+// chunks of the tensor-core path's tile-space partition: one per SM (auto), or of an
+// explicitly requested length, at most this many (which bounds the partial workspace)
+constexpr int kAttnMaxChunksAuto = 256;
+constexpr int kAttnMaxChunksExplicit = 2048;
 struct AttnArgs {
   int C, K, Hq, Hkv, D;
   const void* q; long q_rs;              // token row stride; head h at column h*D
@@ -82,18 +97,25 @@ struct AttnArgs {
   const void* kb; long kb_rs;            // block keys, kv head g at column g*D
   const void* vb; long vb_rs;
   void* out; long o_rs;                  // dtype, token row stride
-  int split_tokens;                      // tokens per split (multiple of 16)
-  int n_splits;                          // splits per (request, kv head) upper bound
+  int split_tokens;                      // fp32 path: tokens per split (multiple of 16);
+                                         // tensor-core path: chunk length (0 = one per SM)
+  int n_splits;                          // fp32 path: splits per (request, kv head) upper bound
+  int max_chunks;                        // tensor-core path: chunk bound of the workspace
   bool causal_block;
   bool block_in_last_split;              // tensor-core path: block keys ride with the last context split
   int sub_splits;                        // partials per split (tensor-core path: one per softmax warpgroup)
   float* ws_acc; float* ws_ml;           // split partials
+  // tensor-core path: [1] total tiles T, [2] chunk length Z, [3] number of chunks,
+  // written by the schedule kernel; from [64] the tile offsets of the requests (C + 1)
+  int* sched;
   int* err;
 };
 // Split policy (tokens per split, splits per request) and workspace bytes.
 int attn_split_tokens(int dtype, int C, int Hkv, int K, int max_ctx, int requested);
 int attn_num_splits(int dtype, int K, int max_ctx, int split_tokens);
-size_t attn_ws_bytes(int C, int Hkv, int K, int G, int D, int n_splits, int sub_splits);
+// Rows of partials (each D fp32 + (m, l)) and workspace bytes.
+size_t attn_partial_rows(int dtype, int C, int Hkv, int K, int G, int n_splits, int max_chunks);
+size_t attn_ws_bytes(int dtype, int C, int Hkv, int K, int G, int D, int n_splits, int max_chunks);
 int attn_sub_splits(int dtype);
 bool attn_supported(int dtype, int K, int G, int D, const char** why);
 // Checks the pointer / stride requirements of the tensor-core path (bf16).

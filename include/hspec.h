@@ -86,7 +86,10 @@ typedef struct hspec_cfg {
   float rope_theta;                 /* RoPE base                                           */
   float norm_eps;                   /* RMSNorm epsilon                                     */
   int ssd_chunk;                    /* SSD chunk length Q (0 = whole block in one chunk)   */
-  int attn_split_tokens;            /* tokens per split-KV partition, multiple of 16 (0 = auto) */
+  int attn_split_tokens;            /* split-KV partition length in tokens, multiple of 16 (0 = auto):
+                                       fp32, tokens per split of a request; bf16, tiles per chunk of
+                                       the even tile-space partition (rounded up to 64 tokens; at
+                                       most 2048 chunks) -- auto: one chunk per SM */
 } hspec_cfg;
 
 /* Weights of one layer (caller-owned device memory; fields of the other layer kind

@@ -14,7 +14,8 @@ import torch
 
 import oracle
 from hybrid_mamba_attention_b200 import inputs as I
-from tests.parity_util import assert_close, assert_close_stored_bf16, host, rel_max, sample_requests, sub_cache, to_np
+from tests.parity_util import (BF16_TOL, assert_close, assert_close_stored_bf16, half_ulp_bf16, host, rel_max, rel_rms,
+                               sample_requests, sub_cache, to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -220,6 +221,21 @@ def test_attention_repeated_calls_complete_and_agree(H, cuda, name, split):
     assert torch.isfinite(outs[0]).all()
 
 
+@pytest.mark.parametrize("C", [1, 8])
+def test_attention_few_requests_long_contexts(H, cuda, C):
+    # few requests over long contexts: the schedule kernel lengthens the splits (about
+    # one work item per SM) and several warps share each output row in the merge
+    wl = I.full_workload(C, 16)
+    sh = wl.shapes
+    inp = I.make_attn_inputs(sh, wl, wl.K, wl.seed, cuda, shuffle=wl.shuffle, slack=wl.slack)
+    out = run_attn(H, sh, inp, wl.K)
+    again = run_attn(H, sh, inp, wl.K)
+    assert H.hspec_sync_status() == 0, H.hspec_last_error()
+    assert torch.equal(out, again)
+    rows = sample_requests(C, 2, seed=5)
+    compare_attn(to_np(out[rows]), oracle_attn(inp, rows), sh, f"attn C={C}")
+
+
 def test_request_order_permutes_output(H, cuda):
     wl = I.WORKLOADS["llama_c32"]
     sh = wl.shapes
@@ -229,7 +245,17 @@ def test_request_order_permutes_output(H, cuda):
     a = run_attn(H, sh, inp, wl.K)
     b = run_attn(H, sh, p, wl.K)
     assert H.hspec_sync_status() == 0
-    assert torch.equal(a[perm], b)
+    # The tile line follows the batch order, so a request's pieces move with the
+    # permutation, and with them the running max against which P is rounded to bf16
+    # and the fp32 summation order: the outputs agree to that rounding.
+    # Both are stored in bf16, so one rounding flip may add an ulp of the larger value
+    # (up to a few percent of rms(o) at the largest outputs); beyond that ulp they agree
+    # to the bf16 bound.
+    x, y = to_np(a[perm]), to_np(b)
+    rms = np.sqrt((x ** 2).mean())
+    beyond = np.maximum(np.abs(x - y) - 2 * half_ulp_bf16(np.maximum(np.abs(x), np.abs(y))), 0.0).max() / rms
+    print(f"permuted batch: max-abs/rms {rel_rms(y, x):.3e}, beyond one bf16 ulp {beyond:.3e}")
+    assert beyond <= BF16_TOL
 
 
 def test_empty_context_single_token_returns_block_value(H, cuda):

@@ -161,8 +161,12 @@ def test_step_request_permutation(H, cuda):
                kv=[dict(c, page_table=c["page_table"][perm]) for c in st["kv"]])
     a = run_step(H, wl, st, layers=False)
     b = run_step(H, wl, st2, layers=False)
-    assert torch.equal(a["hidden"][perm], b["hidden"])
-    assert torch.equal(a["tokens"][perm], b["tokens"])
+    # the attention's tile line follows the batch order, so the permuted batch sums in
+    # another order: equal up to the bf16 drift of the four-layer step, and the same
+    # draft tokens wherever the logits are not nearly tied
+    assert_close(to_np(b["hidden"]), to_np(a["hidden"][perm]), "bf16", "permuted step")
+    agree = (a["tokens"][perm] == b["tokens"]).float().mean().item()
+    assert agree >= 0.95, f"draft tokens of the permuted batch agree on {agree:.3f}"
 
 
 def test_step_counts_its_kernel_launches(H, cuda):
@@ -183,3 +187,17 @@ def test_profile_groups_cover_the_step(H, cuda):
     for name in ("in_proj", "inject", "ssd_scan", "attn_paged", "mlp_gate_up", "mlp_down", "lm_head_argmax"):
         assert name in prof and prof[name][0] > 0
     assert prof["attn_paged"][1] == 2 and prof["inject"][1] == 2
+
+
+@pytest.mark.parametrize("C", [1, 8])
+def test_split_k_step_repeats_bitwise(H, cuda, C):
+    # at one and eight requests the projection and MLP GEMMs split K across CTAs; the
+    # partials are summed in split order by whichever CTA finishes a tile last, so
+    # repeated steps agree bit for bit
+    wl = I.full_workload(C, 16)
+    st = I.make_step_inputs(wl, cuda)
+    a = run_step(H, wl, st, layers=False)
+    for _ in range(2):
+        b = run_step(H, wl, st, layers=False)
+        assert torch.equal(a["hidden"], b["hidden"])
+        assert torch.equal(a["tokens"], b["tokens"])
