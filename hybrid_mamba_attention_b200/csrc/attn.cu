@@ -1,6 +1,7 @@
 // Paged in-place GQA attention of the K block queries over the target's KV cache
-// followed by the block's own keys (H-Spec Abstract: "attention modules reuse target
-// KVs in place"), split-KV across CTAs, then a merge of the partial softmax states.
+// followed by the block's own keys (H-Spec Abstract: the drafter's attention reads
+// the target's KV cache in place), split-KV across CTAs, then a merge of the partial
+// softmax states.
 // bf16 runs on the tensor cores (attn_tc.cu); this file holds the exact fp32 split
 // kernel, the merge shared by both, and the split policy.
 //

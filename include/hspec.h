@@ -130,8 +130,8 @@ typedef struct hspec_kv_view {
 /* ------------------------------------------------------------------ kernels
  * Each of the three calls below is one step of the draft step, usable alone. */
 
-/* State injection (H-Spec Abstract: "Mamba modules are initialized with projected
- * last-token target hidden states").
+/* State injection (H-Spec Abstract: each Mamba layer starts from a projection of the
+ * target's hidden state at the last token).
  *   h0[c][h][p][n] = sum_j W_inj[(h*P+p)*N+n][j] * h_last[c][j]
  * W_inj  device [H*P*N, d] (dtype); h_last device [C, d] (dtype);
  * h0     device [C, H, P, N] fp32, written.  C >= 1. */
@@ -139,8 +139,8 @@ HSPEC_API hspec_status hspec_inject_state(const hspec_cfg* cfg, const void* W_in
                                 float* h0, void* stream);
 
 /* Mamba-2 SSD scan over the K block positions of every request, started from h0
- * (H-Spec Abstract: "Mamba's parallel scan allows H-Spec to preserve block-parallel
- * drafting"), evaluated in chunks of cfg->ssd_chunk positions:
+ * (H-Spec Abstract: the parallel scan is what keeps the drafting block-parallel),
+ * evaluated in chunks of cfg->ssd_chunk positions:
  *   h_t = exp(dt_t A_h) h_{t-1} + dt_t x_t (x) B_t;  y_t = C_t . h_t + D_h x_t.
  * x  device [C, K, H, P] (dtype);  dt device [C, K, H] fp32 (already positive);
  * A, D device [H] fp32;  B, Cm device [C, K, N] (dtype, one group for all heads);
@@ -152,15 +152,19 @@ HSPEC_API hspec_status hspec_ssd_block_scan(const hspec_cfg* cfg, const void* x,
                                   const float* h0, int C, int K, float* y, float* hK, void* stream);
 
 /* Workspace bytes hspec_attn_paged_block needs for C requests of K block tokens and
- * a page table of width max_pages (the split-KV partials). */
+ * a page table of width max_pages (the split-KV partials; on the bf16 path a fixed
+ * number of partial slots, C * Hkv * ceil(K*G/128) + 256, whatever the width). */
 HSPEC_API size_t hspec_attn_workspace_size(const hspec_cfg* cfg, int C, int K, int max_pages);
 
-/* Paged in-place GQA attention of the K block queries (H-Spec Abstract: "attention
- * modules reuse target KVs in place").  Query (c, j, h) attends, with scale
+/* Paged in-place GQA attention of the K block queries (H-Spec Abstract: the drafter's
+ * attention reads the target's KV cache where it lies, with no copy).  Query (c, j, h) attends, with scale
  * 1/sqrt(D), over the ctx_lens[c] context tokens of request c read through the page
  * table, followed by the K block keys of request c (all visible unless
  * HSPEC_FLAG_CAUSAL_BLOCK); kv head = h / (Hq/Hkv).  Long contexts are split across
- * CTAs and the partial (max, sum, acc) merged.
+ * CTAs and the partial (max, sum, acc) merged.  bf16: the split follows an even
+ * partition of all (request, kv head) key tiles of the call over the SMs, so a
+ * request's result depends on the batch (its order and the other lengths) up to
+ * rounding; calls on the same batch give bit-identical results.
  * q      device [C, K, Hq, D] (dtype);   kv: the target cache;
  * ctx_lens device [C] int32, 0 <= ctx_lens[c] <= kv->max_pages * page_size;
  * k_blk, v_blk device [C, K, Hkv, D] (dtype);
