@@ -17,10 +17,19 @@
 //               epilogue (store, residual add, SwiGLU, per-row argmax), while the
 //               next tile accumulates into the other TMEM buffer.
 // Rows/columns beyond M/N are zero-filled by TMA and skipped by the epilogue.
-// With fewer output tiles than SMs (few token rows) the K loop is split: work unit
-// (tile, split) accumulates its K range, writes the fp32 partial of its rows, and the
-// last unit of a tile to finish (an atomic counter per tile) sums the partials in split
-// order and runs the fused epilogue.
+// When whole tiles would leave SMs idle the K loop is cut, in one of two ways:
+//   stream-K (one row of tiles, M <= 128): the (tile, 64-wide K block) pairs form one
+//     line, tile-major, and CTA b takes its equal chunk [b Z, b Z + Z) of it, walked
+//     as segments, one per tile it crosses.  Only a chunk's first and last segments
+//     can be partial, so chunk k owns partial slots 2k (its first) and 2k + 1 (its
+//     last).  With several rows of tiles this would put the CTAs that share a weight
+//     tile at different K offsets (the weight then comes from HBM once per CTA
+//     instead of once from L2), so there:
+//   split-K (fewer tiles than half the SMs): unit (tile, split) covers an equal K
+//     range, all units start at their range's first block together; slot = unit.
+// A segment covering a whole tile runs the fused epilogue itself; the others write the
+// fp32 partial of their rows to their slot, and the last segment of a tile to finish
+// (an atomic counter per tile) sums the partials in K order and runs the epilogue.
 #include <mutex>
 #include <stdint.h>
 
@@ -87,10 +96,52 @@ __device__ __forceinline__ void epi32(const GemmArgs& g, int m, int nb, float (&
   }
 }
 
+// How the K loop is cut: zk > 0 stream-K chunks of zk K blocks; else `splits` equal K
+// ranges of kps blocks (splits = 1: whole tiles).
+struct KCut {
+  int zk, splits, kps;
+};
+
+// The CTA's work as segments (tile t, K blocks [k0, k1)): stream-K positions
+// [b zk, b zk + zk) of the (tile, K block) line; else units b, b + grid, ... of
+// (tile, split) (unit u = t * splits + split).
+struct SegWalk {
+  int num_k, zk, splits, kps, pos, end;
+  __device__ SegWalk(int nk, int n_tiles, KCut cut) : num_k(nk), zk(cut.zk), splits(cut.splits), kps(cut.kps) {
+    if (zk == 0) {
+      pos = blockIdx.x, end = n_tiles * splits;
+    } else {
+      pos = blockIdx.x * zk;
+      end = min(n_tiles * nk, pos + zk);
+    }
+  }
+  __device__ bool next(int& t, int& k0, int& k1) {
+    if (pos >= end) return false;
+    if (zk == 0) {
+      t = pos / splits;
+      k0 = (pos - t * splits) * kps;
+      k1 = min(num_k, k0 + kps);
+      pos += gridDim.x;
+    } else {
+      t = pos / num_k;
+      k0 = pos - t * num_k;
+      k1 = min(num_k, k0 + (end - pos));
+      pos += k1 - k0;
+    }
+    return true;
+  }
+};
+
+// Partial slot of tile t's segment in chunk k (stream-K): the chunk's first segment if
+// the chunk starts inside the tile, else its last.
+__device__ __forceinline__ int seg_slot(int t, int k, int zk, int num_k) {
+  return 2 * k + ((long)k * zk < (long)t * num_k ? 1 : 0);
+}
+
 template <int EPI>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmB2, GemmArgs g, int splits, int* err) {
+                   const __grid_constant__ CUtensorMap tmB2, GemmArgs g, KCut cut, int* err) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = tc::smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023) & ~1023u) - raw);
@@ -99,16 +150,14 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* acc_full = empty + STAGES;   // [2] accumulator b holds a finished unit
   uint64_t* acc_empty = acc_full + 2;    // [2] the epilogue has read accumulator b
   uint32_t* tmem_slot = (uint32_t*)(acc_empty + 2);
-  volatile int* s_last = (volatile int*)(tmem_slot + 1);  // split-K: this unit finishes its tile
-  volatile int* s_fail = s_last + 1;                      // split-K: an epilogue wait gave up
+  volatile int* s_last = (volatile int*)(tmem_slot + 1);  // stream-K: this segment finishes its tile
+  volatile int* s_fail = s_last + 1;                      // stream-K: an epilogue wait gave up
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ncols_out = (EPI == kEpiSwiGLU) ? BN / 2 : BN;
   const int n_mt = (g.M + BM - 1) / BM;
   const int n_tiles = n_mt * ((g.N + ncols_out - 1) / ncols_out);
   const int num_k = (g.K + BK - 1) / BK;
-  const int kps = (num_k + splits - 1) / splits;  // K blocks per split
-  const int n_units = n_tiles * splits;           // unit u: tile u / splits, split u % splits
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -133,12 +182,12 @@ __global__ void __launch_bounds__(THREADS, 1)
     tc::tma_prefetch_desc(&tmA);
     tc::tma_prefetch_desc(&tmB);
     if (EPI == kEpiSwiGLU) tc::tma_prefetch_desc(&tmB2);
-    int it = 0;  // stage-ring position, continued across units
+    int it = 0;  // stage-ring position, continued across segments
     bool ok = true;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const int t = u / splits, sp = u % splits;
+    SegWalk wk(num_k, n_tiles, cut);
+    int t, k_lo, k_hi;
+    while (ok && wk.next(t, k_lo, k_hi)) {
       const int m0 = (t % n_mt) * BM, n0 = (t / n_mt) * ncols_out;
-      const int k_lo = sp * kps, k_hi = min(num_k, k_lo + kps);
       for (int kt = k_lo; kt < k_hi; ++kt, ++it) {
         const int s = it % STAGES;
         if (!(ok = tc::mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, err))) break;
@@ -159,11 +208,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     constexpr uint32_t idesc = tc::idesc_bf16_f32(BM, BN);
     bool ok = true;
     int it = 0, lt = 0;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++lt) {
-      const int sp = u % splits;
-      const int k_lo = sp * kps, k_hi = min(num_k, k_lo + kps);
+    SegWalk wk(num_k, n_tiles, cut);
+    int t, k_lo, k_hi;
+    for (; ok && wk.next(t, k_lo, k_hi); ++lt) {
       const int b = lt & 1;
-      // accumulator b is free once the epilogue has read the unit two back
+      // accumulator b is free once the epilogue has read the segment two back
       if (!(ok = tc::mbar_wait(&acc_empty[b], ((lt >> 1) & 1) ^ 1, err))) break;
       tc::tc_fence_after();
       const uint32_t d = tmem + (uint32_t)(b * BN);
@@ -187,8 +236,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int quarter = warp & 3;  // TMEM lanes this warp may access
     const int row = quarter * 32 + lane;
     int lt = 0;
-    for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++lt) {
-      const int t = u / splits;
+    SegWalk wk(num_k, n_tiles, cut);
+    int t, k_lo, k_hi;
+    for (; wk.next(t, k_lo, k_hi); ++lt) {
       const int b = lt & 1;
       const int m0 = (t % n_mt) * BM, n0 = (t / n_mt) * ncols_out, ntile = t / n_mt;
       const int m = m0 + row;
@@ -197,14 +247,23 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc::tc_fence_after();
       const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(b * BN);
       float v[32], u2[32];
-      if (splits > 1) {
-        // this split's partial of the unit's rows, then: is this the tile's last split?
-        float* pr = g.part + ((size_t)u * BM + row) * BN;
+      if (k_lo != 0 || k_hi != num_k) {
+        // this segment's partial of the tile's rows, then: is it the tile's last segment?
+        const int zk = cut.zk;
+        // the tile's segments q = 0 .. n_seg - 1 in K order and their slots
+        const int kf = zk ? (int)((long)t * num_k / zk) : 0;
+        const int n_seg = zk ? (int)(((long)t * num_k + num_k - 1) / zk) - kf + 1 : cut.splits;
+        auto slot_of = [&](int q) { return zk ? seg_slot(t, kf + q, zk, num_k) : t * cut.splits + q; };
+        const int my_slot = zk ? seg_slot(t, blockIdx.x, zk, num_k) : t * cut.splits + k_lo / cut.kps;
+        // slot layout [32-column chunk][float4 of the chunk][row]: a warp's stores (32
+        // rows, one float4 each) are 512 contiguous bytes
+        float4* pr = (float4*)(g.part + (size_t)my_slot * BM * BN) + row;
         for (int c = 0; c < BN; c += 32) {
           tc::tmem_ld32(taddr + c, v);
           if (ok && m < g.M)
 #pragma unroll
-            for (int i = 0; i < 32; i += 4) *(float4*)(pr + c + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+            for (int i = 0; i < 8; ++i)
+              pr[((c / 32) * 8 + i) * BM] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
         }
         tc::tc_fence_before();
         __syncwarp();
@@ -213,7 +272,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         // the four epilogue warps pass the same three barriers per unit and leave together
         if (!ok) *s_fail = 1;
         asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (threadIdx.x == 64) *s_last = atomicAdd(&g.tile_cnt[t], 1) == splits - 1;
+        if (threadIdx.x == 64) *s_last = atomicAdd(&g.tile_cnt[t], 1) == n_seg - 1;
         asm volatile("bar.sync 1, 128;" ::: "memory");
         const bool last = *s_last != 0, all_ok = *s_fail == 0;
         asm volatile("bar.sync 1, 128;" ::: "memory");  // s_last is read before the next unit writes it
@@ -224,27 +283,27 @@ __global__ void __launch_bounds__(THREADS, 1)
         __threadfence();
         if (all_ok) {
           // the 128 epilogue threads take (valid row, 32-column chunk) items, so that few
-          // valid rows still spread over all of them; loads of several splits in flight
+          // valid rows still spread over all of them; loads of several segments in flight
+          // rows fastest, so that a warp's loads of one float4 are contiguous
           const int rows_v = min(BM, g.M - m0), nch = ncols_out / 32;
           for (int w = threadIdx.x - 64; w < rows_v * nch; w += 128) {
-            const int r = w / nch, c = (w % nch) * 32;
-            const float* p0 = g.part + ((size_t)(t * splits) * BM + r) * BN + c;
+            const int r = w % rows_v, cc = w / rows_v;
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = 0.f, u2[i] = 0.f;
 #pragma unroll 4
-            for (int q = 0; q < splits; ++q) {  // split order: the same sums whoever finishes last
-              const float* pq = p0 + (size_t)q * BM * BN;
+            for (int q = 0; q < n_seg; ++q) {  // segment order: the same sums whoever finishes last
+              const float4* pq = (const float4*)(g.part + (size_t)slot_of(q) * BM * BN) + r;
 #pragma unroll
-              for (int i = 0; i < 32; i += 4) {
-                const float4 a4 = __ldcg((const float4*)(pq + i));
-                v[i] += a4.x, v[i + 1] += a4.y, v[i + 2] += a4.z, v[i + 3] += a4.w;
+              for (int i = 0; i < 8; ++i) {
+                const float4 a4 = __ldcg(pq + (cc * 8 + i) * BM);
+                v[4 * i] += a4.x, v[4 * i + 1] += a4.y, v[4 * i + 2] += a4.z, v[4 * i + 3] += a4.w;
                 if (EPI == kEpiSwiGLU) {
-                  const float4 b4 = __ldcg((const float4*)(pq + BN / 2 + i));
-                  u2[i] += b4.x, u2[i + 1] += b4.y, u2[i + 2] += b4.z, u2[i + 3] += b4.w;
+                  const float4 b4 = __ldcg(pq + ((cc + BN / 64) * 8 + i) * BM);
+                  u2[4 * i] += b4.x, u2[4 * i + 1] += b4.y, u2[4 * i + 2] += b4.z, u2[4 * i + 3] += b4.w;
                 }
               }
             }
-            epi32<EPI>(g, m0 + r, n0 + c, v, u2);
+            epi32<EPI>(g, m0 + r, n0 + cc * 32, v, u2);
           }
         }
         if (threadIdx.x == 64) g.tile_cnt[t] = 0;  // ready for the next launch
@@ -331,7 +390,7 @@ int device_sms() {
 }
 
 template <int EPI>
-bool launch_tc(const GemmArgs& g, int splits, cudaStream_t s, int* err) {
+bool launch_tc(const GemmArgs& g, KCut cut, cudaStream_t s, int* err) {
   static bool attr_set[64] = {};
   static int n_sm[64] = {};
   int dev = 0;
@@ -355,10 +414,12 @@ bool launch_tc(const GemmArgs& g, int splits, cudaStream_t s, int* err) {
     return false;
   }
   const int ncols_out = (EPI == kEpiSwiGLU) ? BN / 2 : BN;
-  const long n_units = (long)cdiv(g.M, BM) * cdiv(g.N, ncols_out) * splits;
+  const long n_tiles = (long)cdiv(g.M, BM) * cdiv(g.N, ncols_out);
+  // chunks, or (tile, split) units
+  const long n_units = cut.zk > 0 ? cdiv(n_tiles * cdiv(g.K, BK), cut.zk) : n_tiles * cut.splits;
   const int sms = dev < 64 && n_sm[dev] > 0 ? n_sm[dev] : 148;
   const int grid = n_units < sms ? (int)n_units : sms;
-  gemm_tc_kernel<EPI><<<grid, THREADS, SMEM_BYTES, s>>>(ta, tb, tb2, g, splits, err);
+  gemm_tc_kernel<EPI><<<grid, THREADS, SMEM_BYTES, s>>>(ta, tb, tb2, g, cut, err);
   note_launch();
   return true;
 }
@@ -374,22 +435,42 @@ int gemm_tile_count(int dtype, GemmEpi epi, int M, int N) {
   return cdiv(M, BM) * cdiv(N, epi == kEpiSwiGLU ? BN / 2 : BN);
 }
 
-// Split K when the output has fewer tiles than SMs: about one unit per SM, at least
-// four 64-wide K blocks per split, every split non-empty.
-int gemm_split_count(int dtype, GemmEpi epi, int M, int N, int K) {
-  if (dtype != HSPEC_DTYPE_BF16 || epi == kEpiArgmax) return 1;
-  const int n_tiles = gemm_tile_count(dtype, epi, M, N), num_k = cdiv(K, BK), sms = device_sms();
-  if (n_tiles <= 0 || n_tiles * 2 > sms) return 1;
-  int sp = sms / n_tiles;
+// How gemm() cuts the K loop of this shape (see the kernel's header):
+//   one row of tiles, and whole tiles would leave more than 8% of the last wave idle
+//   (within 8 waves): stream-K, an equal share of the line per SM, chunks of at least
+//   4 K blocks;
+//   several rows, fewer tiles than half the SMs: about one (tile, split) unit per SM,
+//   at least four K blocks per split, every split non-empty;
+//   else whole tiles.
+KCut gemm_kcut(int dtype, GemmEpi epi, int M, int N, int K) {
+  KCut cut{0, 1, cdiv(K, BK)};
+  if (dtype != HSPEC_DTYPE_BF16 || epi == kEpiArgmax) return cut;
+  const long n_tiles = gemm_tile_count(dtype, epi, M, N), num_k = cdiv(K, BK), sms = device_sms();
+  if (n_tiles <= 0) return cut;
+  if (cdiv(M, BM) == 1) {
+    if (n_tiles >= 8 * sms) return cut;
+    const long waves = cdiv(n_tiles, sms);
+    if ((double)n_tiles / (double)(waves * sms) >= 0.92) return cut;
+    const long zk = cdiv(n_tiles * num_k, sms);
+    if (zk >= 4) cut.zk = (int)zk;
+    return cut;
+  }
+  if (n_tiles * 2 > sms) return cut;
+  long sp = sms / n_tiles;
   if (sp > num_k / 4) sp = num_k / 4;
-  if (sp < 2) return 1;
-  const int kps = cdiv(num_k, sp);
-  return cdiv(num_k, kps);
+  if (sp < 2) return cut;
+  cut.kps = cdiv(num_k, sp);
+  cut.splits = cdiv(num_k, cut.kps);
+  return cut;
 }
 
-size_t gemm_split_bytes(int dtype, GemmEpi epi, int M, int N, int K) {
-  const int sp = gemm_split_count(dtype, epi, M, N, K);
-  return sp > 1 ? (size_t)gemm_tile_count(dtype, epi, M, N) * sp * BM * BN * sizeof(float) : 0;
+// Partial tiles a cut K loop needs: two per stream-K chunk, one per split unit (at most
+// one unit per SM), BM x BN fp32 each.
+size_t gemm_kcut_bytes(int dtype, GemmEpi epi, int M, int N, int K) {
+  const KCut cut = gemm_kcut(dtype, epi, M, N, K);
+  if (cut.zk > 0) return (size_t)2 * device_sms() * BM * BN * sizeof(float);
+  if (cut.splits > 1) return (size_t)gemm_tile_count(dtype, epi, M, N) * cut.splits * BM * BN * sizeof(float);
+  return 0;
 }
 
 bool gemm(int dtype, GemmEpi epi, const GemmArgs& g, cudaStream_t s) {
@@ -405,18 +486,18 @@ bool gemm(int dtype, GemmEpi epi, const GemmArgs& g, cudaStream_t s) {
     return false;
   }
   int* err = device_error_word();
-  int splits = 1;
+  KCut cut{0, 1, cdiv(g.K, BK)};
   if (g.part && g.tile_cnt && !(epi == kEpiStore && g.out_f32)) {
-    const int sp = gemm_split_count(dtype, epi, g.M, g.N, g.K);
-    if (sp > 1 && gemm_split_bytes(dtype, epi, g.M, g.N, g.K) <= g.part_bytes &&
+    const KCut c = gemm_kcut(dtype, epi, g.M, g.N, g.K);
+    if ((c.zk > 0 || c.splits > 1) && gemm_kcut_bytes(dtype, epi, g.M, g.N, g.K) <= g.part_bytes &&
         gemm_tile_count(dtype, epi, g.M, g.N) <= g.max_tiles && !(((uintptr_t)g.part) & 15))
-      splits = sp;
+      cut = c;
   }
   switch (epi) {
-    case kEpiStore: return launch_tc<kEpiStore>(g, splits, s, err);
-    case kEpiResid: return launch_tc<kEpiResid>(g, splits, s, err);
-    case kEpiSwiGLU: return launch_tc<kEpiSwiGLU>(g, splits, s, err);
-    case kEpiArgmax: return launch_tc<kEpiArgmax>(g, splits, s, err);
+    case kEpiStore: return launch_tc<kEpiStore>(g, cut, s, err);
+    case kEpiResid: return launch_tc<kEpiResid>(g, cut, s, err);
+    case kEpiSwiGLU: return launch_tc<kEpiSwiGLU>(g, cut, s, err);
+    case kEpiArgmax: return launch_tc<kEpiArgmax>(g, cut, s, err);
   }
   return false;
 }

@@ -222,7 +222,7 @@ struct StepPlan {
   size_t x, xn, big, y, g, h0, attn, pval, pidx, gpart, gcnt, total;
   AttnPlan ap;
   int n_parts;
-  size_t gpart_bytes;  // split-K partials of the projections / MLP GEMMs
+  size_t gpart_bytes;  // partials of the projection / MLP GEMMs with a cut K loop
   int gmax_tiles;      // tile counters that follow them
 };
 
@@ -262,7 +262,7 @@ StepPlan step_plan(const hspec_cfg* c, int C, int K, int max_pages) {
         {kEpiSwiGLU, c->d_ff, (int)d, c->d_ff > 0}, {kEpiResid, (int)d, c->d_ff, c->d_ff > 0}};
     for (const Shape& sh : shapes) {
       if (!sh.on) continue;
-      const size_t b = gemm_split_bytes(c->dtype, sh.e, Mi, sh.n, sh.k);
+      const size_t b = gemm_kcut_bytes(c->dtype, sh.e, Mi, sh.n, sh.k);
       if (b > s.gpart_bytes) s.gpart_bytes = b;
       if (b > 0) {
         const int nt = gemm_tile_count(c->dtype, sh.e, Mi, sh.n);

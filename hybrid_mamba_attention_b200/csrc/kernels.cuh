@@ -45,16 +45,16 @@ struct GemmArgs {
   bool out_f32;                // kEpiStore: fp32 output instead of dtype
   float* pval; int32_t* pidx;  // kEpiArgmax partials [M, n_parts]
   int n_parts;
-  // Split-K workspace (optional): with fewer output tiles than SMs the K loop is cut into
-  // splits whose fp32 partials go to `part`; the last split of a tile to finish (counter
-  // in `tile_cnt`, zero on entry and left zero) sums them in split order and applies the
+  // Workspace of a cut K loop (optional): when whole tiles would leave SMs idle the K
+  // loop is cut (stream-K or split-K); segments that cover part of a tile write fp32
+  // partials to `part`, and the last segment of a tile to finish (counter in
+  // `tile_cnt`, zero on entry and left zero) sums them in K order and applies the
   // epilogue, so the result does not depend on scheduling.
   float* part; int* tile_cnt; size_t part_bytes; int max_tiles;
 };
-// Splits of the K loop that gemm() uses for this shape (1 = no split), and the workspace
-// bytes (partials) and counters it then needs.
-int gemm_split_count(int dtype, GemmEpi epi, int M, int N, int K);
-size_t gemm_split_bytes(int dtype, GemmEpi epi, int M, int N, int K);
+// Workspace bytes (partials) that gemm() needs for this shape when it cuts the K loop
+// (stream-K or split-K; 0 for whole tiles); counters: gemm_tile_count().
+size_t gemm_kcut_bytes(int dtype, GemmEpi epi, int M, int N, int K);
 int gemm_tile_count(int dtype, GemmEpi epi, int M, int N);
 
 // Column tile width of the argmax partials (n_parts = ceil(N / argmax_tile_n(dtype))).

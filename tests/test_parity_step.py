@@ -189,11 +189,11 @@ def test_profile_groups_cover_the_step(H, cuda):
     assert prof["attn_paged"][1] == 2 and prof["inject"][1] == 2
 
 
-@pytest.mark.parametrize("C", [1, 8])
-def test_split_k_step_repeats_bitwise(H, cuda, C):
-    # at one and eight requests the projection and MLP GEMMs split K across CTAs; the
-    # partials are summed in split order by whichever CTA finishes a tile last, so
-    # repeated steps agree bit for bit
+@pytest.mark.parametrize("C", [1, 8, 32])
+def test_stream_k_step_repeats_bitwise(H, cuda, C):
+    # at these batch sizes the projection and MLP GEMMs run stream-K (tiles cut across
+    # CTAs); the partials are summed in segment order by whichever CTA finishes a tile
+    # last, so repeated steps agree bit for bit
     wl = I.full_workload(C, 16)
     st = I.make_step_inputs(wl, cuda)
     a = run_step(H, wl, st, layers=False)
