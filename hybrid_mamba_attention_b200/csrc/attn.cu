@@ -29,6 +29,8 @@ constexpr int kTile = 16;
 
 template <typename T, int TPR>
 __global__ void __launch_bounds__(kThreads) attn_split_kernel(AttnArgs a, float scale_log2) {
+  pdl_wait();  // the previous kernel on the stream is complete from here on
+  pdl_trigger();
   extern __shared__ float sm[];
   const int D = a.D, Dp = D + 1;
   float* sK = sm;                           // [kTile][D+1]
@@ -147,6 +149,8 @@ __global__ void __launch_bounds__(kThreads) attn_split_kernel(AttnArgs a, float 
 // 4 lane .. 4 lane + 3 (float4 loads); else lane + 32 i.
 template <typename T, int W, bool V4>
 __global__ void __launch_bounds__(256) attn_merge_kernel(AttnArgs a) {
+  pdl_wait();  // the previous kernel on the stream is complete from here on
+  pdl_trigger();
   constexpr int RPC = 8 / W;  // rows per CTA
   __shared__ float s_acc[W > 1 ? 8 : 1][128];
   __shared__ float s_ml[8][2];
@@ -300,7 +304,7 @@ template <typename T, int TPR>
 void launch_split(const AttnArgs& a, cudaStream_t s) {
   const size_t smem = (size_t)2 * kTile * (a.D + 1) * sizeof(float);
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)a.D);
-  attn_split_kernel<T, TPR><<<dim3(a.n_splits, a.Hkv, a.C), kThreads, smem, s>>>(a, scale_log2);
+  launch_pdl(attn_split_kernel<T, TPR>, dim3(a.n_splits, a.Hkv, a.C), kThreads, smem, s, a, scale_log2);
   note_launch();
 }
 
@@ -323,8 +327,8 @@ void launch_simt(const AttnArgs& a, cudaStream_t s) {
 template <typename T, int W>
 void launch_merge_w(const AttnArgs& a, long rows, cudaStream_t s) {
   const int grid = (int)((rows + 8 / W - 1) / (8 / W));
-  if (a.D % 4 == 0) attn_merge_kernel<T, W, true><<<grid, 256, 0, s>>>(a);
-  else attn_merge_kernel<T, W, false><<<grid, 256, 0, s>>>(a);
+  if (a.D % 4 == 0) launch_pdl(attn_merge_kernel<T, W, true>, grid, 256, 0, s, a);
+  else launch_pdl(attn_merge_kernel<T, W, false>, grid, 256, 0, s, a);
   note_launch();
 }
 

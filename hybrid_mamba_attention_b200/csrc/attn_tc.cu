@@ -115,6 +115,8 @@ __device__ __forceinline__ int seq_tiles(int ctx, long max_ctx, int nbt) {
 __global__ void __launch_bounds__(1024) attn_sched_kernel(const int32_t* ctx_lens, int C, long max_ctx, int nbt,
                                                           int spr, int grid, int z_req, int max_chunks, int* sched,
                                                           int* off, int* err) {
+  pdl_wait();  // the previous kernel on the stream is complete from here on
+  pdl_trigger();
   __shared__ int part[1024];
   const int per = (C + 1023) / 1024;
   const int c0 = min(C, (int)threadIdx.x * per), c1 = min(C, c0 + per);
@@ -211,6 +213,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // the previous kernel on the stream is complete from here on
+  pdl_trigger();
 
   if (warp < NPW) {
     // ------------------------------------------------------------ producers
@@ -731,11 +735,11 @@ bool launch_tc(const AttnArgs& a, cudaStream_t s) {
   const int sms = dev < 64 && n_sm[dev] > 0 ? n_sm[dev] : 148;
   const int grid = min(sms, kAttnMaxChunksAuto);
   const int z_req = a.split_tokens > 0 ? (a.split_tokens + TT - 1) / TT : 0;
-  attn_sched_kernel<<<1, 1024, 0, s>>>(a.ctx_lens, a.C, (long)a.max_pages * a.page_size, (a.K + TT - 1) / TT,
+  launch_pdl(attn_sched_kernel, 1, 1024, 0, s, a.ctx_lens, a.C, (long)a.max_pages * a.page_size, (a.K + TT - 1) / TT,
                                        a.Hkv * n_rb, grid, z_req, a.max_chunks, a.sched, a.sched + 64, a.err);
   note_launch();
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
-  attn_tc_kernel<D, SP><<<grid, THREADS, Lay<D, SP>::SMEM, s>>>(maps, a, scale_log2, n_rb);
+  launch_pdl(attn_tc_kernel<D, SP>, grid, THREADS, Lay<D, SP>::SMEM, s, maps, a, scale_log2, n_rb);
   note_launch();
   return true;
 }

@@ -55,6 +55,16 @@ __device__ __forceinline__ void flag_error(int* err, int bits) {
   if (err) atomicOr(err, bits);
 }
 
+// Programmatic dependent launch.  A kernel launched with launch_pdl() may start while
+// the previous kernel on its stream is still running: it does its own set-up (shared
+// memory barriers, TMEM, descriptor prefetch), then every thread passes pdl_wait()
+// -- which returns once the previous grid has completed and its memory is visible --
+// before it reads or writes any global memory.  pdl_trigger() lets the next kernel
+// launch (its threads still wait for this grid to complete).  Both are no-ops when the
+// kernel was launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- host side
 
 // Counts a kernel launch of this library (reported by hspec_launch_count).
@@ -64,5 +74,26 @@ void note_launch(int n = 1);
 void set_error(const char* fmt, ...);
 
 inline int cdiv(long a, long b) { return (int)((a + b - 1) / b); }
+
+// Whether launch_pdl() sets the programmatic-serialization attribute (HSPEC_PDL=1 in the
+// environment; off by default).
+bool pdl_enabled();
+
+// Launches `kernel` on `s`, allowed to start before the previous kernel on the stream
+// has finished (the kernel must call pdl_wait() before touching global memory).
+template <typename... KArgs, typename... Args>
+void launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
 
 }  // namespace hspec

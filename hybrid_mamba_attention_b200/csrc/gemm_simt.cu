@@ -16,6 +16,8 @@ constexpr int BM = 64, BN = 64, BK = 16, PAD = 4;
 
 template <int EPI>
 __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmArgs g) {
+  pdl_wait();  // the previous kernel on the stream is complete from here on
+  pdl_trigger();
   __shared__ float As[BK][BM + PAD];
   __shared__ float Bs[BK][BN + PAD];
   __shared__ float B2s[EPI == kEpiSwiGLU ? BK : 1][BN + PAD];
@@ -107,10 +109,10 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmArgs g) {
 void gemm_simt_f32(GemmEpi epi, const GemmArgs& g, cudaStream_t s) {
   dim3 grid(cdiv(g.N, BN), cdiv(g.M, BM));
   switch (epi) {
-    case kEpiStore: gemm_simt_kernel<kEpiStore><<<grid, 256, 0, s>>>(g); break;
-    case kEpiResid: gemm_simt_kernel<kEpiResid><<<grid, 256, 0, s>>>(g); break;
-    case kEpiSwiGLU: gemm_simt_kernel<kEpiSwiGLU><<<grid, 256, 0, s>>>(g); break;
-    case kEpiArgmax: gemm_simt_kernel<kEpiArgmax><<<grid, 256, 0, s>>>(g); break;
+    case kEpiStore: launch_pdl(gemm_simt_kernel<kEpiStore>, grid, 256, 0, s, g); break;
+    case kEpiResid: launch_pdl(gemm_simt_kernel<kEpiResid>, grid, 256, 0, s, g); break;
+    case kEpiSwiGLU: launch_pdl(gemm_simt_kernel<kEpiSwiGLU>, grid, 256, 0, s, g); break;
+    case kEpiArgmax: launch_pdl(gemm_simt_kernel<kEpiArgmax>, grid, 256, 0, s, g); break;
   }
   note_launch();
 }

@@ -176,6 +176,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // the previous kernel on the stream is complete from here on
+  pdl_trigger();
 
   if (warp == 0 && lane == 0) {
     // ---------------------------------------------------------- TMA producer
@@ -419,7 +421,7 @@ bool launch_tc(const GemmArgs& g, KCut cut, cudaStream_t s, int* err) {
   const long n_units = cut.zk > 0 ? cdiv(n_tiles * cdiv(g.K, BK), cut.zk) : n_tiles * cut.splits;
   const int sms = dev < 64 && n_sm[dev] > 0 ? n_sm[dev] : 148;
   const int grid = n_units < sms ? (int)n_units : sms;
-  gemm_tc_kernel<EPI><<<grid, THREADS, SMEM_BYTES, s>>>(ta, tb, tb2, g, cut, err);
+  launch_pdl(gemm_tc_kernel<EPI>, grid, THREADS, SMEM_BYTES, s, ta, tb, tb2, g, cut, err);
   note_launch();
   return true;
 }

@@ -14,6 +14,8 @@ constexpr int kRowThreads = 256;
 template <typename T>
 __global__ void embed_kernel(const int32_t* __restrict__ tokens, const T* __restrict__ table, int vocab,
                              float* __restrict__ x, int d, int* err) {
+  pdl_wait();  // the previous kernel on the stream is complete from here on
+  pdl_trigger();
   const int m = blockIdx.x;
   const int tok = tokens[m];
   const bool ok = tok >= 0 && tok < vocab;
@@ -24,6 +26,8 @@ __global__ void embed_kernel(const int32_t* __restrict__ tokens, const T* __rest
 
 template <typename T>
 __global__ void to_f32_kernel(const T* __restrict__ in, float* __restrict__ x, long n) {
+  pdl_wait();  // the previous kernel on the stream is complete from here on
+  pdl_trigger();
   for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x)
     x[i] = to_f(in[i]);
 }
@@ -32,6 +36,8 @@ __global__ void to_f32_kernel(const T* __restrict__ in, float* __restrict__ x, l
 template <typename T>
 __global__ void rmsnorm_kernel(const float* __restrict__ x, const float* __restrict__ w,
                                T* __restrict__ out, int n, float eps) {
+  pdl_wait();  // the previous kernel on the stream is complete from here on
+  pdl_trigger();
   __shared__ float red[32];
   const float* row = x + (size_t)blockIdx.x * n;
   float ss = 0.f;
@@ -69,6 +75,8 @@ template <typename T>
 __global__ void __launch_bounds__(kRowThreads) rmsnorm_v4_kernel(const float* __restrict__ x,
                                                                  const float* __restrict__ w,
                                                                  T* __restrict__ out, int n, float eps) {
+  pdl_wait();  // the previous kernel on the stream is complete from here on
+  pdl_trigger();
   __shared__ float red[32];
   const int n4 = n / 4;
   const float4* row = (const float4*)(x + (size_t)blockIdx.x * n);
@@ -98,6 +106,8 @@ __global__ void __launch_bounds__(kRowThreads) gated_rmsnorm_v4_kernel(const flo
                                                                        const T* __restrict__ z, long z_stride,
                                                                        const float* __restrict__ w,
                                                                        T* __restrict__ out, int n, float eps) {
+  pdl_wait();  // the previous kernel on the stream is complete from here on
+  pdl_trigger();
   __shared__ float red[32];
   const int n4 = n / 4;
   const float* yr = y + (size_t)blockIdx.x * n;
@@ -135,6 +145,8 @@ template <typename T>
 __global__ void __launch_bounds__(kRowThreads) rope_rows_kernel(T* __restrict__ qkv, long row_stride,
                                                                 const int32_t* __restrict__ ctx_lens, int K,
                                                                 int n_heads, int D, double log_theta) {
+  pdl_wait();  // the previous kernel on the stream is complete from here on
+  pdl_trigger();
   const int half = D / 2, groups = kRowThreads / half;
   const int t = threadIdx.x, i = t % half, hg = t / half;
   if (hg >= groups) return;
@@ -158,6 +170,8 @@ template <typename T>
 __global__ void gated_rmsnorm_kernel(const float* __restrict__ y, const T* __restrict__ z, long z_stride,
                                      const float* __restrict__ w, T* __restrict__ out, int n, float eps,
                                      bool gate) {
+  pdl_wait();  // the previous kernel on the stream is complete from here on
+  pdl_trigger();
   __shared__ float red[32];
   const float* yr = y + (size_t)blockIdx.x * n;
   T* o = out + (size_t)blockIdx.x * n;
@@ -183,6 +197,8 @@ __global__ void gated_rmsnorm_kernel(const float* __restrict__ y, const T* __res
 template <typename T>
 __global__ void rope_kernel(T* __restrict__ qkv, long row_stride, const int32_t* __restrict__ ctx_lens,
                             int K, int n_heads, int D, double log_theta, long total) {
+  pdl_wait();  // the previous kernel on the stream is complete from here on
+  pdl_trigger();
   const long idx = blockIdx.x * (long)blockDim.x + threadIdx.x;
   if (idx >= total) return;
   const int half = D / 2;
@@ -206,6 +222,8 @@ __global__ void rope_kernel(T* __restrict__ qkv, long row_stride, const int32_t*
 __global__ void argmax_reduce_kernel(const float* __restrict__ pval, const int32_t* __restrict__ pidx,
                                      int M, int n_parts, int32_t* __restrict__ tokens,
                                      float* __restrict__ top) {
+  pdl_wait();  // the previous kernel on the stream is complete from here on
+  pdl_trigger();
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (warp >= M) return;
   float best = -INFINITY;
@@ -232,9 +250,9 @@ __global__ void argmax_reduce_kernel(const float* __restrict__ pval, const int32
 void embed_rows(int dtype, const int32_t* tokens, const void* table, int vocab, float* x, int M, int d,
                 int* err, cudaStream_t s) {
   if (dtype == HSPEC_DTYPE_BF16)
-    embed_kernel<bf16><<<M, kRowThreads, 0, s>>>(tokens, (const bf16*)table, vocab, x, d, err);
+    launch_pdl(embed_kernel<bf16>, M, kRowThreads, 0, s, tokens, (const bf16*)table, vocab, x, d, err);
   else
-    embed_kernel<float><<<M, kRowThreads, 0, s>>>(tokens, (const float*)table, vocab, x, d, err);
+    launch_pdl(embed_kernel<float>, M, kRowThreads, 0, s, tokens, (const float*)table, vocab, x, d, err);
   note_launch();
 }
 
@@ -242,9 +260,9 @@ void rows_to_f32(int dtype, const void* in, float* x, long n, cudaStream_t s) {
   int grid = (int)((n + kRowThreads - 1) / kRowThreads);
   if (grid > 148 * 16) grid = 148 * 16;
   if (dtype == HSPEC_DTYPE_BF16)
-    to_f32_kernel<bf16><<<grid, kRowThreads, 0, s>>>((const bf16*)in, x, n);
+    launch_pdl(to_f32_kernel<bf16>, grid, kRowThreads, 0, s, (const bf16*)in, x, n);
   else
-    to_f32_kernel<float><<<grid, kRowThreads, 0, s>>>((const float*)in, x, n);
+    launch_pdl(to_f32_kernel<float>, grid, kRowThreads, 0, s, (const float*)in, x, n);
   note_launch();
 }
 
@@ -252,12 +270,12 @@ void rmsnorm_rows(int dtype, const float* x, const float* w, void* out, int M, i
                   cudaStream_t s) {
   const bool v4 = n % 4 == 0 && n <= 4 * kRowThreads * kV4 && !(((uintptr_t)x | (uintptr_t)w | (uintptr_t)out) & 15);
   if (v4) {
-    if (dtype == HSPEC_DTYPE_BF16) rmsnorm_v4_kernel<bf16><<<M, kRowThreads, 0, s>>>(x, w, (bf16*)out, n, eps);
-    else rmsnorm_v4_kernel<float><<<M, kRowThreads, 0, s>>>(x, w, (float*)out, n, eps);
+    if (dtype == HSPEC_DTYPE_BF16) launch_pdl(rmsnorm_v4_kernel<bf16>, M, kRowThreads, 0, s, x, w, (bf16*)out, n, eps);
+    else launch_pdl(rmsnorm_v4_kernel<float>, M, kRowThreads, 0, s, x, w, (float*)out, n, eps);
   } else if (dtype == HSPEC_DTYPE_BF16)
-    rmsnorm_kernel<bf16><<<M, kRowThreads, 0, s>>>(x, w, (bf16*)out, n, eps);
+    launch_pdl(rmsnorm_kernel<bf16>, M, kRowThreads, 0, s, x, w, (bf16*)out, n, eps);
   else
-    rmsnorm_kernel<float><<<M, kRowThreads, 0, s>>>(x, w, (float*)out, n, eps);
+    launch_pdl(rmsnorm_kernel<float>, M, kRowThreads, 0, s, x, w, (float*)out, n, eps);
   note_launch();
 }
 
@@ -268,15 +286,15 @@ void gated_rmsnorm_rows(int dtype, const float* y, const void* z, long z_stride,
                   !(((uintptr_t)y | (uintptr_t)w | (uintptr_t)out) & 15) && !(((uintptr_t)z) & 7);
   if (v4) {
     if (dtype == HSPEC_DTYPE_BF16)
-      gated_rmsnorm_v4_kernel<bf16><<<M, kRowThreads, 0, s>>>(y, (const bf16*)z, z_stride, w, (bf16*)out, n, eps);
+      launch_pdl(gated_rmsnorm_v4_kernel<bf16>, M, kRowThreads, 0, s, y, (const bf16*)z, z_stride, w, (bf16*)out, n, eps);
     else
-      gated_rmsnorm_v4_kernel<float><<<M, kRowThreads, 0, s>>>(y, (const float*)z, z_stride, w, (float*)out, n,
+      launch_pdl(gated_rmsnorm_v4_kernel<float>, M, kRowThreads, 0, s, y, (const float*)z, z_stride, w, (float*)out, n,
                                                                eps);
   } else if (dtype == HSPEC_DTYPE_BF16)
-    gated_rmsnorm_kernel<bf16><<<M, kRowThreads, 0, s>>>(y, (const bf16*)z, z_stride, w, (bf16*)out, n,
+    launch_pdl(gated_rmsnorm_kernel<bf16>, M, kRowThreads, 0, s, y, (const bf16*)z, z_stride, w, (bf16*)out, n,
                                                          eps, gate);
   else
-    gated_rmsnorm_kernel<float><<<M, kRowThreads, 0, s>>>(y, (const float*)z, z_stride, w, (float*)out,
+    launch_pdl(gated_rmsnorm_kernel<float>, M, kRowThreads, 0, s, y, (const float*)z, z_stride, w, (float*)out,
                                                           n, eps, gate);
   note_launch();
 }
@@ -288,14 +306,14 @@ void rope_rows(int dtype, void* qkv, long row_stride, const int32_t* ctx_lens, i
   const double lt = log((double)theta);
   if (D % 2 == 0 && D / 2 <= kRowThreads) {
     if (dtype == HSPEC_DTYPE_BF16)
-      rope_rows_kernel<bf16><<<C * K, kRowThreads, 0, s>>>((bf16*)qkv, row_stride, ctx_lens, K, n_heads, D, lt);
+      launch_pdl(rope_rows_kernel<bf16>, C * K, kRowThreads, 0, s, (bf16*)qkv, row_stride, ctx_lens, K, n_heads, D, lt);
     else
-      rope_rows_kernel<float><<<C * K, kRowThreads, 0, s>>>((float*)qkv, row_stride, ctx_lens, K, n_heads, D, lt);
+      launch_pdl(rope_rows_kernel<float>, C * K, kRowThreads, 0, s, (float*)qkv, row_stride, ctx_lens, K, n_heads, D, lt);
   } else if (dtype == HSPEC_DTYPE_BF16)
-    rope_kernel<bf16><<<grid, kRowThreads, 0, s>>>((bf16*)qkv, row_stride, ctx_lens, K, n_heads, D, lt,
+    launch_pdl(rope_kernel<bf16>, grid, kRowThreads, 0, s, (bf16*)qkv, row_stride, ctx_lens, K, n_heads, D, lt,
                                                    total);
   else
-    rope_kernel<float><<<grid, kRowThreads, 0, s>>>((float*)qkv, row_stride, ctx_lens, K, n_heads, D,
+    launch_pdl(rope_kernel<float>, grid, kRowThreads, 0, s, (float*)qkv, row_stride, ctx_lens, K, n_heads, D,
                                                     lt, total);
   note_launch();
 }
@@ -303,8 +321,7 @@ void rope_rows(int dtype, void* qkv, long row_stride, const int32_t* ctx_lens, i
 void argmax_reduce(const float* pval, const int32_t* pidx, int M, int n_parts, int32_t* tokens,
                    float* top, cudaStream_t s) {
   const int warps_per_block = 8;
-  argmax_reduce_kernel<<<(M + warps_per_block - 1) / warps_per_block, 32 * warps_per_block, 0, s>>>(
-      pval, pidx, M, n_parts, tokens, top);
+  launch_pdl(argmax_reduce_kernel, (M + warps_per_block - 1) / warps_per_block, 32 * warps_per_block, 0, s, pval, pidx, M, n_parts, tokens, top);
   note_launch();
 }
 

@@ -45,6 +45,8 @@ __host__ __device__ inline SsdSmem ssd_layout(int P, int N, int Q) {
 
 template <typename T, typename TDT>
 __global__ void __launch_bounds__(kThreads) ssd_chunk_kernel(SsdArgs a) {
+  pdl_wait();  // the previous kernel on the stream is complete from here on
+  pdl_trigger();
   extern __shared__ float sm[];
   const int h = blockIdx.x, c = blockIdx.y;
   const int P = a.P, N = a.N, K = a.K, Q = a.Q, Np = N + 1, Qp = Q + 1;
@@ -236,7 +238,7 @@ void launch(const SsdArgs& a, cudaStream_t s) {
     cudaFuncSetAttribute(ssd_chunk_kernel<T, TDT>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
     attr_set[dev] = true;
   }
-  ssd_chunk_kernel<T, TDT><<<dim3(a.H, a.C), kThreads, bytes, s>>>(a);
+  launch_pdl(ssd_chunk_kernel<T, TDT>, dim3(a.H, a.C), kThreads, bytes, s, a);
   note_launch();
 }
 

@@ -176,6 +176,8 @@ __global__ void __launch_bounds__(THREADS, 1) ssd_tc_kernel(const __grid_constan
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // the previous kernel on the stream is complete from here on
+  pdl_trigger();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -488,7 +490,7 @@ bool launch_ssd_tc(const SsdArgs& a, cudaStream_t s) {
   t.n_items = a.C * t.n_tiles;
   const int sms = dev < 64 && n_sm[dev] > 0 ? n_sm[dev] : 148;
   const int grid = t.n_items < sms ? t.n_items : sms;
-  ssd_tc_kernel<TDT><<<grid, THREADS, SsdTcLay::SMEM, s>>>(map, t);
+  launch_pdl(ssd_tc_kernel<TDT>, grid, THREADS, SsdTcLay::SMEM, s, map, t);
   note_launch();
   return true;
 }
