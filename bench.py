@@ -173,7 +173,9 @@ def step_work(sh, C, K, ctx_lens):
         w[name] = {"flops": 2.0 * m * n * k, "bytes": float(n * k * E + m * k * E + extra_bytes)}
 
     gemm("in_proj", M, n_in, d, M * n_in * E)
-    gemm("inject", C, HPN, d, C * HPN * 4)
+    # the draft step as benchmarked stores h0 (the fused injection readout is opt-in)
+    fused = False
+    gemm("inject", C, HPN, d, M * (N + H) * E + M * HP * 8 if fused else C * HPN * 4)
     gemm("out_proj", M, d, HP, M * d * 8)
     gemm("qkv_proj", M, n_qkv, d, M * n_qkv * E)
     gemm("o_proj", M, d, sh.Hq * sh.D, M * d * 8)
@@ -184,8 +186,12 @@ def step_work(sh, C, K, ctx_lens):
         gemm("lm_head_argmax", M, sh.vocab, d)
     w["attn_paged"] = {"flops": 4.0 * sh.Hq * sh.D * K * (ctx_sum + C * K),
                        "bytes": float(kv_bytes + 2 * M * sh.Hq * sh.D * E + 2 * M * sh.Hkv * sh.D * E)}
-    w["ssd_scan"] = {"flops": float(C * H * (2 * K * P * N + K * K * (N + P))),
-                     "bytes": float(C * HPN * 4 + M * (HP + 2 * N + H) * E + M * HP * 4)}
+    if fused:  # zero-state scan: in-block terms and D x only
+        w["ssd_scan"] = {"flops": float(C * H * K * K * (N + P)),
+                         "bytes": float(M * (HP + 2 * N + H) * E + M * HP * 4)}
+    else:
+        w["ssd_scan"] = {"flops": float(C * H * (2 * K * P * N + K * K * (N + P))),
+                         "bytes": float(C * HPN * 4 + M * (HP + 2 * N + H) * E + M * HP * 4)}
     return w
 
 

@@ -312,7 +312,85 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (!all_ok) break;
         continue;
       }
-      if (EPI == kEpiArgmax) {
+      if (EPI == kEpiSsdRead) {
+        // The tile's 256 columns are the two state rows hp0, hp0 + 1 (d_state 128) of
+        // one head h of request m: add their readout C_t . h0[hp] times the head's decay
+        // to y.  All loads of a round are issued before their use -- dt of 16 positions,
+        // C of 4 positions x 32 states (shared by both rows), y as float2 pairs -- so a
+        // tile costs a few L2 round trips.  TMEM loads by all lanes; global memory only
+        // for valid rows.
+        const SsdReadArgs& r = g.ssd;
+        const bool live = ok && m < g.M;
+        const bf16* cm = (const bf16*)r.Cm;
+        const bf16* dtr = (const bf16*)r.dt_raw;
+        const int hp0 = n0 / 128, h = hp0 / r.P;
+        const float Ah = r.A[h], bias = r.dt_bias ? r.dt_bias[h] : 0.f;
+        float cum = 0.f;
+        for (int t0 = 0; t0 < r.K; t0 += 16) {
+          const int tn = min(16, r.K - t0);
+          float e[16], acc0[16], acc1[16];
+#pragma unroll
+          for (int t = 0; t < 16; ++t) {
+            float dt = 0.f;
+            if (live && t < tn) dt = __bfloat162float(dtr[((size_t)m * r.K + t0 + t) * r.dt_rs + h]);
+            e[t] = dt;
+            acc0[t] = 0.f, acc1[t] = 0.f;
+          }
+#pragma unroll
+          for (int t = 0; t < 16; ++t) {
+            float dt = e[t];
+            if (r.dt_bias) dt = softplus(dt + bias);
+            cum += t < tn ? dt * Ah : 0.f;
+            e[t] = expf(cum);
+          }
+          for (int cb = 0; cb < 128; cb += 32) {
+            float v1[32];
+            tc::tmem_ld32(taddr + cb, v);
+            tc::tmem_ld32(taddr + 128 + cb, v1);
+            if (!live) continue;
+#pragma unroll
+            for (int tg = 0; tg < 16; tg += 4) {
+              if (tg >= tn) break;
+              uint4 w[4][4];
+#pragma unroll
+              for (int t = 0; t < 4; ++t) {
+                const int tt = min(tg + t, tn - 1);
+                const uint4* cp = (const uint4*)(cm + ((size_t)m * r.K + t0 + tt) * r.c_rs + cb);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) w[t][q] = __ldg(cp + q);
+              }
+#pragma unroll
+              for (int t = 0; t < 4; ++t) {
+                float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                  const uint32_t wv[4] = {w[t][q].x, w[t][q].y, w[t][q].z, w[t][q].w};
+#pragma unroll
+                  for (int k = 0; k < 4; ++k) {
+                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv[k]));
+                    a0 = fmaf(f.x, v[q * 8 + 2 * k], a0);
+                    a0 = fmaf(f.y, v[q * 8 + 2 * k + 1], a0);
+                    a1 = fmaf(f.x, v1[q * 8 + 2 * k], a1);
+                    a1 = fmaf(f.y, v1[q * 8 + 2 * k + 1], a1);
+                  }
+                }
+                acc0[tg + t] += a0;
+                acc1[tg + t] += a1;
+              }
+            }
+          }
+          if (!live) continue;
+          float2 yv[16];
+#pragma unroll
+          for (int t = 0; t < 16; ++t)
+            if (t < tn) yv[t] = *(const float2*)(r.y + ((size_t)m * r.K + t0 + t) * r.y_rs + hp0);
+#pragma unroll
+          for (int t = 0; t < 16; ++t)
+            if (t < tn)
+              *(float2*)(r.y + ((size_t)m * r.K + t0 + t) * r.y_rs + hp0) =
+                  make_float2(fmaf(e[t], acc0[t], yv[t].x), fmaf(e[t], acc1[t], yv[t].y));
+        }
+      } else if (EPI == kEpiArgmax) {
         float best = -INFINITY;
         int bidx = 0x7fffffff;
         for (int c = 0; c < BN; c += 32) {
@@ -446,7 +524,7 @@ int gemm_tile_count(int dtype, GemmEpi epi, int M, int N) {
 //   else whole tiles.
 KCut gemm_kcut(int dtype, GemmEpi epi, int M, int N, int K) {
   KCut cut{0, 1, cdiv(K, BK)};
-  if (dtype != HSPEC_DTYPE_BF16 || epi == kEpiArgmax) return cut;
+  if (dtype != HSPEC_DTYPE_BF16 || epi == kEpiArgmax || epi == kEpiSsdRead) return cut;
   const long n_tiles = gemm_tile_count(dtype, epi, M, N), num_k = cdiv(K, BK), sms = device_sms();
   if (n_tiles <= 0) return cut;
   if (cdiv(M, BM) == 1) {
@@ -477,8 +555,17 @@ size_t gemm_kcut_bytes(int dtype, GemmEpi epi, int M, int N, int K) {
 
 bool gemm(int dtype, GemmEpi epi, const GemmArgs& g, cudaStream_t s) {
   if (dtype != HSPEC_DTYPE_BF16) {
+    if (epi == kEpiSsdRead) {
+      set_error("the SSD readout epilogue is bf16-only");
+      return false;
+    }
     gemm_simt_f32(epi, g, s);
     return true;
+  }
+  if (epi == kEpiSsdRead && (g.ssd.N != 128 || g.ssd.P % 2 || g.ssd.c_rs % 8 || g.ssd.y_rs % 2 ||
+                             (((uintptr_t)g.ssd.Cm) & 15) || (((uintptr_t)g.ssd.y) & 7))) {
+    set_error("SSD readout epilogue: d_state 128, even head dim, 16-byte aligned C rows, 8-byte aligned y");
+    return false;
   }
   // TMA needs 16-byte aligned bases and row strides.
   if ((g.lda % 8) || (g.ldb % 8) || (((uintptr_t)g.A) & 15) || (((uintptr_t)g.B) & 15) ||
@@ -500,6 +587,7 @@ bool gemm(int dtype, GemmEpi epi, const GemmArgs& g, cudaStream_t s) {
     case kEpiResid: return launch_tc<kEpiResid>(g, cut, s, err);
     case kEpiSwiGLU: return launch_tc<kEpiSwiGLU>(g, cut, s, err);
     case kEpiArgmax: return launch_tc<kEpiArgmax>(g, cut, s, err);
+    case kEpiSsdRead: return launch_tc<kEpiSsdRead>(g, cut, s, err);
   }
   return false;
 }

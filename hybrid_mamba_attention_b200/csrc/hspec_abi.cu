@@ -138,7 +138,7 @@ hspec_status validate_cfg(const hspec_cfg* c, bool need_attn, bool need_ssm) {
   if (!c) FAIL(HSPEC_ERR_INVALID_ARG, "cfg is NULL");
   if (c->dtype != HSPEC_DTYPE_F32 && c->dtype != HSPEC_DTYPE_BF16)
     FAIL(HSPEC_ERR_INVALID_ARG, "dtype %d is neither HSPEC_DTYPE_F32 nor HSPEC_DTYPE_BF16", c->dtype);
-  if (c->flags & ~(HSPEC_FLAG_ROPE | HSPEC_FLAG_GATE | HSPEC_FLAG_CAUSAL_BLOCK))
+  if (c->flags & ~(HSPEC_FLAG_ROPE | HSPEC_FLAG_GATE | HSPEC_FLAG_CAUSAL_BLOCK | HSPEC_FLAG_FUSE_INJECT))
     FAIL(HSPEC_ERR_INVALID_ARG, "unknown flag bits 0x%x", c->flags);
   if (c->d_model <= 0) FAIL(HSPEC_ERR_INVALID_ARG, "d_model must be positive");
   if (need_attn) {
@@ -228,6 +228,19 @@ AttnArgs attn_args(const hspec_cfg* c, const AttnPlan& p, const hspec_kv_view* k
   return a;
 }
 
+// bf16 draft step with HSPEC_FLAG_FUSE_INJECT: the injected state's share of the SSD
+// output is added in the injection GEMM's epilogue (h0 never stored; the scan runs
+// from a zero state).  Default: h0 stored, read by the tensor-core scan -- measured
+// faster from 8 requests up (the epilogue's L2 reads of C stall the weight stream, and
+// the zero-state CUDA-core scan costs more than the tensor-core readout it replaces).
+bool step_fuses_inject(const hspec_cfg* c) {
+  const int N = c->d_state;
+  const long HP = (long)c->n_ssm_heads * c->ssm_head_dim;
+  const long n_in = 2 * HP + 2L * N + c->n_ssm_heads;
+  return c->dtype == HSPEC_DTYPE_BF16 && (c->flags & HSPEC_FLAG_FUSE_INJECT) && N == 128 && c->ssm_head_dim % 2 == 0 &&
+         n_in % 8 == 0 && (2 * HP + N) % 8 == 0 && HP % 2 == 0;
+}
+
 // Step workspace layout (all sub-buffers 256-byte aligned).
 struct StepPlan {
   size_t x, xn, big, y, g, h0, attn, pval, pidx, gpart, gcnt, total;
@@ -255,7 +268,7 @@ StepPlan step_plan(const hspec_cfg* c, int C, int K, int max_pages) {
   s.big = off, off += align256(M * big * E);
   s.y = off, off += align256(ssm ? M * HP * 4 : 0);
   s.g = off, off += align256(M * gw * E);
-  s.h0 = off, off += align256(ssm ? (size_t)C * HPN * 4 : 0);
+  s.h0 = off, off += align256(ssm && !step_fuses_inject(c) ? (size_t)C * HPN * 4 : 0);
   s.attn = off;
   if (att) {
     s.ap = attn_plan(c, C, K, max_pages);
@@ -630,23 +643,43 @@ hspec_status hspec_draft_step(hspec_drafter* dr, const hspec_step_in* in, const 
         if (!gemm(dtype, kEpiStore, split(gemm_args(M, n_in, d, xn, d, L.W_in, d, big, n_in)), s))
           return HSPEC_ERR_UNSUPPORTED;
       }
-      // injected initial state h0 = W_inj h_last
-      GemmArgs gi = gemm_args(C, (int)HPN, d, in->h_last, d, L.W_inj, d, h0, HPN);
-      gi.out_f32 = true;
-      {
-        ProfScope p("inject", s);
-        if (!gemm(dtype, kEpiStore, gi, s)) return HSPEC_ERR_UNSUPPORTED;
-      }
       SsdArgs a = {};
       a.C = C, a.K = K, a.H = H, a.P = P, a.N = N, a.Q = ssd_chunk_len(c, K);
       a.x = big + (size_t)HP * E, a.x_rs = n_in;
       a.dt = big + (size_t)(2 * HP + 2 * N) * E, a.dt_rs = n_in, a.dt_bias = L.dt_bias;
       a.A = L.A, a.D = L.D;
       a.B = big + (size_t)(2 * HP) * E, a.Cm = big + (size_t)(2 * HP + N) * E, a.bc_rs = n_in;
-      a.h0 = h0, a.y = y, a.y_rs = HP, a.hK = nullptr;
-      {
-        ProfScope p("ssd_scan", s);
-        ssd_scan(dtype, a, s);
+      a.y = y, a.y_rs = HP, a.hK = nullptr;
+      if (step_fuses_inject(c)) {
+        // y = the scan from a zero state (in-block terms, D x), then the injection GEMM
+        // adds exp(cum_t) C_t . h0 from its accumulator: h0 = W_inj h_last is never stored
+        a.h0 = nullptr;
+        {
+          ProfScope p("ssd_scan", s);
+          ssd_scan(dtype, a, s);
+        }
+        GemmArgs gi = gemm_args(C, (int)HPN, d, in->h_last, d, L.W_inj, d, nullptr, 0);
+        gi.ssd.K = K, gi.ssd.P = P, gi.ssd.N = N;
+        gi.ssd.Cm = a.Cm, gi.ssd.c_rs = n_in;
+        gi.ssd.dt_raw = a.dt, gi.ssd.dt_rs = n_in, gi.ssd.dt_bias = L.dt_bias, gi.ssd.A = L.A;
+        gi.ssd.y = y, gi.ssd.y_rs = HP;
+        {
+          ProfScope p("inject", s);
+          if (!gemm(dtype, kEpiSsdRead, gi, s)) return HSPEC_ERR_UNSUPPORTED;
+        }
+      } else {
+        // injected initial state h0 = W_inj h_last, stored, then the scan from it
+        GemmArgs gi = gemm_args(C, (int)HPN, d, in->h_last, d, L.W_inj, d, h0, HPN);
+        gi.out_f32 = true;
+        {
+          ProfScope p("inject", s);
+          if (!gemm(dtype, kEpiStore, gi, s)) return HSPEC_ERR_UNSUPPORTED;
+        }
+        a.h0 = h0;
+        {
+          ProfScope p("ssd_scan", s);
+          ssd_scan(dtype, a, s);
+        }
       }
       {
         ProfScope p("gated_norm", s);

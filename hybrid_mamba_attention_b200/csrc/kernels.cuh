@@ -34,6 +34,21 @@ enum GemmEpi : int {
   kEpiResid = 1,      // x (fp32) += acc
   kEpiSwiGLU = 2,     // out (dtype) = silu(acc(B)) * acc(B2)
   kEpiArgmax = 3,     // (pval, pidx)[m][n_tile] = per-row max / argmax over the tile's columns
+  kEpiSsdRead = 4,    // bf16 only, acc = injected state h0: y += decay * (C . h0) (see SsdReadArgs)
+};
+
+// kEpiSsdRead (d_state N = 128, even P): the injection GEMM (row m = request c, column
+// (h*P + p)*N + n of h0) adds the initial state's share of the SSD output without
+// storing h0:
+//   y[c*K + t][h*P + p] += exp(sum_{s<=t} dt[c,s,h] A[h]) * sum_n C[c*K + t][n] * h0[c][h][p][n]
+// with dt = softplus(dt_raw + dt_bias) (dt_raw, C: dtype rows of the in-projection).
+struct SsdReadArgs {
+  int K, P, N;
+  const void* Cm; long c_rs;       // C [C*K, N] (dtype), row stride
+  const void* dt_raw; long dt_rs;  // [C*K, H] (dtype), row stride
+  const float* dt_bias;            // [H]
+  const float* A;                  // [H]
+  float* y; long y_rs;             // [C*K, H*P] fp32, row stride
 };
 
 struct GemmArgs {
@@ -51,6 +66,7 @@ struct GemmArgs {
   // `tile_cnt`, zero on entry and left zero) sums them in K order and applies the
   // epilogue, so the result does not depend on scheduling.
   float* part; int* tile_cnt; size_t part_bytes; int max_tiles;
+  SsdReadArgs ssd;             // kEpiSsdRead
 };
 // Workspace bytes (partials) that gemm() needs for this shape when it cuts the K loop
 // (stream-K or split-K; 0 for whole tiles); counters: gemm_tile_count().

@@ -14,6 +14,9 @@
 // y_t = C_t . h_t + D x_t.  The state S [P][N] lives in shared memory in fp32 (padded
 // rows so that a warp reading one column across 32 rows hits 32 banks); the chunk
 // pass between chunks is the only sequential part.  Everything is fp32 FMA.
+// Stateless form (no h0, no final state, one chunk): S is always zero, so it has no
+// shared memory and the readout term is skipped -- the in-block terms and D x only
+// (the draft step adds the h0 term in the injection GEMM's epilogue).
 #include "../../include/hspec.h"
 #include "common.cuh"
 #include "kernels.cuh"
@@ -28,11 +31,11 @@ struct SsdSmem {
   int S, xs, Bs, Cs, dts, cum, w, CB, total;
 };
 
-__host__ __device__ inline SsdSmem ssd_layout(int P, int N, int Q) {
+__host__ __device__ inline SsdSmem ssd_layout(int P, int N, int Q, bool stateless = false) {
   SsdSmem L;
   const int Np = N + 1, Qp = Q + 1;
   L.S = 0;
-  L.xs = L.S + P * Np;
+  L.xs = L.S + (stateless ? 0 : P * Np);
   L.Bs = L.xs + Q * P;
   L.Cs = L.Bs + Q * Np;
   L.dts = L.Cs + Q * Np;
@@ -50,7 +53,8 @@ __global__ void __launch_bounds__(kThreads) ssd_chunk_kernel(SsdArgs a) {
   extern __shared__ float sm[];
   const int h = blockIdx.x, c = blockIdx.y;
   const int P = a.P, N = a.N, K = a.K, Q = a.Q, Np = N + 1, Qp = Q + 1;
-  const SsdSmem L = ssd_layout(P, N, Q);
+  const bool stateless = !a.h0 && !a.hK && Q >= K;
+  const SsdSmem L = ssd_layout(P, N, Q, stateless);
   float* S = sm + L.S;     // [P][N+1] state entering the chunk
   float* xs = sm + L.xs;   // [Q][P]   x of the chunk (later x * weight into the chunk-end state)
   float* Bs = sm + L.Bs;   // [Q][N+1]
@@ -69,7 +73,8 @@ __global__ void __launch_bounds__(kThreads) ssd_chunk_kernel(SsdArgs a) {
 
   // initial state (the injected h0, or zero)
   const float* h0 = a.h0 ? a.h0 + ((size_t)c * a.H + h) * P * N : nullptr;
-  if (h0 && (N % 4) == 0) {
+  if (stateless) {
+  } else if (h0 && (N % 4) == 0) {
     const float4* h4 = (const float4*)h0;
     for (int i = tid; i < P * N / 4; i += kThreads) {
       const float4 v = h4[i];
@@ -138,7 +143,7 @@ __global__ void __launch_bounds__(kThreads) ssd_chunk_kernel(SsdArgs a) {
         tr[i] = min(4 * tb + i, q - 1);
         pr[i] = min(4 * pb + i, P - 1);
       }
-      for (int n = nq; n < N; n += 4) {
+      for (int n = stateless ? N : nq; n < N; n += 4) {  // S = 0 in the stateless form
         float cv[4], sv[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -230,7 +235,8 @@ __global__ void __launch_bounds__(kThreads) ssd_chunk_kernel(SsdArgs a) {
 
 template <typename T, typename TDT>
 void launch(const SsdArgs& a, cudaStream_t s) {
-  const size_t bytes = ssd_smem_bytes(a.P, a.N, a.Q);
+  const bool stateless = !a.h0 && !a.hK && a.Q >= a.K;
+  const size_t bytes = (size_t)ssd_layout(a.P, a.N, a.Q, stateless).total * sizeof(float);
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);

@@ -28,6 +28,7 @@ HSPEC_DTYPE_BF16 = 1
 HSPEC_FLAG_ROPE = 1
 HSPEC_FLAG_GATE = 2
 HSPEC_FLAG_CAUSAL_BLOCK = 4
+HSPEC_FLAG_FUSE_INJECT = 8
 HSPEC_MAX_LAYERS = 16
 
 # Every function include/hspec.h declares (checked by the CPU export test).
@@ -143,11 +144,11 @@ def _stream(stream):
 
 # --------------------------------------------------------------- config helpers
 
-def make_cfg(shapes, ssd_chunk: int = 0, attn_split_tokens: int = 0) -> hspec_cfg:
+def make_cfg(shapes, ssd_chunk: int = 0, attn_split_tokens: int = 0, fuse_inject: bool = False) -> hspec_cfg:
     """hspec_cfg from an inputs.Shapes (or any object with the same fields)."""
     sh = shapes
     flags = (HSPEC_FLAG_ROPE if sh.use_rope else 0) | (HSPEC_FLAG_GATE if sh.use_gate else 0) | (
-        HSPEC_FLAG_CAUSAL_BLOCK if sh.causal_block else 0)
+        HSPEC_FLAG_CAUSAL_BLOCK if sh.causal_block else 0) | (HSPEC_FLAG_FUSE_INJECT if fuse_inject else 0)
     return hspec_cfg(d_model=sh.d, n_q_heads=sh.Hq, n_kv_heads=sh.Hkv, head_dim=sh.D, n_ssm_heads=sh.H,
                      ssm_head_dim=sh.P, d_state=sh.N, page_size=sh.page, d_ff=sh.d_ff, vocab=sh.vocab,
                      n_layers=len(sh.layers), layer_kinds=sh.layers.encode(),
@@ -267,9 +268,10 @@ def hspec_profile_read(max_entries: int = 64) -> dict:
 class Drafter:
     """Holds a drafter handle plus the weights it points at (kept alive here)."""
 
-    def __init__(self, shapes, weights: dict, ssd_chunk: int = 0, attn_split_tokens: int = 0):
+    def __init__(self, shapes, weights: dict, ssd_chunk: int = 0, attn_split_tokens: int = 0,
+                 fuse_inject: bool = False):
         self.shapes = shapes
-        self.cfg = make_cfg(shapes, ssd_chunk, attn_split_tokens)
+        self.cfg = make_cfg(shapes, ssd_chunk, attn_split_tokens, fuse_inject)
         self.weights = weights
         mw = hspec_model_weights()
         for i, w in enumerate(weights["layers"]):

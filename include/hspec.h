@@ -63,6 +63,10 @@ typedef int hspec_status;
 #define HSPEC_FLAG_ROPE 1           /* rotary embedding on q and block keys at ctx_c + j */
 #define HSPEC_FLAG_GATE 2           /* Mamba-2 gated RMSNorm y <- norm(y * silu(z)) w_g  */
 #define HSPEC_FLAG_CAUSAL_BLOCK 4   /* block query j sees block key i only when i <= j   */
+#define HSPEC_FLAG_FUSE_INJECT 8    /* bf16 draft step, d_state 128: the injection GEMM   */
+                                    /* adds h0's share of the scan output from its        */
+                                    /* accumulator (h0 never stored) after a zero-state   */
+                                    /* scan; default: h0 stored and read by the scan      */
 
 #define HSPEC_MAX_LAYERS 16
 

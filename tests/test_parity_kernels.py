@@ -111,6 +111,19 @@ def test_ssd_chunk_length_is_only_an_evaluation_order(H, cuda, K, chunks):
         assert_close(to_np(y), ref, "f32", f"ssd K={K} chunk={q}")
 
 
+@pytest.mark.parametrize("name,C,K", [("llama_c32", 6, 16), ("qwen_c128", 3, 16), ("llama_c32", 4, 7)])
+def test_ssd_stateless_scan_matches_zero_state_recurrence(H, cuda, name, C, K):
+    # No h0, no final state, one chunk: the stateless form (no state in shared memory,
+    # no readout) that the bf16 draft step runs before the injection GEMM adds the h0 term
+    sh = I.WORKLOADS[name].shapes
+    inp = I.make_ssd_inputs(sh, C, K, 41 + C, cuda)
+    y, _ = run_ssd(H, sh, inp, K, h0=False)
+    zero = torch.zeros_like(host(inp["h0"]))
+    ref = oracle.ssd_scan(host(inp["x"]), host(inp["dt"]), host(inp["A"]), host(inp["B"]), host(inp["Cm"]),
+                          host(inp["D"]), zero, want_state=False)
+    assert_close(to_np(y), ref, "f32", f"stateless ssd {name} C={C} K={K}")
+
+
 def test_ssd_zero_injection_equals_zero_state(H, cuda):
     sh = I.TINY
     inp = I.make_ssd_inputs(sh, 2, 8, 5, cuda)
