@@ -55,6 +55,7 @@ class Shapes:
     layers: str = "MA"      # layer kinds in order, M = Mamba-2, A = attention
     d_ff: int = 0           # SwiGLU intermediate size, 0 = no MLP sub-layer
     vocab: int = 0          # LM head rows, 0 = no head (output is the hidden state)
+    draft_vocab: int = 0    # reduced draft head rows (0 = the full vocab head)
     page: int = PAGE
     eps: float = 1e-6
     use_rope: bool = True
@@ -123,9 +124,13 @@ FULL_SWEEP_K = (8, 16, 32)
 FULL_SWEEP_C = (1, 8, 32, 128)
 
 
-def full_workload(C: int, K: int) -> Workload:
-    """One point of the full-step sweep (K in {8,16,32} x C in {1,8,32,128})."""
-    return replace(WORKLOADS["full"], C=C, K=K, name=f"full_C{C}_K{K}")
+def full_workload(C: int, K: int, draft_vocab: int = 0) -> Workload:
+    """One point of the full-step sweep (K in {8,16,32} x C in {1,8,32,128}); with
+    draft_vocab, the same drafter with a reduced draft head of that many rows."""
+    wl = replace(WORKLOADS["full"], C=C, K=K, name=f"full_C{C}_K{K}")
+    if draft_vocab:
+        wl = replace(wl, shapes=replace(wl.shapes, draft_vocab=draft_vocab), name=f"full_C{C}_K{K}_V{draft_vocab}")
+    return wl
 
 
 # ----------------------------------------------------------------------------- rng
@@ -201,6 +206,13 @@ def make_weights(sh: Shapes, seed: int, device="cpu") -> dict:
     if sh.vocab:
         out["final_norm"] = _randn((sh.d,), 0.1, torch.float32, device, seed, "final_norm", mean=1.0)
         out["W_lm"] = _randn((sh.vocab, sh.d), 1 / math.sqrt(sh.d), dt, device, seed, "W_lm")
+        if sh.draft_vocab:
+            # reduced draft head: its own rows, each standing for one target token (a seeded
+            # subset of the vocabulary, in increasing id order)
+            out["W_lm_draft"] = _randn((sh.draft_vocab, sh.d), 1 / math.sqrt(sh.d), dt, device, seed, "W_lm_draft")
+            g = _gen(seed, "draft_to_target", "cpu")
+            ids = torch.randperm(sh.vocab, generator=g)[: sh.draft_vocab].sort().values
+            out["draft_to_target"] = ids.to(torch.int32).to(device)
     return out
 
 

@@ -216,7 +216,8 @@ class _Layer(ct.Structure):
 class _Step(ct.Structure):
     _fields_ = [("C", ct.c_int), ("K", ct.c_int), ("tokens", ct.c_void_p), ("x_in", ct.c_void_p),
                 ("x_in_type", ct.c_int), ("h_last", ct.c_void_p), ("ctx_lens", ct.c_void_p), ("final_norm", ct.c_void_p),
-                ("W_lm", ct.c_void_p), ("hidden", ct.c_void_p), ("layer_out", ct.c_void_p),
+                ("W_lm", ct.c_void_p), ("draft_vocab", ct.c_int), ("W_lm_draft", ct.c_void_p),
+                ("draft_to_target", ct.c_void_p), ("hidden", ct.c_void_p), ("layer_out", ct.c_void_p),
                 ("final_normed", ct.c_void_p), ("draft_tokens", ct.c_void_p), ("top1", ct.c_void_p),
                 ("top2", ct.c_void_p)]
 
@@ -281,6 +282,12 @@ def draft_step(shapes, weights, kv, h_last, ctx_lens, tokens=None, x_in=None, la
         io.tokens = tok.data_ptr()
         io.final_norm = hold(weights["final_norm"], True)
         io.W_lm = hold(weights["W_lm"])
+        if getattr(sh, "draft_vocab", 0):
+            io.draft_vocab = sh.draft_vocab
+            io.W_lm_draft = hold(weights["W_lm_draft"])
+            d2t = _i32(weights["draft_to_target"])
+            keep.append(d2t)
+            io.draft_to_target = d2t.data_ptr()
         res["final_normed"] = _f64_out(C, K, sh.d)
         res["draft_tokens"] = np.zeros((C, K), dtype=np.int32)
         res["top1"], res["top2"] = _f64_out(C, K), _f64_out(C, K)

@@ -413,9 +413,13 @@ int oracle_draft_step(const oracle_cfg* cfg, const oracle_layer* layers, oracle_
         for (size_t i = 0; i < xn.size(); ++i) io->final_normed[(size_t)c * K * d + i] = xn[i];
       std::vector<int32_t> am(K);
       std::vector<double> t1(K), t2(K);
-      lm_head_argmax(K, d, cfg->vocab, xn.data(), io->W_lm, dtype, am.data(), t1.data(), t2.data());
+      // full head, or the reduced draft head whose row r stands for target token
+      // draft_to_target[r] (argmax over the draft rows, lowest row on ties)
+      const bool reduced = io->draft_vocab > 0;
+      lm_head_argmax(K, d, reduced ? io->draft_vocab : cfg->vocab, xn.data(), reduced ? io->W_lm_draft : io->W_lm,
+                     dtype, am.data(), t1.data(), t2.data());
       for (int j = 0; j < K; ++j) {
-        if (io->draft_tokens) io->draft_tokens[(size_t)c * K + j] = am[j];
+        if (io->draft_tokens) io->draft_tokens[(size_t)c * K + j] = reduced ? io->draft_to_target[am[j]] : am[j];
         if (io->top1) io->top1[(size_t)c * K + j] = t1[j];
         if (io->top2) io->top2[(size_t)c * K + j] = t2[j];
       }

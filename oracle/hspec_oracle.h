@@ -110,6 +110,11 @@ typedef struct {
   const void* h_last;      /* [C,d] target last-token hidden state */
   const int32_t* ctx_lens; /* [C] */
   const float* final_norm; const void* W_lm;   /* [d], [vocab,d]; W_lm is also the embedding */
+  /* reduced-vocabulary draft head (draft_vocab > 0): logits over W_lm_draft [draft_vocab,d]
+   * and the draft token draft_to_target[argmax] (evolve.pub review of H-Spec, Frequently
+   * asked questions: the drafter's vocabulary may be cut to 32k frequent tokens; the
+   * target's verification keeps the output exact).  draft_vocab = 0: the full W_lm head. */
+  int draft_vocab; const void* W_lm_draft; const int32_t* draft_to_target;
   /* outputs (any may be NULL) */
   double* hidden;          /* [C,K,d] residual stream after the last layer */
   double* layer_out;       /* [n_layers,C,K,d] residual stream after each layer */

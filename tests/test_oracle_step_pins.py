@@ -202,3 +202,36 @@ def test_bf16_step_stays_close_to_fp32_step():
     h16 = run_oracle(w16, st16)["hidden"]
     rel = np.abs(h16 - h32).max() / np.sqrt((h32 ** 2).mean())
     assert rel < 0.1
+
+
+def test_reduced_draft_head_is_the_full_head_restricted_and_remapped():
+    # Reduced-vocabulary draft head (evolve.pub review of H-Spec, Frequently asked
+    # questions: the drafter's vocabulary cut to frequent tokens): with the draft rows
+    # taken from the full head (W_lm_draft = W_lm[ids]), the draft token is the target id
+    # whose logit is highest among ids, read from the full head's own final hidden state.
+    sh = replace(SMALL_FULL, draft_vocab=97)
+    w = wl(sh)
+    st = I.make_step_inputs(w)
+    ids = st["weights"]["draft_to_target"]
+    assert ids.shape == (97,) and bool((ids[1:] > ids[:-1]).all()) and int(ids.max()) < sh.vocab
+    st["weights"]["W_lm_draft"] = st["weights"]["W_lm"][ids.long()].clone()
+    full = run_oracle(wl(SMALL_FULL), st)
+    got = run_oracle(w, st)
+    np.testing.assert_array_equal(got["hidden"], full["hidden"])
+    logits = torch.from_numpy(full["final_normed"]) @ d64(st["weights"]["W_lm"]).T  # [C,K,V]
+    sub = logits[..., ids.long()]
+    want = ids.long()[sub.argmax(-1)].numpy()
+    assert np.array_equal(got["draft_tokens"], want)
+    np.testing.assert_allclose(got["top1"], sub.max(-1).values.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_reduced_draft_head_with_every_id_in_order_is_the_full_head():
+    sh = replace(SMALL_FULL, draft_vocab=SMALL_FULL.vocab)
+    w = wl(sh)
+    st = I.make_step_inputs(w)
+    assert torch.equal(st["weights"]["draft_to_target"].long(), torch.arange(sh.vocab))
+    st["weights"]["W_lm_draft"] = st["weights"]["W_lm"].clone()
+    full = run_oracle(wl(SMALL_FULL), st)
+    got = run_oracle(w, st)
+    for k in ("draft_tokens", "top1", "top2"):
+        assert np.array_equal(got[k], full[k])
