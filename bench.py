@@ -183,7 +183,7 @@ def step_work(sh, C, K, ctx_lens):
         gemm("mlp_gate_up", M, 2 * sh.d_ff, d, M * sh.d_ff * E)
         gemm("mlp_down", M, d, sh.d_ff, M * d * 8)
     if sh.vocab:
-        gemm("lm_head_argmax", M, sh.vocab, d)
+        gemm("lm_head_argmax", M, sh.draft_vocab or sh.vocab, d)
     w["attn_paged"] = {"flops": 4.0 * sh.Hq * sh.D * K * (ctx_sum + C * K),
                        "bytes": float(kv_bytes + 2 * M * sh.Hq * sh.D * E + 2 * M * sh.Hkv * sh.D * E)}
     if fused:  # zero-state scan: in-block terms and D x only
@@ -351,7 +351,7 @@ def run_ours(args, rank, world, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     peaks = load_peaks()
-    wl = replica_workload(I, I.full_workload(args.C, args.K), rank)
+    wl = replica_workload(I, I.full_workload(args.C, args.K, args.draft_vocab), rank)
     clocks = ClockSampler(local)
     clocks.start()  # before the inputs are built: sampling by the time the steps run
     runner = StepRunner(H, I, wl, dev)
@@ -398,7 +398,7 @@ def run_ours(args, rank, world, local):
             if C == wl.C and K == wl.K:
                 m2, lens2 = ms_max, runner.st["ctx_lens"].cpu()
             else:
-                w2 = I.full_workload(C, K)
+                w2 = I.full_workload(C, K, args.draft_vocab)
                 r2 = StepRunner(H, I, w2, dev, weights=runner.st["weights"])
                 m2, _, _ = time_steps(r2, max(5, args.steps // 2), 3, 1)
                 lens2 = r2.st["ctx_lens"].cpu()
@@ -424,7 +424,9 @@ def run_ours(args, rank, world, local):
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
                 "data": "synthetic (seeded random-init weights and KV of the stated shapes)",
                 "config": {"workload": f"full draft step {wl.name}: 4-layer M,A,M,A hybrid drafter, Llama-3-8B "
-                                       f"shapes, SwiGLU 16384, vocab 128256, ctx U[512,16384], 16-token pages",
+                                       f"shapes, SwiGLU 16384, vocab 128256"
+                                       + (f" (draft head {wl.shapes.draft_vocab} rows)" if wl.shapes.draft_vocab else "")
+                                       + ", ctx U[512,16384], 16-token pages",
                            "C": wl.C, "K": wl.K, "global_batch": wl.C * world, "parallelism": f"replicas x{world}",
                            "l2": "inputs ~20 GB > 126 MB L2 (no flush needed)"},
                 "roofline": roof, "attention_roofline": attn_roof, "kernels": kernels,
@@ -515,7 +517,7 @@ def run_reference(args, rank, world):
     if rank != 0:
         return
     from hybrid_mamba_attention_b200 import inputs as I
-    wl = I.full_workload(args.C, args.K)
+    wl = I.full_workload(args.C, args.K, args.draft_vocab)
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     st = I.make_step_inputs(wl, dev)
 
@@ -553,6 +555,8 @@ def main():
     ap.add_argument("--impl", choices=["hspec", "reference"], default="hspec")
     ap.add_argument("--C", type=int, default=128)
     ap.add_argument("--K", type=int, default=16)
+    ap.add_argument("--draft-vocab", type=int, default=0,
+                    help="reduced draft head rows (0 = the full 128256-token head)")
     ap.add_argument("--sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel", choices=["step", "attn", "inject", "ssd"], default="step",

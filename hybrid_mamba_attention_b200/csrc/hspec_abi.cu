@@ -274,7 +274,8 @@ StepPlan step_plan(const hspec_cfg* c, int C, int K, int max_pages) {
     s.ap = attn_plan(c, C, K, max_pages);
     off += s.ap.ws;
   }
-  s.n_parts = c->vocab > 0 ? cdiv(c->vocab, argmax_tile_n(c->dtype)) : 0;
+  const int head_rows = c->draft_vocab > 0 ? c->draft_vocab : c->vocab;
+  s.n_parts = c->vocab > 0 ? cdiv(head_rows, argmax_tile_n(c->dtype)) : 0;
   s.pval = off, off += align256(M * s.n_parts * 4);
   s.pidx = off, off += align256(M * s.n_parts * 4);
   // split-K workspace: the largest need of the step's projection and MLP GEMMs
@@ -528,6 +529,8 @@ hspec_status hspec_drafter_create(const hspec_cfg* cfg, const hspec_model_weight
   hspec_status st = validate_cfg(cfg, has_kind(cfg, 'A'), has_kind(cfg, 'M'));
   if (st) return st;
   if (cfg->d_ff < 0 || cfg->vocab < 0) FAIL(HSPEC_ERR_INVALID_ARG, "d_ff and vocab must be >= 0");
+  if (cfg->draft_vocab < 0 || (cfg->draft_vocab > 0 && cfg->vocab == 0))
+    FAIL(HSPEC_ERR_INVALID_ARG, "draft_vocab must be >= 0, and needs a vocab (the embedding table)");
   if (cfg->dtype == HSPEC_DTYPE_BF16) {
     // tensor-core GEMM operands are streamed by TMA: every GEMM reduction dimension
     // (= operand row stride) must be a multiple of 8 elements (16 bytes)
@@ -550,6 +553,8 @@ hspec_status hspec_drafter_create(const hspec_cfg* cfg, const hspec_model_weight
       FAIL(HSPEC_ERR_INVALID_ARG, "layer %d: an MLP weight is NULL", i);
   }
   if (cfg->vocab > 0 && (!w->final_norm || !w->W_lm)) FAIL(HSPEC_ERR_INVALID_ARG, "final_norm / W_lm is NULL");
+  if (cfg->draft_vocab > 0 && (!w->W_lm_draft || !w->draft_to_target))
+    FAIL(HSPEC_ERR_INVALID_ARG, "W_lm_draft / draft_to_target is NULL (draft_vocab > 0)");
   hspec_drafter* d = new hspec_drafter;
   d->cfg = *cfg;
   d->w = *w;
@@ -744,7 +749,9 @@ hspec_status hspec_draft_step(hspec_drafter* dr, const hspec_step_in* in, const 
       rmsnorm_rows(dtype, x, W.final_norm, xn, M, d, eps, s);
     }
     if (out->final_normed) cudaMemcpyAsync(out->final_normed, xn, (size_t)M * d * E, cudaMemcpyDeviceToDevice, s);
-    GemmArgs ga = gemm_args(M, c->vocab, d, xn, d, W.W_lm, d, nullptr, 0);
+    const bool reduced = c->draft_vocab > 0;
+    GemmArgs ga = gemm_args(M, reduced ? c->draft_vocab : c->vocab, d, xn, d, reduced ? W.W_lm_draft : W.W_lm, d,
+                            nullptr, 0);
     ga.pval = (float*)(ws + sp.pval);
     ga.pidx = (int32_t*)(ws + sp.pidx);
     ga.n_parts = sp.n_parts;
@@ -754,7 +761,8 @@ hspec_status hspec_draft_step(hspec_drafter* dr, const hspec_step_in* in, const 
     }
     {
       ProfScope p("argmax_reduce", s);
-      argmax_reduce(ga.pval, ga.pidx, M, sp.n_parts, out->draft_tokens, out->top_logit, s);
+      argmax_reduce(ga.pval, ga.pidx, M, sp.n_parts, out->draft_tokens, out->top_logit,
+                    reduced ? W.draft_to_target : nullptr, c->vocab, err, s);
     }
   }
   if (out->hidden) cudaMemcpyAsync(out->hidden, x, (size_t)M * d * 4, cudaMemcpyDeviceToDevice, s);

@@ -25,8 +25,10 @@ void gated_rmsnorm_rows(int dtype, const float* y, const void* z, long z_stride,
 void rope_rows(int dtype, void* qkv, long row_stride, const int32_t* ctx_lens, int C, int K,
                int n_heads, int D, float theta, cudaStream_t s);
 // tokens[m] = argmax over parts of (pval, pidx)[m][:] (lowest id on ties); top[m] = its value.
+// Per row the max over the partials (lowest id on ties); with `map` (reduced draft
+// head) the token is map[id], checked against [0, vocab) (else -1 and kErrTokenOOB).
 void argmax_reduce(const float* pval, const int32_t* pidx, int M, int n_parts, int32_t* tokens,
-                   float* top, cudaStream_t s);
+                   float* top, const int32_t* map, int vocab, int* err, cudaStream_t s);
 
 // ------------------------------------------------------------ gemm_simt.cu / gemm_tc.cu
 enum GemmEpi : int {

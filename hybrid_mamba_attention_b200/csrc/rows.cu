@@ -221,7 +221,8 @@ __global__ void rope_kernel(T* __restrict__ qkv, long row_stride, const int32_t*
 // the first (lowest id) of equal maxima.
 __global__ void argmax_reduce_kernel(const float* __restrict__ pval, const int32_t* __restrict__ pidx,
                                      int M, int n_parts, int32_t* __restrict__ tokens,
-                                     float* __restrict__ top) {
+                                     float* __restrict__ top, const int32_t* __restrict__ map, int vocab,
+                                     int* err) {
   pdl_wait();  // the previous kernel on the stream is complete from here on
   pdl_trigger();
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
@@ -240,7 +241,15 @@ __global__ void argmax_reduce_kernel(const float* __restrict__ pval, const int32
     if (v > best || (v == best && id < bidx)) best = v, bidx = id;
   }
   if (lane == 0) {
-    tokens[warp] = bidx;
+    int tok = bidx;
+    if (map) {  // reduced draft head: row -> target token id
+      tok = map[bidx];
+      if (tok < 0 || tok >= vocab) {
+        flag_error(err, kErrTokenOOB);
+        tok = -1;
+      }
+    }
+    tokens[warp] = tok;
     if (top) top[warp] = best;
   }
 }
@@ -319,9 +328,9 @@ void rope_rows(int dtype, void* qkv, long row_stride, const int32_t* ctx_lens, i
 }
 
 void argmax_reduce(const float* pval, const int32_t* pidx, int M, int n_parts, int32_t* tokens,
-                   float* top, cudaStream_t s) {
+                   float* top, const int32_t* map, int vocab, int* err, cudaStream_t s) {
   const int warps_per_block = 8;
-  launch_pdl(argmax_reduce_kernel, (M + warps_per_block - 1) / warps_per_block, 32 * warps_per_block, 0, s, pval, pidx, M, n_parts, tokens, top);
+  launch_pdl(argmax_reduce_kernel, (M + warps_per_block - 1) / warps_per_block, 32 * warps_per_block, 0, s, pval, pidx, M, n_parts, tokens, top, map, vocab, err);
   note_launch();
 }
 

@@ -55,7 +55,8 @@ class hspec_cfg(ct.Structure):
                 ("d_state", ct.c_int), ("page_size", ct.c_int), ("d_ff", ct.c_int), ("vocab", ct.c_int),
                 ("n_layers", ct.c_int), ("layer_kinds", ct.c_char * HSPEC_MAX_LAYERS),
                 ("dtype", ct.c_int), ("flags", ct.c_int), ("rope_theta", ct.c_float),
-                ("norm_eps", ct.c_float), ("ssd_chunk", ct.c_int), ("attn_split_tokens", ct.c_int)]
+                ("norm_eps", ct.c_float), ("ssd_chunk", ct.c_int), ("attn_split_tokens", ct.c_int),
+                ("draft_vocab", ct.c_int)]
 
 
 class hspec_layer_weights(ct.Structure):
@@ -65,7 +66,7 @@ class hspec_layer_weights(ct.Structure):
 
 class hspec_model_weights(ct.Structure):
     _fields_ = [("layers", hspec_layer_weights * HSPEC_MAX_LAYERS), ("final_norm", ct.c_void_p),
-                ("W_lm", ct.c_void_p)]
+                ("W_lm", ct.c_void_p), ("W_lm_draft", ct.c_void_p), ("draft_to_target", ct.c_void_p)]
 
 
 class hspec_kv_view(ct.Structure):
@@ -154,7 +155,7 @@ def make_cfg(shapes, ssd_chunk: int = 0, attn_split_tokens: int = 0, fuse_inject
                      n_layers=len(sh.layers), layer_kinds=sh.layers.encode(),
                      dtype=HSPEC_DTYPE_F32 if sh.dtype == "f32" else HSPEC_DTYPE_BF16, flags=flags,
                      rope_theta=sh.rope_theta, norm_eps=sh.eps, ssd_chunk=ssd_chunk,
-                     attn_split_tokens=attn_split_tokens)
+                     attn_split_tokens=attn_split_tokens, draft_vocab=getattr(sh, "draft_vocab", 0))
 
 
 def kv_view(cache: dict) -> hspec_kv_view:
@@ -282,6 +283,9 @@ class Drafter:
         if "final_norm" in weights:
             mw.final_norm = _ptr(weights["final_norm"])
             mw.W_lm = _ptr(weights["W_lm"])
+        if "W_lm_draft" in weights:
+            mw.W_lm_draft = _ptr(weights["W_lm_draft"])
+            mw.draft_to_target = _ptr(weights["draft_to_target"])
         self._mw = mw
         self.handle = hspec_drafter_create(self.cfg, mw)
 

@@ -94,6 +94,8 @@ typedef struct hspec_cfg {
                                        fp32, tokens per split of a request; bf16, tiles per chunk of
                                        the even tile-space partition (rounded up to 64 tokens; at
                                        most 2048 chunks) -- auto: one chunk per SM */
+  int draft_vocab;                  /* reduced draft head rows (0 = the full vocab head):    */
+                                    /* logits over W_lm_draft, draft token = the mapped id  */
 } hspec_cfg;
 
 /* Weights of one layer (caller-owned device memory; fields of the other layer kind
@@ -119,6 +121,12 @@ typedef struct hspec_model_weights {
   hspec_layer_weights layers[HSPEC_MAX_LAYERS];
   const float* final_norm; /* [d]                                                        */
   const void* W_lm;        /* [vocab, d] shared LM head, also the token embedding table  */
+  /* reduced-vocabulary draft head (cfg.draft_vocab > 0; H-Spec's evolve.pub review,
+   * Frequently asked questions: the drafter's vocabulary may be cut to frequent tokens):
+   * row r of W_lm_draft stands for target token draft_to_target[r] (0 <= id < vocab, a
+   * bad id sets the device error word and the token is written as -1) */
+  const void* W_lm_draft;          /* [draft_vocab, d]                                   */
+  const int32_t* draft_to_target;  /* [draft_vocab]                                      */
 } hspec_model_weights;
 
 /* The target's paged KV cache, read in place (never written, never copied). */
@@ -246,8 +254,9 @@ HSPEC_API size_t hspec_step_workspace_size(const hspec_cfg* cfg, int C, int K, i
  *   M: x += W_out gnorm(SSD(in_proj(norm(x)); h0 = W_inj h_last) * silu(z))
  *   A: x += W_o attn(rope(q), target KV in place ++ rope(k_blk), v_blk)
  *   MLP (d_ff > 0): x += W_down (silu(W_gate norm(x)) * W_up norm(x))
- * then draft_tokens = argmax(W_lm final_norm(x)).  max_pages of every kv view must be
- * <= the max_pages given to hspec_step_workspace_size. */
+ * then draft_tokens = argmax(W_lm final_norm(x)) (with draft_vocab > 0:
+ * draft_to_target[argmax(W_lm_draft final_norm(x))]).  max_pages of every kv view must
+ * be <= the max_pages given to hspec_step_workspace_size. */
 HSPEC_API hspec_status hspec_draft_step(hspec_drafter* drafter, const hspec_step_in* in,
                               const hspec_step_out* out, void* workspace, size_t ws_bytes,
                               void* stream);

@@ -34,10 +34,10 @@ def test_library_exports_every_declared_function(H):
 
 def test_struct_layouts_match_header(H, tmp_path):
     prog = tmp_path / "sz.c"
-    fields = {"hspec_cfg": ["d_model", "layer_kinds", "dtype", "rope_theta", "attn_split_tokens"],
+    fields = {"hspec_cfg": ["d_model", "layer_kinds", "dtype", "rope_theta", "attn_split_tokens", "draft_vocab"],
               "hspec_step_in": ["C", "h_last", "ctx_lens", "kv"],
               "hspec_kv_view": ["v_pool", "num_pages", "page_table", "max_pages"],
-              "hspec_model_weights": ["layers", "final_norm", "W_lm"],
+              "hspec_model_weights": ["layers", "final_norm", "W_lm", "W_lm_draft", "draft_to_target"],
               "hspec_layer_weights": ["W_inj", "W_down"],
               "hspec_step_out": ["draft_tokens", "top_logit"]}
     lines = ['#include <stdio.h>', '#include <stddef.h>', f'#include "{HEADER}"', "int main(void){"]

@@ -94,7 +94,11 @@ def check_stagewise(wl, st, out, rows, wh):
         else:
             assert_close(to_np(out["final_normed"][rows]), fn_ref, sh.dtype, f"{wl.name} final norm")
         fn = out["final_normed"][rows]
-        am, t1, t2 = oracle.lm_head_argmax(host(fn).reshape(-1, sh.d), wh["W_lm"])
+        if sh.draft_vocab:  # reduced draft head: argmax over its rows, then the id map
+            am, t1, t2 = oracle.lm_head_argmax(host(fn).reshape(-1, sh.d), wh["W_lm_draft"])
+            am = wh["draft_to_target"].numpy()[am]
+        else:
+            am, t1, t2 = oracle.lm_head_argmax(host(fn).reshape(-1, sh.d), wh["W_lm"])
         gpu_tok = host(out["tokens"][rows]).reshape(-1).numpy()
         decided = (t1 - t2) >= GAP
         assert decided.mean() > 0.5
@@ -222,3 +226,18 @@ def test_fused_injection_readout_equals_stored_h0(H, cuda, C, K):
             assert e <= BF16_TOL
     e = rel_rms(to_np(a["hidden"]), to_np(b["hidden"]))
     assert np.isfinite(to_np(a["hidden"])).all() and e <= DRIFT_BOUND, e
+
+
+@pytest.mark.parametrize("C,K", [(1, 16), (8, 16), (128, 16)])
+def test_reduced_vocab_draft_head(H, cuda, C, K):
+    # 32768-row draft head over the same drafter: stage-wise parity, the draft tokens
+    # mapped to target ids (evolve.pub review of H-Spec, Frequently asked questions)
+    wl = I.full_workload(C, K, draft_vocab=32768)
+    st = I.make_step_inputs(wl, cuda)
+    out = run_step(H, wl, st)
+    assert H.hspec_sync_status() == 0, H.hspec_last_error()
+    rows = sample_requests(wl.C, 2, seed=wl.seed)
+    wh = host_weights(st["weights"])
+    check_stagewise(wl, st, out, rows, wh)
+    ids = set(wh["draft_to_target"].tolist())
+    assert set(host(out["tokens"]).reshape(-1).tolist()) <= ids
