@@ -170,6 +170,22 @@ def lm_head_argmax(hn, W_lm):
     return am, t1, t2
 
 
+def verify_greedy(logits, drafts, ctx_lens=None):
+    """logits [C, K+1, V] (fp32 or bf16), drafts [C, K] int32 -> (accepted [C], next_token
+    [C], new ctx_lens [C] or None).  See oracle_verify_greedy."""
+    lg, lt = _cpu(logits)
+    dr = _i32(drafts)
+    C, K1, V = lg.shape
+    K = K1 - 1
+    assert tuple(dr.shape) == (C, K)
+    acc = np.zeros(C, dtype=np.int32)
+    nxt = np.zeros(C, dtype=np.int32)
+    ctx = None if ctx_lens is None else _i32(ctx_lens).numpy().copy()
+    lib().oracle_verify_greedy(C, K, V, _ptr(lg), lt, _ptr(dr), _dptr(acc), _dptr(nxt),
+                               _dptr(ctx) if ctx is not None else None)
+    return acc, nxt, ctx
+
+
 # ------------------------------------------------------------ host copies
 
 def host_weights(w: dict) -> dict:

@@ -274,6 +274,31 @@ void oracle_lm_head_argmax(int rows, int d, int V, const void* hn, int hn_type, 
   lm_head_argmax(rows, d, V, a.data(), W_lm, w_type, argmax, top1, top2);
 }
 
+// Greedy verification: the target's argmax per row, the longest prefix of drafts that
+// matches it, and the target's token after that prefix.
+void oracle_verify_greedy(int C, int K, int V, const void* logits, int ltype, const int32_t* drafts,
+                          int32_t* accepted, int32_t* next_token, int32_t* ctx_lens) {
+  for (int c = 0; c < C; ++c) {
+    std::vector<int32_t> t(K + 1);
+    for (int j = 0; j <= K; ++j) {
+      const size_t base = ((size_t)c * (K + 1) + j) * V;
+      int32_t best = -1;
+      double bv = 0.0;
+      for (int v = 0; v < V; ++v) {
+        const double x = load(logits, ltype, base + v);
+        if (std::isnan(x)) continue;
+        if (best < 0 || x > bv) best = v, bv = x;
+      }
+      t[j] = best;
+    }
+    int a = 0;
+    while (a < K && drafts[(size_t)c * K + a] == t[a]) ++a;
+    accepted[c] = a;
+    next_token[c] = t[a];
+    if (ctx_lens) ctx_lens[c] += a + 1;
+  }
+}
+
 // One draft step.  Per layer (pre-norm residual blocks):
 //   M: xn = R(rmsnorm(x) w); [z, xs, B, C, dt_raw] = R(xn W_in^T); dt = softplus(dt_raw + dt_bias);
 //      h0 = W_inj h_last (reshaped [H,P,N]); y = SSD recurrence from h0;

@@ -80,6 +80,17 @@ void oracle_bf16_round_array(long n, const double* in, double* out);
 void oracle_lm_head_argmax(int rows, int d, int V, const void* hn, int hn_type, const void* W_lm,
                            int w_type, int32_t* argmax, double* top1, double* top2);
 
+/* Greedy verification of K drafts per request (standard speculative decoding, which
+ * H-Spec follows -- evolve.pub review of H-Spec, Frequently asked questions).  logits
+ * [C, K+1, V] (type ltype) are the target's, row j predicting block position j;
+ * drafts [C, K].  Per request: t_j = argmax_v logits[c][j][v] (lowest id on ties, NaN
+ * never wins; -1 if the row has no number), accepted a = number of leading j < K with
+ * drafts[c][j] == t_j, next_token = t_a, and ctx_lens[c] += a + 1 when ctx_lens is not
+ * NULL (the accepted drafts and the target's token enter the context; the K - a
+ * rejected positions roll back). */
+void oracle_verify_greedy(int C, int K, int V, const void* logits, int ltype, const int32_t* drafts,
+                          int32_t* accepted, int32_t* next_token, int32_t* ctx_lens);
+
 typedef struct {
   int d, Hq, Hkv, D, H, P, N, page, d_ff, vocab, n_layers;
   char kinds[16];       /* 'M' or 'A' per layer */
