@@ -17,6 +17,7 @@ time is the max over ranks.
 from __future__ import annotations
 
 import argparse
+from dataclasses import replace
 import json
 import re
 import math
@@ -462,6 +463,19 @@ def run_kernel(args, rank, world, local):
         work = {"bytes": float(ctx * sh.Hkv * sh.D * 2 * E + 2 * C * K * sh.Hq * sh.D * E),
                 "flops": 4.0 * sh.Hq * sh.D * K * (ctx + C * K)}
         name = "attn_paged"
+    elif args.kernel == "verify":
+        # the target's logits for the K + 1 block positions of every request (synthetic)
+        V = sh.vocab or 128256
+        g = torch.Generator(device=dev).manual_seed(wl.seed)
+        logits = torch.randn(C, K + 1, V, generator=g, device=dev).to(sh.torch_dtype)
+        drafts = torch.randint(0, V, (C, K), generator=g, device=dev, dtype=torch.int32)
+        vcfg = H.make_cfg(replace(sh, vocab=V))
+        ws = H.alloc_workspace(H.hspec_verify_workspace_size(vcfg, C, K), dev)
+        acc = torch.empty(C, dtype=torch.int32, device=dev)
+        nxt = torch.empty(C, dtype=torch.int32, device=dev)
+        call = lambda: H.hspec_verify_greedy(vcfg, logits, drafts, acc, nxt, ws)
+        work = {"bytes": float(C * (K + 1) * V * E), "flops": 0.0}
+        name = "verify_greedy"
     elif args.kernel == "inject":
         inp = I.make_inject_inputs(sh, C, wl.seed, dev)
         HPN = sh.H * sh.P * sh.N
@@ -559,7 +573,7 @@ def main():
                     help="reduced draft head rows (0 = the full 128256-token head)")
     ap.add_argument("--sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel", choices=["step", "attn", "inject", "ssd"], default="step",
+    ap.add_argument("--kernel", choices=["step", "attn", "inject", "ssd", "verify"], default="step",
                     help="time one C-ABI call on --workload instead of the full draft step")
     ap.add_argument("--workload", default="llama_c32", help="kernel-level workload (tiny, llama_c1, llama_c32, qwen_c128, or full_C<C>_K<K>: one layer of the full step)")
     args = ap.parse_args()

@@ -517,6 +517,30 @@ hspec_status hspec_attn_paged_block(const hspec_cfg* cfg, const void* q, const h
   return check_launch("hspec_attn_paged_block");
 }
 
+size_t hspec_verify_workspace_size(const hspec_cfg* cfg, int C, int K) {
+  if (!cfg || cfg->vocab < 1 || C < 1 || K < 1 || K > 64) return 0;
+  return align256(verify_ws_bytes(cfg->dtype, C, K, cfg->vocab));
+}
+
+hspec_status hspec_verify_greedy(const hspec_cfg* cfg, const void* logits, const int32_t* drafts, int C, int K,
+                                 int32_t* accepted, int32_t* next_token, int32_t* ctx_lens, void* workspace,
+                                 size_t ws_bytes, void* stream) {
+  if (!cfg) FAIL(HSPEC_ERR_INVALID_ARG, "cfg is NULL");
+  if (cfg->dtype != HSPEC_DTYPE_F32 && cfg->dtype != HSPEC_DTYPE_BF16)
+    FAIL(HSPEC_ERR_INVALID_ARG, "dtype %d is neither HSPEC_DTYPE_F32 nor HSPEC_DTYPE_BF16", cfg->dtype);
+  if (cfg->vocab < 1) FAIL(HSPEC_ERR_INVALID_ARG, "verification needs cfg->vocab >= 1");
+  if (!logits || !drafts || !accepted || !next_token)
+    FAIL(HSPEC_ERR_INVALID_ARG, "logits, drafts, accepted and next_token must be non-NULL");
+  if (C < 1 || K < 1 || K > 64) FAIL(HSPEC_ERR_UNSUPPORTED, "C=%d K=%d (need C >= 1, 1 <= K <= 64)", C, K);
+  if ((long)C * (K + 1) > 0x7fffffffL || cfg->vocab > 65535L * 16384) FAIL(HSPEC_ERR_UNSUPPORTED, "too many rows or logits");
+  const size_t need = hspec_verify_workspace_size(cfg, C, K);
+  if (!workspace || ((uintptr_t)workspace & 255) || ws_bytes < need)
+    FAIL(HSPEC_ERR_WORKSPACE, "verification needs a 256-byte aligned workspace of %zu bytes (got %zu)", need, ws_bytes);
+  verify_greedy(cfg->dtype, logits, cfg->vocab, drafts, C, K, accepted, next_token, ctx_lens, workspace,
+                (cudaStream_t)stream);
+  return check_launch("hspec_verify_greedy");
+}
+
 hspec_status hspec_drafter_create(const hspec_cfg* cfg, const hspec_model_weights* w, hspec_drafter** out) {
   if (!out || !w) FAIL(HSPEC_ERR_INVALID_ARG, "weights and out must be non-NULL");
   *out = nullptr;

@@ -142,4 +142,10 @@ bool attn_tc_launch(const AttnArgs& a, cudaStream_t s);
 // Split kernel + merge; false (message recorded) if it cannot launch.
 bool attn_paged(int dtype, const AttnArgs& a, cudaStream_t s);
 
+// ------------------------------------------------------------ verify.cu
+// Greedy verification (see verify.cu); workspace of verify_ws_bytes(dtype, C, K, V) bytes.
+size_t verify_ws_bytes(int dtype, int C, int K, int V);
+void verify_greedy(int dtype, const void* logits, int V, const int32_t* drafts, int C, int K,
+                   int32_t* accepted, int32_t* next_token, int32_t* ctx_lens, void* ws, cudaStream_t s);
+
 }  // namespace hspec

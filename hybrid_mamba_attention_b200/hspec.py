@@ -36,7 +36,8 @@ EXPORTS = ("hspec_inject_state", "hspec_ssd_block_scan", "hspec_attn_workspace_s
            "hspec_attn_paged_block", "hspec_drafter_create", "hspec_drafter_destroy",
            "hspec_step_workspace_size", "hspec_draft_step", "hspec_sync_status",
            "hspec_status_string", "hspec_last_error", "hspec_launch_count", "hspec_version",
-           "hspec_profile_enable", "hspec_profile_read", "hspec_attn_paged_block_noalloc")
+           "hspec_profile_enable", "hspec_profile_read", "hspec_attn_paged_block_noalloc",
+           "hspec_verify_workspace_size", "hspec_verify_greedy")
 HSPEC_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
@@ -109,6 +110,8 @@ def _load():
         "hspec_profile_enable": (I, [I]),
         "hspec_profile_read": (I, [P, P, P, I]),
         "hspec_attn_paged_block_noalloc": (I, [cfgp, P, ct.POINTER(hspec_kv_view), P, P, P, I, I, P, V]),
+        "hspec_verify_workspace_size": (Z, [cfgp, I, I]),
+        "hspec_verify_greedy": (I, [cfgp, P, P, I, I, P, P, P, P, Z, V]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -195,6 +198,23 @@ def hspec_attn_paged_block(cfg: hspec_cfg, q, kv: hspec_kv_view, ctx_lens, k_blk
                                        _ptr(v_blk), C, K, _ptr(out), _ptr(workspace),
                                        workspace.numel() * workspace.element_size(), _stream(stream)),
            "hspec_attn_paged_block")
+
+
+def hspec_verify_workspace_size(cfg: hspec_cfg, C: int, K: int) -> int:
+    return int(_lib.hspec_verify_workspace_size(ct.byref(cfg), C, K))
+
+
+def hspec_verify_greedy(cfg: hspec_cfg, logits, drafts, accepted, next_token, workspace, ctx_lens=None,
+                        stream=None):
+    """Greedy verification: logits [C, K+1, cfg.vocab] (cfg dtype), drafts [C, K] int32;
+    writes accepted [C] and next_token [C] (int32) and advances ctx_lens [C] in place when
+    given."""
+    C, K = int(drafts.shape[0]), int(drafts.shape[1])
+    _check(_lib.hspec_verify_greedy(ct.byref(cfg), _ptr(logits), _ptr(drafts), C, K, _ptr(accepted),
+                                    _ptr(next_token), _ptr(ctx_lens) if ctx_lens is not None else None,
+                                    _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                    _stream(stream)),
+           "hspec_verify_greedy")
 
 
 def hspec_attn_paged_block_noalloc(cfg: hspec_cfg, q, kv: hspec_kv_view, ctx_lens, k_blk, v_blk, out,

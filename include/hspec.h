@@ -249,6 +249,25 @@ typedef struct hspec_step_out {
  * split-KV partials, argmax partials). */
 HSPEC_API size_t hspec_step_workspace_size(const hspec_cfg* cfg, int C, int K, int max_pages);
 
+/* Workspace bytes of hspec_verify_greedy for C requests of K drafts over cfg->vocab. */
+HSPEC_API size_t hspec_verify_workspace_size(const hspec_cfg* cfg, int C, int K);
+
+/* Greedy verification of the drafts against the target's logits (standard
+ * speculative-decoding verification, kept by H-Spec -- evolve.pub review, Frequently
+ * asked questions).  Row j of request c is the target's prediction for block position j:
+ *   t_j = argmax_v logits[c][j][v]   (lowest id on ties; NaN never wins; -1 if none)
+ *   accepted[c] = longest prefix j < K with drafts[c][j] == t_j
+ *   next_token[c] = t_accepted;  ctx_lens[c] += accepted[c] + 1 when ctx_lens != NULL
+ * (the accepted drafts and the target's token enter the context; the rejected
+ * positions roll back -- their KV slots lie past the new length).
+ * logits device [C, K+1, cfg->vocab] (cfg->dtype); drafts device [C, K] int32;
+ * accepted, next_token device [C] int32, written; ctx_lens device [C] int32 or NULL;
+ * workspace device, >= hspec_verify_workspace_size() bytes, 256-byte aligned.
+ * C >= 1, 1 <= K <= 64, cfg->vocab >= 1. */
+HSPEC_API hspec_status hspec_verify_greedy(const hspec_cfg* cfg, const void* logits, const int32_t* drafts, int C,
+                                           int K, int32_t* accepted, int32_t* next_token, int32_t* ctx_lens,
+                                           void* workspace, size_t ws_bytes, void* stream);
+
 /* One block-parallel draft step (all layers, then the LM-head argmax when vocab > 0):
  * per layer, pre-norm residual blocks
  *   M: x += W_out gnorm(SSD(in_proj(norm(x)); h0 = W_inj h_last) * silu(z))
