@@ -463,6 +463,18 @@ def run_kernel(args, rank, world, local):
         work = {"bytes": float(ctx * sh.Hkv * sh.D * 2 * E + 2 * C * K * sh.Hq * sh.D * E),
                 "flops": 4.0 * sh.Hq * sh.D * K * (ctx + C * K)}
         name = "attn_paged"
+    elif args.kernel == "gemm":
+        # the tcgen05 GEMM alone in its tensor-bound regime: the injection GEMM of an
+        # eighth of the heads (N = H/8 * P * N_state) for all C*K block rows (M = 2048 at
+        # C=128, K=16), K = d; about 1.1 GB on the device
+        sh8 = replace(sh, H=max(1, sh.H // 8))
+        HPN, Mr = sh8.H * sh8.P * sh8.N, C * K
+        inp = I.make_inject_inputs(sh8, Mr, wl.seed, dev)
+        h0 = torch.empty(Mr, HPN, device=dev)
+        gcfg = H.make_cfg(sh8)
+        call = lambda: H.hspec_inject_state(gcfg, inp["W_inj"], inp["h_last"], h0)
+        work = {"bytes": float(HPN * sh.d * E + Mr * HPN * 4 + Mr * sh.d * E), "flops": 2.0 * Mr * HPN * sh.d}
+        name = "gemm_tc"
     elif args.kernel == "verify":
         # the target's logits for the K + 1 block positions of every request (synthetic)
         V = sh.vocab or 128256
@@ -573,7 +585,7 @@ def main():
                     help="reduced draft head rows (0 = the full 128256-token head)")
     ap.add_argument("--sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel", choices=["step", "attn", "inject", "ssd", "verify"], default="step",
+    ap.add_argument("--kernel", choices=["step", "attn", "inject", "ssd", "verify", "gemm"], default="step",
                     help="time one C-ABI call on --workload instead of the full draft step")
     ap.add_argument("--workload", default="llama_c32", help="kernel-level workload (tiny, llama_c1, llama_c32, qwen_c128, or full_C<C>_K<K>: one layer of the full step)")
     args = ap.parse_args()
