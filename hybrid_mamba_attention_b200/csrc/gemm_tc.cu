@@ -28,8 +28,13 @@
 //   split-K (fewer tiles than half the SMs): unit (tile, split) covers an equal K
 //     range, all units start at their range's first block together; slot = unit.
 // A segment covering a whole tile runs the fused epilogue itself; the others write the
-// fp32 partial of their rows to their slot, and the last segment of a tile to finish
-// (an atomic counter per tile) sums the partials in K order and runs the epilogue.
+// fp32 partial of their rows to their slot and count in (an atomic counter per tile).
+// Split-K: the last segment of a tile to finish sums the partials in K order and runs
+// the epilogue.  Stream-K: after its own segments every CTA takes an equal share of the
+// split tiles' (row, 32-column) sums, each waiting until its tile is complete -- with
+// many rows one CTA summing a tile's ~10 partials at one SM's bandwidth was the limit.
+// The counters are not reset (each call site of the draft step has its own, zeroed
+// once per step).
 #include <mutex>
 #include <stdint.h>
 
@@ -131,6 +136,25 @@ struct SegWalk {
     return true;
   }
 };
+
+// Waits (bounded) until *cnt >= target; the acquire load orders the reads that follow.
+__device__ __forceinline__ bool wait_count(const int* cnt, int target, int* err) {
+  auto ld = [&]() {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(cnt) : "memory");
+    return v;
+  };
+  if (ld() >= target) return true;
+  const uint64_t t0 = tc::global_ns();
+  while (ld() < target) {
+    __nanosleep(256);
+    if (tc::global_ns() - t0 > tc::kWaitLimitNs) {
+      flag_error(err, tc::kErrTimeout);
+      return false;
+    }
+  }
+  return true;
+}
 
 // Partial slot of tile t's segment in chunk k (stream-K): the chunk's first segment if
 // the chunk starts inside the tile, else its last.
@@ -271,9 +295,17 @@ __global__ void __launch_bounds__(THREADS, 1)
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&acc_empty[b]);
         __threadfence();
-        // the four epilogue warps pass the same three barriers per unit and leave together
+        // the four epilogue warps pass the same barriers per unit and leave together
         if (!ok) *s_fail = 1;
         asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (zk) {
+          // stream-K: count the segment in; every CTA sums split tiles after its own work
+          if (threadIdx.x == 64) atomicAdd(&g.tile_cnt[t], 1);
+          const bool all_ok = *s_fail == 0;
+          asm volatile("bar.sync 1, 128;" ::: "memory");
+          if (!all_ok) break;
+          continue;
+        }
         if (threadIdx.x == 64) *s_last = atomicAdd(&g.tile_cnt[t], 1) == n_seg - 1;
         asm volatile("bar.sync 1, 128;" ::: "memory");
         const bool last = *s_last != 0, all_ok = *s_fail == 0;
@@ -418,6 +450,43 @@ __global__ void __launch_bounds__(THREADS, 1)
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&acc_empty[b]);
       if (!ok) break;
+    }
+    if (cut.zk && *s_fail == 0) {
+      // stream-K (one row of tiles): the sums of the split tiles, spread over the epilogue
+      // threads of all CTAs as (tile, row, 32-column chunk) items, rows fastest.  An item
+      // waits (bounded) until all segments of its tile are counted in, then adds their
+      // partials in K order -- the same sums whichever CTA takes it.  Every CTA reaches
+      // this phase only after its own segments, so no wait depends on a waiting CTA.
+      const int zk = cut.zk, rows_v = min(BM, g.M), nch = ncols_out / 32;
+      const long per_tile = (long)rows_v * nch, n_items = (long)n_tiles * per_tile;
+      float v[32], u2[32];
+      int waited = -1;
+      for (long it = (long)blockIdx.x * 128 + (threadIdx.x - 64); it < n_items; it += (long)gridDim.x * 128) {
+        const int t = (int)(it / per_tile), rem = (int)(it - (long)t * per_tile);
+        const int r = rem % rows_v, cc = rem / rows_v;
+        const int kf = (int)((long)t * num_k / zk), n_seg = (int)(((long)t * num_k + num_k - 1) / zk) - kf + 1;
+        if (n_seg == 1) continue;
+        if (t != waited) {
+          if (!wait_count(&g.tile_cnt[t], n_seg, err)) break;
+          waited = t;
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = 0.f, u2[i] = 0.f;
+#pragma unroll 2
+        for (int q = 0; q < n_seg; ++q) {
+          const float4* pq = (const float4*)(g.part + (size_t)seg_slot(t, kf + q, zk, num_k) * BM * BN) + r;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float4 a4 = __ldcg(pq + (cc * 8 + i) * BM);
+            v[4 * i] += a4.x, v[4 * i + 1] += a4.y, v[4 * i + 2] += a4.z, v[4 * i + 3] += a4.w;
+            if (EPI == kEpiSwiGLU) {
+              const float4 b4 = __ldcg(pq + ((cc + BN / 64) * 8 + i) * BM);
+              u2[4 * i] += b4.x, u2[4 * i + 1] += b4.y, u2[4 * i + 2] += b4.z, u2[4 * i + 3] += b4.w;
+            }
+          }
+        }
+        epi32<EPI>(g, r, t * ncols_out + cc * 32, v, u2);
+      }
     }
   }
   __syncthreads();

@@ -247,7 +247,8 @@ struct StepPlan {
   AttnPlan ap;
   int n_parts;
   size_t gpart_bytes;  // partials of the projection / MLP GEMMs with a cut K loop
-  int gmax_tiles;      // tile counters that follow them
+  int gmax_tiles;      // tile counters that follow them (per call site)
+  int gcnt_sites;      // call sites with their own counter slice
 };
 
 StepPlan step_plan(const hspec_cfg* c, int C, int K, int max_pages) {
@@ -296,7 +297,10 @@ StepPlan step_plan(const hspec_cfg* c, int C, int K, int max_pages) {
     }
   }
   s.gpart = off, off += align256(s.gpart_bytes);
-  s.gcnt = off, off += align256((size_t)s.gmax_tiles * 4);
+  // one slice of tile counters per K-cut GEMM call of the step (at most 4 per layer),
+  // all zeroed once at the start of the step
+  s.gcnt_sites = 4 * c->n_layers;
+  s.gcnt = off, off += align256((size_t)s.gmax_tiles * s.gcnt_sites * 4);
   s.total = off;
   return s;
 }
@@ -643,11 +647,14 @@ hspec_status hspec_draft_step(hspec_drafter* dr, const hspec_step_in* in, const 
   uint8_t* g = ws + sp.g;
   float* h0 = (float*)(ws + sp.h0);
   int* err = device_error_word();
-  if (sp.gmax_tiles > 0 && cudaMemsetAsync(ws + sp.gcnt, 0, (size_t)sp.gmax_tiles * 4, s) != cudaSuccess)
+  if (sp.gmax_tiles > 0 && cudaMemsetAsync(ws + sp.gcnt, 0, (size_t)sp.gmax_tiles * sp.gcnt_sites * 4, s) != cudaSuccess)
     FAIL(HSPEC_ERR_CUDA, "clearing the GEMM tile counters failed");
   // the projection and MLP GEMMs may split K over the step workspace
+  int site = 0;  // the K-cut GEMM calls take the counter slices in turn
   auto split = [&](GemmArgs ga) {
-    ga.part = (float*)(ws + sp.gpart), ga.tile_cnt = (int*)(ws + sp.gcnt);
+    ga.part = (float*)(ws + sp.gpart);
+    ga.tile_cnt = site < sp.gcnt_sites ? (int*)(ws + sp.gcnt) + (size_t)site * sp.gmax_tiles : nullptr;
+    ++site;
     ga.part_bytes = sp.gpart_bytes, ga.max_tiles = sp.gmax_tiles;
     return ga;
   };
