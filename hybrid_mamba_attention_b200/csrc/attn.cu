@@ -177,7 +177,7 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(AttnArgs a) {
   // A partial with l = 0 saw no key and is skipped.
   int ns = 0, s0 = 0, k0 = 0, t_seq = 0, Z = 1;
   size_t base0 = 0, stride = R;
-  if (a.block_in_last_split) {
+  if (a.tile_pieces) {
     const int* off = a.sched + 64;
     const int n_rb = (R + kAttnTcRows - 1) / kAttnTcRows, spr = a.Hkv * n_rb;
     const int rb = row / kAttnTcRows, rr = row % kAttnTcRows;
@@ -196,7 +196,7 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(AttnArgs a) {
     base0 = (((size_t)c * a.Hkv + g) * a.n_splits * a.sub_splits) * R + row;
   }
   auto has = [&](int q) -> bool {
-    if (!a.block_in_last_split) return true;
+    if (!a.tile_pieces) return true;
     const int p = q >> 1, hh = q & 1;
     const int lo = max(s0, (k0 + p) * Z), hi = min(s0 + t_seq, (k0 + p + 1) * Z);
     return hi - lo > hh;

@@ -219,7 +219,7 @@ AttnArgs attn_args(const hspec_cfg* c, const AttnPlan& p, const hspec_kv_view* k
   a.n_splits = p.n_splits;
   a.max_chunks = p.max_chunks;
   a.causal_block = (c->flags & HSPEC_FLAG_CAUSAL_BLOCK) != 0;
-  a.block_in_last_split = c->dtype == HSPEC_DTYPE_BF16;
+  a.tile_pieces = c->dtype == HSPEC_DTYPE_BF16;
   a.sub_splits = attn_sub_splits(c->dtype);
   a.ws_acc = (float*)ws;
   a.ws_ml = a.ws_acc + p.rows * a.D;

@@ -120,7 +120,8 @@ struct AttnArgs {
   int n_splits;                          // fp32 path: splits per (request, kv head) upper bound
   int max_chunks;                        // tensor-core path: chunk bound of the workspace
   bool causal_block;
-  bool block_in_last_split;              // tensor-core path: block keys ride with the last context split
+  bool tile_pieces;                      // tensor-core path: partials are the pieces of the tile-space
+                                         // partition (the block's keys end each sequence)
   int sub_splits;                        // partials per split (tensor-core path: one per softmax warpgroup)
   float* ws_acc; float* ws_ml;           // split partials
   // tensor-core path: [1] total tiles T, [2] chunk length Z, [3] number of chunks,
