@@ -202,63 +202,52 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(AttnArgs a) {
     return hi - lo > hh;
   };
   auto ml_of = [&](int q) -> float2 { return *(const float2*)(a.ws_ml + (base0 + (size_t)q * stride) * 2); };
-  // this warp's partials: q = wq + W k
+  // This warp's partials q = wq + W k, k < nk, in blocks of 4: the (m, l) and the rows
+  // of a block are loaded together (one round trip), then folded into the running
+  // (M, L, o), rescaled when the block raises the max -- one pass of the softmax merge
+  // in a fixed order.  A missing partial is read (in range) but not used.
   const int nk = ns > wq ? (ns - wq + W - 1) / W : 0;
-  float M = -INFINITY;
-  for (int k = lane; k < nk; k += 32) {
-    const int q = wq + W * k;
-    if (has(q)) {
-      const float2 ml = ml_of(q);
-      if (ml.y > 0.f) M = fmaxf(M, ml.x);
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  float L = 0.f;
-  for (int k = lane; k < nk; k += 32) {
-    const int q = wq + W * k;
-    if (has(q)) {
-      const float2 ml = ml_of(q);
-      if (ml.y > 0.f) L += exp2f(ml.x - M) * ml.y;
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-  // o_w = sum_q 2^(m_q - M_w) acc_q: the acc loads do not depend on the weights, so the
-  // loads of several partials are in flight together (a missing partial is read but
-  // not used)
+  float M = -INFINITY, L = 0.f;
   float o[4] = {0.f, 0.f, 0.f, 0.f};
   const bool v4_lane = V4 && 4 * lane < a.D;
-  for (int kk0 = 0; kk0 < nk; kk0 += 32) {
-    float w_l = 0.f;
-    if (kk0 + lane < nk && has(wq + W * (kk0 + lane))) {
-      const float2 ml = ml_of(wq + W * (kk0 + lane));
-      if (ml.y > 0.f) w_l = exp2f(ml.x - M);
-    }
-    const int cnt = min(32, nk - kk0);
-#pragma unroll 8
-    for (int k = 0; k < cnt; ++k) {
-      const float w = __shfl_sync(0xffffffffu, w_l, k);
-      const float* accp = a.ws_acc + (base0 + (size_t)(wq + W * (kk0 + k)) * stride) * a.D;
+  for (int k0 = 0; k0 < nk; k0 += 4) {
+    float2 ml[4];
+    float x[4][4];
+    bool use[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int k = k0 + u;
+      const int q = wq + W * min(k, nk - 1);
+      use[u] = k < nk && has(q);
+      ml[u] = ml_of(q);
+      const float* accp = a.ws_acc + (base0 + (size_t)q * stride) * a.D;
       if (V4) {
-        if (v4_lane) {
-          const float4 x = *(const float4*)(accp + 4 * lane);
-          o[0] = w != 0.f ? fmaf(w, x.x, o[0]) : o[0];
-          o[1] = w != 0.f ? fmaf(w, x.y, o[1]) : o[1];
-          o[2] = w != 0.f ? fmaf(w, x.z, o[2]) : o[2];
-          o[3] = w != 0.f ? fmaf(w, x.w, o[3]) : o[3];
-        }
+        float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (v4_lane) f = *(const float4*)(accp + 4 * lane);
+        x[u][0] = f.x, x[u][1] = f.y, x[u][2] = f.z, x[u][3] = f.w;
       } else {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int e = lane + 32 * i;
-          if (e < a.D) {
-            const float x = accp[e];
-            o[i] = w != 0.f ? fmaf(w, x, o[i]) : o[i];
-          }
-        }
+        for (int i = 0; i < 4; ++i) x[u][i] = lane + 32 * i < a.D ? accp[lane + 32 * i] : 0.f;
       }
     }
+    float mb = M;
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (use[u] && ml[u].y > 0.f) mb = fmaxf(mb, ml[u].x);
+    if (mb == -INFINITY) continue;  // no partial with keys yet
+    const float sc = M == -INFINITY ? 0.f : exp2f(M - mb);
+    L *= sc;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o[i] *= sc;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (!(use[u] && ml[u].y > 0.f)) continue;
+      const float w = exp2f(ml[u].x - mb);
+      L = fmaf(w, ml[u].y, L);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) o[i] = fmaf(w, x[u][i], o[i]);
+    }
+    M = mb;
   }
   T* out = (T*)a.out + (size_t)(c * a.K + j) * a.o_rs + (size_t)h * a.D;
   auto store = [&](const float* v, float inv) {
