@@ -164,13 +164,13 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* kv_full = (uint64_t*)(smem + L::OFF_BAR);  // one arrival per producer warp
   uint64_t* kv_empty = kv_full + NS;
   uint64_t* s_full = kv_empty + NS;   // [NSB] S_b written by Q.K^T
-  uint64_t* s_free = s_full + NSB;    // [NSB] P.V of S_b's tile finished (S_b / P free)
+  uint64_t* s_free = s_full + NSB;    // [NSB] P.V of S_b's tile finished (S_b / P free, O_w
+                                      // holds that tile)
   // P of S_b's tile written (one barrier per S buffer: a group's next tile may finish
   // its softmax before the MMA thread has taken this one, and the phases of one
   // barrier must not run two ahead of its waiter)
   uint64_t* p_full = s_free + NSB;    // [NSB]
-  uint64_t* pv_done = p_full + NSB;   // [2]   group w's P.V finished (O_w quiescent)
-  uint64_t* q_full = pv_done + 2;     // [2]
+  uint64_t* q_full = p_full + NSB;    // [2]
   uint64_t* q_empty = q_full + 2;     // [2]
   uint64_t* drain = q_empty + 2;      // [2] every MMA of an issuer (and its arrivals) finished
   uint32_t* tmem_slot = (uint32_t*)(drain + 2);
@@ -195,7 +195,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc::mbar_init(&p_full[b], 4);
     }
     for (int w = 0; w < 2; ++w) {
-      tc::mbar_init(&pv_done[w], 1);
       tc::mbar_init(&q_full[w], 1);
       tc::mbar_init(&q_empty[w], 1);
     }
@@ -442,7 +441,6 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc::mma_bf16_ts(tmem + L::O_COL(w), pt + kk * 8, tc::sdesc_mn128(v + kk * L::V_PAGE, 2048), idesc_pv,
                             (kk > 0 || !first) ? 1u : 0u);
           tc::mma_commit(&kv_empty[s]);
-          tc::mma_commit(&pv_done[w]);
           tc::mma_commit(&s_free[pv & (NSB - 1)]);  // P read: S buffer free for tile pv + NSB
           ++pv;
           idle_since = 0;
@@ -492,7 +490,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     for (int i = wg; ok; i += 2) {
-      const int n = i >> 1;                 // this group's tile count so far
       const int b = i & (NSB - 1);
       ok = __all_sync(0xffffffffu, tc::mbar_wait(&s_full[b], (i / NSB) & 1, err));
       if (!ok || i >= *end_tile) break;
@@ -563,16 +560,14 @@ __global__ void __launch_bounds__(THREADS, 1)
       // P over the first half of S_b (bf16 pairs: the row's keys 2c, 2c + 1 in column c)
       if constexpr (SP) tc::tmem_st16x2_16u<TT / 4>(tmem + lane_off + L::S_COL(b), pk);
       else tc::tmem_stu(tmem + lane_off + L::S_COL(b), pk);
-      // The group's previous P.V (before O_w may be rescaled).  It is waited for at
-      // every tile, not only before a rescale: softmax may run several tiles ahead of
-      // the P.V's, and a parity wait is only unambiguous while its waiter is at most
-      // one phase behind the barrier.
-      if (n >= 1) {
-        ok = __all_sync(0xffffffffu, tc::mbar_wait(&pv_done[wg], (n - 1) & 1, err));
+      if (__any_sync(0xffffffffu, rescale)) {
+        // O_w may be rescaled only once the group's previous P.V (tile i - 2, S buffer
+        // (i - 2) % NSB) has finished.  Its phase of s_free is unambiguous here: the
+        // phase before it (tile i - 2 - NSB) completed before the Q.K^T of tile i - 2
+        // was issued, and the one after it needs a P this group has not written yet.
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(&s_free[(i - 2) & (NSB - 1)], ((i - 2) / NSB) & 1, err));
         if (!ok) break;
         tc::tc_fence_after();
-      }
-      if (__any_sync(0xffffffffu, rescale)) {
         // O_w holds this group's earlier tiles of the piece
 #pragma unroll
         for (int cb = 0; cb < OCB; ++cb) {
@@ -602,7 +597,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 
       if (local >= n_tiles - 2) {
         // this group's last tile of the piece: write its partial (half of the piece)
-        ok = __all_sync(0xffffffffu, tc::mbar_wait(&pv_done[wg], n & 1, err));
+        // this tile's P.V (same argument for the parity of s_free as above)
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(&s_free[b], (i / NSB) & 1, err));
         if (!ok) break;
         tc::tc_fence_after();
         // half (local & 1): the piece's even or odd tiles, whichever group ran them,
