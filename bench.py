@@ -222,11 +222,11 @@ def step_roofline_ms(sh, C, K, ctx_lens, peaks):
 
 # DRAM bytes (read + write) per algorithmic byte of the paged-attention kernel, from
 # one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum) of the current
-# attn_tc_kernel at Llama-3-8B shapes, C=32, ctx U[512,8192] (677.7 MB for 656.2 MB of
+# attn_tc_kernel at Llama-3-8B shapes, C=32, ctx U[512,8192] (677.2 MB for 656.2 MB of
 # K/V; the excess is the partials of the pieces).  The step's attention launch is too large
 # to capture; its traffic is this ratio times its algorithmic bytes (traffic grows
 # with the K/V read).  Set to None whenever the kernel changes until re-captured.
-ATTN_TRAFFIC_PER_BYTE = 1.0328
+ATTN_TRAFFIC_PER_BYTE = 1.0320
 
 
 def roofline_of(name, work, avg_ms, peaks, traffic=None, sustained=True):
