@@ -1,0 +1,95 @@
+"""Host-side checks of the benchmark's work model and roofline arithmetic (no GPU).
+
+Every roofline fraction that bench.py reports divides by the algorithmic bytes and
+flops of `bench.step_work`, which is written from the layer shapes.  These tests tie
+that model to the weight tensors the seeded generators actually allocate (a wrong
+dimension or a missing matrix in the model fails them), and check the fraction
+arithmetic on made-up timings.
+"""
+from dataclasses import replace
+
+import numpy as np
+import pytest
+
+import bench
+from hybrid_mamba_attention_b200 import inputs as I
+
+# A small drafter with every part of the full one: M,A,M,A layers, a SwiGLU MLP after
+# each mixer and the shared LM head.
+SMALL = replace(I.LLAMA_FULL, name="small_full", d=128, Hq=4, Hkv=2, D=32, H=4, P=16, N=8, d_ff=256,
+                vocab=1000)
+PEAKS = {"hbm_gbs": 6452.8, "bf16_tflops": 1644.4, "bf16_tflops_sustained": 1395.6}
+
+PER_TOKEN = ("W_in", "W_out", "W_qkv", "W_o", "W_gate", "W_up", "W_down")  # applied to every block token
+
+
+def _launches(sh):
+    """Launches of each kernel group in one draft step."""
+    nM, nA, nL = sh.layers.count("M"), sh.layers.count("A"), len(sh.layers)
+    return {"in_proj": nM, "inject": nM, "ssd_scan": nM, "out_proj": nM, "qkv_proj": nA, "attn_paged": nA,
+            "o_proj": nA, "mlp_gate_up": nL, "mlp_down": nL, "lm_head_argmax": 1}
+
+
+def _weights(sh):
+    w = I.make_weights(sh, seed=7)
+    per_token = sum(t.numel() for layer in w["layers"] for k, t in layer.items() if k in PER_TOKEN)
+    per_token += w["W_lm"].numel()
+    per_request = sum(layer["W_inj"].numel() for layer in w["layers"] if "W_inj" in layer)
+    esize = w["W_lm"].element_size()
+    return per_token, per_request, esize
+
+
+def test_weight_bytes_equal_the_generated_weights():
+    # with no requests only the weights are left to read, once per launch
+    per_token, per_request, esize = _weights(SMALL)
+    w = bench.step_work(SMALL, 0, 4, np.zeros(0, dtype=np.int64))
+    total = sum(n * w[g]["bytes"] for g, n in _launches(SMALL).items())
+    assert total == (per_token + per_request) * esize
+
+
+@pytest.mark.parametrize("C,K", [(1, 1), (3, 4), (16, 16)])
+def test_gemm_flops_equal_two_per_weight_and_row(C, K):
+    # every block token meets every per-token matrix once; the injection runs once per request
+    per_token, per_request, _ = _weights(SMALL)
+    ctx = np.full(C, 37, dtype=np.int64)
+    w = bench.step_work(SMALL, C, K, ctx)
+    gemms = {g: n for g, n in _launches(SMALL).items() if g not in ("attn_paged", "ssd_scan")}
+    flops = sum(n * w[g]["flops"] for g, n in gemms.items())
+    assert flops == 2.0 * (C * K * per_token + C * per_request)
+
+
+def test_attention_bytes_grow_with_the_context_read():
+    # one more context token of one request adds its K and V rows of every kv head
+    sh = SMALL
+    ctx = np.array([100, 250], dtype=np.int64)
+    a = bench.step_work(sh, 2, 4, ctx)["attn_paged"]["bytes"]
+    b = bench.step_work(sh, 2, 4, ctx + np.array([1, 0]))["attn_paged"]["bytes"]
+    assert b - a == 2 * sh.Hkv * sh.D * 2  # K and V, bf16
+
+
+def test_roofline_fraction_is_achieved_over_the_peak():
+    # HBM-bound: the peak's bytes in twice the time is half the peak
+    r = bench.roofline_of("mlp_down", {"bytes": 6452.8e9, "flops": 1.0}, 2000.0, PEAKS)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert r["achieved"] == pytest.approx(3226.4) and r["frac"] == pytest.approx(0.5)
+    # tensor-bound: a millisecond of sustained-peak flops in a millisecond is 1.0
+    fl = 1395.6e12 * 1e-3
+    r = bench.roofline_of("mlp_gate_up", {"bytes": 1.0, "flops": fl}, 1.0, PEAKS)
+    assert r["bound"] == "tensor" and r["frac"] == pytest.approx(1.0)
+    # a kernel timed alone is held to the burst peak instead
+    r = bench.roofline_of("mlp_gate_up", {"bytes": 1.0, "flops": fl}, 1.0, PEAKS, sustained=False)
+    assert r["peak"] == 1644.4 and r["frac"] == pytest.approx(1395.6 / 1644.4, abs=1e-4)
+    # the attention and the scan are reported against HBM even where their flops would dominate
+    r = bench.roofline_of("attn_paged", {"bytes": 1.0, "flops": fl}, 1.0, PEAKS, traffic=123)
+    assert r["bound"] == "hbm" and r["traffic"] == 123
+
+
+def test_step_roofline_never_shrinks_with_more_work():
+    prev = 0.0
+    for C in (1, 2, 8, 32):
+        t = bench.step_roofline_ms(SMALL, C, 16, np.full(C, 512, dtype=np.int64), PEAKS)
+        assert t >= prev
+        prev = t
+    short = bench.step_roofline_ms(SMALL, 4, 16, np.full(4, 512, dtype=np.int64), PEAKS)
+    long = bench.step_roofline_ms(SMALL, 4, 16, np.full(4, 4096, dtype=np.int64), PEAKS)
+    assert long > short
