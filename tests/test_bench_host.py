@@ -4,7 +4,8 @@ Every roofline fraction that bench.py reports divides by the algorithmic bytes a
 flops of `bench.step_work`, which is written from the layer shapes.  These tests tie
 that model to the weight tensors the seeded generators actually allocate (a wrong
 dimension or a missing matrix in the model fails them), and check the fraction
-arithmetic on made-up timings.
+arithmetic on made-up timings.  The clock summary, which decides whether a timed run
+saw a slowdown, is checked on made-up nvidia-smi lines.
 """
 from dataclasses import replace
 
@@ -93,3 +94,52 @@ def test_step_roofline_never_shrinks_with_more_work():
     short = bench.step_roofline_ms(SMALL, 4, 16, np.full(4, 512, dtype=np.int64), PEAKS)
     long = bench.step_roofline_ms(SMALL, 4, 16, np.full(4, 4096, dtype=np.int64), PEAKS)
     assert long > short
+
+
+class _Done:
+    """Stands in for the finished nvidia-smi process and its reader thread."""
+
+    def terminate(self):
+        pass
+
+    def wait(self, timeout=None):
+        return 0
+
+    def kill(self):
+        pass
+
+    def join(self, timeout=None):
+        pass
+
+
+def _smi(sm, smax, power_cap="Not Active", hw="Not Active"):
+    # the FIELDS order: index, clocks.sm, clocks.max.sm, power.draw, active mask, hw_slowdown,
+    # hw_thermal_slowdown, sw_thermal_slowdown, sw_power_cap
+    return f"0, {sm}, {smax}, 950.1, 0x0000000000000004, {hw}, Not Active, Not Active, {power_cap}"
+
+
+def test_clock_summary_keeps_the_timed_region_only():
+    cs = bench.ClockSampler(0)
+    cs.proc, cs.thread = _Done(), _Done()
+    cs.lines = [(0.0, _smi(1965, 1965)),                       # before the region: not counted
+                (1.0, _smi(1500, 1965, power_cap="Active")),
+                (1.1, _smi(1520, 1965, power_cap="Active")),
+                (1.2, _smi(1540, 1965)),
+                (1.3, "garbled line"),                          # skipped
+                (9.0, _smi(900, 1965, hw="Active"))]            # after the region: not counted
+    cs.window(0.95, 1.25)
+    r = cs.stop()
+    assert r["sm_mhz"] == 1520 and r["sm_max_mhz"] == 1965 and r["samples"] == 3
+    assert r["reasons"] == ["sw_power_cap"] and r["in_timed_region"] is True
+
+
+def test_clock_summary_reports_a_slowdown_inside_the_region():
+    cs = bench.ClockSampler(0)
+    cs.proc, cs.thread = _Done(), _Done()
+    cs.lines = [(1.0, _smi(1200, 1965, hw="Active")), (1.1, _smi(1250, 1965))]
+    cs.window(0.9, 1.2)
+    assert bench.ClockSampler.stop(cs)["reasons"] == ["hw_slowdown"]
+
+
+def test_clock_summary_without_nvidia_smi_says_so():
+    assert bench.ClockSampler(0).stop()["reasons"] == ["unavailable"]
