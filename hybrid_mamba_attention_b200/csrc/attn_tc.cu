@@ -18,27 +18,31 @@
 // byte read from HBM feeds all R queries; with R <= 64 the rows are spread 16 per
 // 32-lane TMEM quarter so that all four SM sub-partitions share the softmax work;
 // rows without a query are zero.
-// Warp roles (320 threads):
-//   warp 0      producer: walks the CTA's pieces, loads each one's Q tile (TMA) into one of
-//               two Q buffers, reads page ids two tiles ahead, and streams its
-//               64-token K/V tiles through a 4-stage ring -- per tile one 3-D TMA box
-//               of 16 tokens x 64 dims of head g per page and column block (128-byte
-//               swizzle), all boxes of a tile issued at once, one lane each -- and
-//               writes the tile's description next to it.  A sequence's last tiles
-//               are the block's own keys (one more tile for K <= 64).
-//   warp 1      TMEM owner and single-thread MMA issuer, driven by readiness rather
-//               than by a fixed order: it issues O_w += P_w . V_i (M=128, N=D, K=64)
-//               as soon as the P of tile i is in shared memory, and S_b = Q . K_i^T
-//               (M=128, N=64, K=D) into S buffer b = i % 4 as soon as tile i has
-//               landed and softmax has read S_b's previous tile, so that the S of a
-//               group's next tile is ready while it still works on the current one.
-//   warps 2..5  softmax warpgroup 0 (tiles i even), warps 6..9 warpgroup 1 (i odd):
-//               one TMEM lane (query row) per thread; mask, running max in the exp2
-//               domain, P = exp2(s - m) to shared memory as bf16; O_w is rescaled in
-//               TMEM only when the running max grows by more than 8.  Each group
-//               keeps its own (m, l, O) per piece and writes its own partial when its
-//               last tile of the piece is done -- the half of the piece made of its
-//               even (or odd) tiles, so the arithmetic does not depend on timing;
+// Warp roles (448 threads, one CTA per SM):
+//   warps 0..3  producers: all four walk the CTA's pieces.  Warp 0 loads each piece's
+//               Q tile (TMA) into one of two Q buffers.  Page ids are read two tiles
+//               ahead.  The 64-token K/V tiles stream through a ring of 6 stages (5 for
+//               M = 128) -- per tile one 3-D K box per page and 64-dim column block
+//               (16 tokens x 64 dims of head g, 128-byte swizzle) and one 4-D V box per
+//               page (both column blocks), box x issued by warp x % 4, all boxes of a
+//               tile at once -- and warp 0 writes the tile's description next to it.
+//               A sequence's last tiles are the block's own keys (one more tile for
+//               K <= 64).
+//   warp 4      TMEM owner and Q.K^T issuer: S_b = Q . K_i^T (N = 64, K = D) into S
+//               buffer b = i % 4 as soon as tile i has landed and the P.V of tile
+//               i - 4 has read S_b, so that the S of a group's next tile is ready while
+//               the group still works on the current one.
+//   warp 5      P.V issuer: O_w += P_i . V_i (N = D, K = 64) as soon as the P of tile
+//               i is in TMEM, with P (the A operand) read from TMEM; its commit frees
+//               the K/V stage and the S buffer.
+//   warps 6..9  softmax warpgroup 0 (tiles i even), warps 10..13 warpgroup 1 (i odd):
+//               one query row per thread (M = 64: two threads per row, one in each
+//               half-warp, 32 scores each); mask, running max in the exp2 domain, P = exp2(s - m)
+//               written back over S as packed bf16; O_w is rescaled in TMEM only when
+//               the running max grows by more than 8, after the group's previous P.V.
+//               Each group keeps its own (m, l, O) per piece and writes its own partial
+//               when its last tile of the piece is done -- the half of the piece made of
+//               its even (or odd) tiles, so the arithmetic does not depend on timing;
 //               the merge kernel combines the halves and the pieces.
 // Every wait gives up after a time bound and sets the device error word.
 #include <stdint.h>
