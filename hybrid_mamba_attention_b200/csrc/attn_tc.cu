@@ -37,9 +37,10 @@
 //               the K/V stage and the S buffer.
 //   warps 6..9  softmax warpgroup 0 (tiles i even), warps 10..13 warpgroup 1 (i odd):
 //               one query row per thread (M = 64: two threads per row, one in each
-//               half-warp, 32 scores each); mask, running max in the exp2 domain, P = exp2(s - m)
-//               written back over S as packed bf16; O_w is rescaled in TMEM only when
-//               the running max grows by more than 8, after the group's previous P.V.
+//               half-warp, 32 scores each); mask, running max in the exp2 domain,
+//               P = exp2(s - m) written back over S as packed bf16; O_w is rescaled in
+//               TMEM only when the running max grows by more than 8, after the group's
+//               previous P.V.
 //               Each group keeps its own (m, l, O) per piece and writes its own partial
 //               when its last tile of the piece is done -- the half of the piece made of
 //               its even (or odd) tiles, so the arithmetic does not depend on timing;
