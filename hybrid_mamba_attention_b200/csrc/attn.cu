@@ -15,8 +15,12 @@
 // the softmax runs online in the exp2 domain.  The CTA writes its partial
 // (m, l, unnormalised acc) per row.
 //
-// attn_merge_kernel: one warp per output row (c, j, h) combines the splits of that
-// request: o = sum_s 2^(m_s - M) acc_s / sum_s 2^(m_s - M) l_s.
+// attn_merge_kernel: W = 1, 2, 4 or 8 warps per output row (c, j, h) combine the
+// partials of that row, o = sum_s 2^(m_s - M) acc_s / sum_s 2^(m_s - M) l_s.  Warp w
+// takes the partials s = w (mod W) in one pass over blocks of four (their (m, l) and
+// rows loaded together, folded into a running (M, L, o) that is rescaled when a block
+// raises the maximum); the W warps' states are then combined in warp order through
+// shared memory, so the result does not depend on timing.
 #include "../../include/hspec.h"
 #include "common.cuh"
 #include "kernels.cuh"

@@ -14,8 +14,9 @@
 //               commits each stage back to the producer and each finished
 //               accumulator to the epilogue;
 //   warps 2..5  epilogue: tcgen05.ld of their 32-lane quarter of TMEM, then the fused
-//               epilogue (store, residual add, SwiGLU, per-row argmax), while the
-//               next tile accumulates into the other TMEM buffer.
+//               epilogue (store, residual add, SwiGLU, per-row argmax, or the readout
+//               of the injected SSD state into y), while the next tile accumulates
+//               into the other TMEM buffer.
 // Rows/columns beyond M/N are zero-filled by TMA and skipped by the epilogue.
 // When whole tiles would leave SMs idle the K loop is cut, in one of two ways:
 //   stream-K (one row of tiles, M <= 128): the (tile, 64-wide K block) pairs form one
