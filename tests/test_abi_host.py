@@ -167,3 +167,43 @@ def test_step_rejects_missing_inputs(H):
     st = H._lib.hspec_draft_step(h, ct.byref(si), ct.byref(so), 256, 16, None)
     assert st == H.HSPEC_ERR_WORKSPACE
     H.hspec_drafter_destroy(h)
+
+
+def test_empty_batches_and_block_sizes_rejected_before_launch(H):
+    # C = 0 requests and K outside 1..64 are refused by every entry point before anything is
+    # launched (the header states C >= 1 and 1 <= K <= 64); the workspace queries answer 0
+    from hybrid_mamba_attention_b200 import inputs as I
+    cfg = small_cfg(H)
+    kv = H.hspec_kv_view(k_pool=256, v_pool=256, num_pages=4, page_table=256, max_pages=4)
+    n0 = H.hspec_launch_count()
+    assert H._lib.hspec_inject_state(ct.byref(cfg), 256, 256, 0, 256, None) == H.HSPEC_ERR_INVALID_ARG
+    st = H._lib.hspec_ssd_block_scan(ct.byref(cfg), 256, 256, 256, 256, 256, 256, 256, 0, 8, 256, None, None)
+    assert st == H.HSPEC_ERR_INVALID_ARG
+    for C, K in ((0, 8), (1, 0), (1, 65)):
+        st = H._lib.hspec_attn_paged_block(ct.byref(cfg), 256, ct.byref(kv), 256, 256, 256, C, K, 256, 256,
+                                           1 << 30, None)
+        assert st == H.HSPEC_ERR_UNSUPPORTED, (C, K)
+        st = H._lib.hspec_attn_paged_block_noalloc(ct.byref(cfg), 256, ct.byref(kv), 256, 256, 256, C, K, 256,
+                                                   None)
+        assert st == H.HSPEC_ERR_UNSUPPORTED, (C, K)
+    assert H.hspec_attn_workspace_size(cfg, 0, 8, 4) == 0 and H.hspec_attn_workspace_size(cfg, 1, 0, 4) == 0
+    # verification over a vocabulary
+    vcfg = H.make_cfg(I.LLAMA_FULL)
+    for C, K in ((0, 8), (1, 0), (1, 65)):
+        st = H._lib.hspec_verify_greedy(ct.byref(vcfg), 256, 256, C, K, 256, 256, None, 256, 1 << 30, None)
+        assert st == H.HSPEC_ERR_UNSUPPORTED, (C, K)
+    assert H.hspec_verify_workspace_size(vcfg, 0, 8) == 0
+    # the whole draft step
+    mw = H.hspec_model_weights()
+    for i in range(2):
+        for f, _ in H.hspec_layer_weights._fields_:
+            setattr(mw.layers[i], f, 256)
+    h = H.hspec_drafter_create(H.make_cfg(I.TINY), mw)
+    so = H.hspec_step_out()
+    for C, K in ((0, 8), (1, 0), (1, 65)):
+        si = H.hspec_step_in(C=C, K=K, h_last=256, x_in=256, ctx_lens=256)
+        si.kv[0] = kv
+        assert H._lib.hspec_draft_step(h, ct.byref(si), ct.byref(so), 256, 1 << 30, None) == H.HSPEC_ERR_UNSUPPORTED
+    assert H.hspec_step_workspace_size(H.make_cfg(I.TINY), 0, 8, 4) == 0
+    H.hspec_drafter_destroy(h)
+    assert H.hspec_launch_count() == n0
