@@ -424,12 +424,7 @@ def run_ours(args, rank, world, local):
                 "warmup": args.warmup, "ms_per_step": round(ms_max, 4), "us_per_step": round(ms_max * 1e3, 1),
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
                 "data": "synthetic (seeded random-init weights and KV of the stated shapes)",
-                "config": {"workload": f"full draft step {wl.name}: 4-layer M,A,M,A hybrid drafter, Llama-3-8B "
-                                       f"shapes, SwiGLU 16384, vocab 128256"
-                                       + (f" (draft head {wl.shapes.draft_vocab} rows)" if wl.shapes.draft_vocab else "")
-                                       + ", ctx U[512,16384], 16-token pages",
-                           "C": wl.C, "K": wl.K, "global_batch": wl.C * world, "parallelism": f"replicas x{world}",
-                           "l2": "inputs ~20 GB > 126 MB L2 (no flush needed)"},
+                "config": step_config(wl, world),
                 "roofline": roof, "attention_roofline": attn_roof, "kernels": kernels,
                 "kernels_pass_ms_per_step": round(pms, 4),
                 "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clk}
@@ -538,6 +533,16 @@ def run_kernel(args, rank, world, local):
 
 # ---------------------------------------------------------------- reference arm
 
+def step_config(wl, world):
+    """The `config` object of the draft-step line, the same for both arms."""
+    return {"workload": f"full draft step {wl.name}: 4-layer M,A,M,A hybrid drafter, Llama-3-8B shapes, "
+                        f"SwiGLU 16384, vocab 128256"
+                        + (f" (draft head {wl.shapes.draft_vocab} rows)" if wl.shapes.draft_vocab else "")
+                        + ", ctx U[512,16384], 16-token pages",
+            "C": wl.C, "K": wl.K, "global_batch": wl.C * world, "parallelism": f"replicas x{world}",
+            "l2": "inputs ~20 GB > 126 MB L2 (no flush needed)"}
+
+
 def run_reference(args, rank, world):
     """The CPU oracle as the reference arm, on this arm's config and metric."""
     if rank != 0:
@@ -565,10 +570,10 @@ def run_reference(args, rank, world):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(sec * 1e3, 1),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded random-init weights and KV of the stated shapes)",
-            "config": {"workload": f"full draft step {wl.name} (CPU oracle, one request per step)", "C": wl.C,
-                       "K": wl.K},
+            "config": step_config(wl, world),
             "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
-                             "sample": f"one request of the {wl.C}-request batch per step"},
+                             "sample": f"one request of the {wl.C}-request batch per step (requests are "
+                                       f"independent, so the batch takes C times as long)"},
             "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 

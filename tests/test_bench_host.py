@@ -143,3 +143,24 @@ def test_clock_summary_reports_a_slowdown_inside_the_region():
 
 def test_clock_summary_without_nvidia_smi_says_so():
     assert bench.ClockSampler(0).stop()["reasons"] == ["unavailable"]
+
+
+def test_reference_line_carries_this_arms_config_and_metric(monkeypatch, capsys):
+    # the reference arm (the CPU oracle) reports on the same config, metric and unit as the
+    # CUDA arm; its end-to-end figure is its own value with no host-device copies
+    import json
+    monkeypatch.setattr(I, "make_step_inputs", lambda wl, dev: {})
+    monkeypatch.setattr(bench, "oracle_one_request", lambda I_, wl, r, request=0: (2.0, 1000, 8))
+
+    class Args:
+        steps, warmup, C, K, draft_vocab = 2, 3, 128, 16, 0
+
+    bench.run_reference(Args(), rank=0, world=1)
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference"
+    assert line["config"] == bench.step_config(I.full_workload(128, 16), 1)
+    assert line["metric"] == bench.METRIC and line["unit"] == bench.UNIT and line["higher_is_better"] is True
+    assert line["value"] == pytest.approx(16 / 2.0)
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"] == {"value": line["value"], "unit": bench.UNIT, "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
