@@ -22,7 +22,9 @@ _lib = None
 def lib():
     global _lib
     if _lib is None:
-        _lib = ct.CDLL(_build.build())
+        # HSPEC_ORACLE_LIB loads another build of this same source instead (the mutation
+        # test builds copies with one planted mistake each and checks that a pin fails)
+        _lib = ct.CDLL(os.environ.get("HSPEC_ORACLE_LIB") or _build.build())
         _lib.oracle_bf16_round.restype = ct.c_double
         _lib.oracle_bf16_round.argtypes = [ct.c_double]
         for name in ("oracle_attn_paged", "oracle_draft_step"):
