@@ -57,6 +57,21 @@ MUTATIONS = [
     ("injected state read as [H][N][P] instead of [H][P][N]",
      "h[i] = h0 ? h0[(size_t)hh * P * N + i] : 0.0;",
      "h[i] = h0 ? h0[(size_t)hh * P * N + (i % N) * P + i / N] : 0.0;"),
+    ("LM-head argmax tie won by the highest id",
+     "if (lg[v] > lg[best]) best = v;",
+     "if (lg[v] >= lg[best]) best = v;"),
+    ("verification lets a NaN logit win",
+     "if (std::isnan(x)) continue;",
+     "if (false) continue;"),
+    ("verification returns the last accepted token instead of the target's next one",
+     "next_token[c] = t[a];",
+     "next_token[c] = t[a > 0 ? a - 1 : 0];"),
+    ("verification advances the context by the accepted drafts only",
+     "if (ctx_lens) ctx_lens[c] += a + 1;",
+     "if (ctx_lens) ctx_lens[c] += a;"),
+    ("reduced draft head returns the draft row instead of the target id",
+     "reduced ? io->draft_to_target[am[j]] : am[j]",
+     "am[j]"),
 ]
 
 
