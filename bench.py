@@ -1,7 +1,8 @@
 """Benchmark of the H-Spec block-parallel draft step on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl hspec|reference]
-                    [--C 128] [--K 16] [--sweep] [--no-cpu-baseline]
+                    [--C 128] [--K 16] [--sweep] [--draft-vocab V] [--no-cpu-baseline]
+                    [--kernel step|attn|inject|ssd|verify|gemm] [--workload NAME]
 
 One step = one hspec_draft_step over a batch of C requests of the 4-layer M,A,M,A
 drafter on Llama-3-8B shapes (SwiGLU 16384, shared 128256-token LM head), K block
@@ -13,6 +14,9 @@ and KV) exceed the 126 MB L2, so no flush is needed between steps.
 Multi-GPU: requests are independent, so each rank runs its own batch of C
 requests (weak scaling, replicas only, no collective on the data path); the step
 time is the max over ranks.
+
+--impl reference times the CPU oracle on the same config and metric (rank 0 only).
+--kernel times one kernel-level call on a named workload instead of the step.
 """
 from __future__ import annotations
 
