@@ -207,3 +207,34 @@ def test_empty_batches_and_block_sizes_rejected_before_launch(H):
     assert H.hspec_step_workspace_size(H.make_cfg(I.TINY), 0, 8, 4) == 0
     H.hspec_drafter_destroy(h)
     assert H.hspec_launch_count() == n0
+
+
+def test_plain_c_program_links_and_calls_the_library(H, tmp_path):
+    # a C caller needs only the header and the shared library: build one against them and
+    # call the host-side entry points (no device work)
+    prog = tmp_path / "use.c"
+    prog.write_text(r'''
+#include <stdio.h>
+#include "hspec.h"
+int main(void) {
+  hspec_cfg cfg = {0};
+  cfg.d_model = 256; cfg.n_q_heads = 4; cfg.n_kv_heads = 2; cfg.head_dim = 64;
+  cfg.n_ssm_heads = 4; cfg.ssm_head_dim = 64; cfg.d_state = 16; cfg.page_size = 16;
+  cfg.n_layers = 2; cfg.layer_kinds[0] = 'M'; cfg.layer_kinds[1] = 'A';
+  cfg.dtype = HSPEC_DTYPE_F32; cfg.rope_theta = 1e4f; cfg.norm_eps = 1e-6f;
+  printf("%s\n", hspec_version());
+  printf("%zu\n", hspec_attn_workspace_size(&cfg, 1, 8, 4));
+  printf("%d\n", hspec_inject_state(&cfg, NULL, NULL, 1, NULL, NULL));
+  printf("%s\n", hspec_status_string(HSPEC_ERR_INVALID_ARG));
+  return 0;
+}
+''')
+    libdir = os.path.dirname(H.LIBRARY_PATH)
+    exe = tmp_path / "use"
+    subprocess.run(["gcc", str(prog), "-I", os.path.join(ROOT, "include"), "-L", libdir, "-l:" +
+                    os.path.basename(H.LIBRARY_PATH), f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split("\n")
+    assert "sm_100a" in out[0]
+    ws = int(out[1])
+    assert ws > 0 and ws % 256 == 0
+    assert int(out[2]) == H.HSPEC_ERR_INVALID_ARG and out[3]
