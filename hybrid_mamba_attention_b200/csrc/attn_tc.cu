@@ -33,12 +33,14 @@
 //               i - 4 has read S_b, so that the S of a group's next tile is ready while
 //               the group still works on the current one.
 //   warp 5      P.V issuer: O_w += P_i . V_i (N = D, K = 64) as soon as the P of tile
-//               i is in TMEM, with P (the A operand) read from TMEM; its commit frees
-//               the K/V stage and the S buffer.
+//               i is in TMEM, with P (the A operand) read from TMEM, as two products
+//               (its bf16 high and low parts); its commit frees the K/V stage and the S
+//               buffer.
 //   warps 6..9  softmax warpgroup 0 (tiles i even), warps 10..13 warpgroup 1 (i odd):
 //               one query row per thread (M = 64: two threads per row, one in each
 //               half-warp, 32 scores each); mask, running max in the exp2 domain,
-//               P = exp2(s - m) written back over S as packed bf16; O_w is rescaled in
+//               P = exp2(s - m) written back over S as bf16 hi = bf16(P) and lo =
+//               bf16(P - hi), which carry P to about 16 bits; O_w is rescaled in
 //               TMEM only when the running max grows by more than 8, after the group's
 //               previous P.V.
 //               Each group keeps its own (m, l, O) per piece and writes its own partial
@@ -96,8 +98,9 @@ struct Lay {
   static constexpr int OFF_META = OFF_KV + NS * STAGE;
   static constexpr int OFF_BAR = OFF_META + 64 * NS;
   static constexpr int SMEM = OFF_BAR + 512 + 1024;
-  // TMEM columns: S_b [TT b, TT b + TT) for b < NSB (P of the tile, bf16 packed,
-  // overwrites its first TT / 2 columns), O_w [256 + 128w, 256 + 128w + D)
+  // TMEM columns: S_b [TT b, TT b + TT) for b < NSB (P of the tile as bf16 pairs
+  // overwrites it: hi = bf16(p) in its first TT / 2 columns, lo = bf16(p - hi) in the
+  // rest), O_w [256 + 128w, 256 + 128w + D)
   static constexpr uint32_t TMEM_COLS = 512;
   __host__ __device__ static constexpr uint32_t S_COL(int b) { return (uint32_t)(b * TT); }
   __host__ __device__ static constexpr uint32_t O_COL(int w) { return (uint32_t)(256 + w * 128); }
@@ -187,6 +190,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int RB = R < ROWS ? R : ROWS;  // rows of a row block's partial
   constexpr bool spread = SP;
   int* err = a.err;
+  const uint64_t lim = a.wait_ns ? (uint64_t)a.wait_ns : tc::kWaitLimitNs;  // pipeline waits
   constexpr int QK_WARP = NPW, PV_WARP = NPW + 1, SM_WARP0 = NPW + 2;
 
   if (threadIdx.x == 0) {
@@ -263,7 +267,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     int k = blockIdx.x;  // this CTA's chunk
     int pos = k < n_chunks ? k * Z : 0, end = k < n_chunks ? min(T, pos + Z) : 0;
     int c = pos < end ? locate(pos) : 0;
-    int tile_i = 0;
+    int tile_i = 0;   // K/V tiles this warp has armed (its arrival on their stage)
+    int q_last = -1;  // warp 0: the last piece whose Q load it armed
     bool ok = true;
     // Every producer warp walks the same pieces and passes the same barriers: the loop
     // ends only after one, when the work is done or a producer has given up waiting.
@@ -292,10 +297,11 @@ __global__ void __launch_bounds__(THREADS, 1)
 
       // Q tile of the piece into Q buffer `slot` once the piece two back is done with it
       if (pw == 0) {
-        if (lane == 0) ok = tc::mbar_wait(&q_empty[slot], ((seq >> 1) & 1) ^ 1, err);
+        if (lane == 0) ok = tc::mbar_wait(&q_empty[slot], ((seq >> 1) & 1) ^ 1, err, lim);
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         if (ok) {
           uint8_t* qbuf = sQ + slot * L::Q_BYTES;
+          q_last = seq;
           if (lane == 0)
             tc::mbar_arrive_expect_tx(&q_full[slot], (uint32_t)(q_boxes * L::DB * q_pos * G * 128));
           __syncwarp();
@@ -324,7 +330,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         pid0 = pid1;
         pid1 = page_of(local + 2);
         const int s = tile_i % NS;
-        if (lane == 0) ok = tc::mbar_wait(&kv_empty[s], ((tile_i / NS) & 1) ^ 1, err);
+        if (lane == 0) ok = tc::mbar_wait(&kv_empty[s], ((tile_i / NS) & 1) ^ 1, err, lim);
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         if (!ok) break;
         uint8_t* kd = sKV + s * L::STAGE;
@@ -376,11 +382,23 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       if (!ok) *s_stop = 1;
     }
+    // No copy may land after the CTA has finished: wait, with the full limit, for the
+    // last filling of every stage this warp armed (complete once the copies of all four
+    // warps have landed, whatever the consumers do; unless a wait gave up it is complete
+    // already), and warp 0 for its last two Q loads.  This comes before the sentinel
+    // below, which completes the next phase of one of these stages: a parity wait is
+    // unambiguous only while the barrier is at most one phase past it.
+    if (lane == 0) {
+      for (int j = tile_i > NS ? tile_i - NS : 0; j < tile_i; ++j)
+        tc::mbar_wait(&kv_full[j % NS], (j / NS) & 1, err);
+      for (int q = q_last > 0 ? q_last - 1 : 0; q <= q_last; ++q) tc::mbar_wait(&q_full[q & 1], (q >> 1) & 1, err);
+    }
+    __syncwarp();
     // sentinel stage: no more work
     if (!*s_stop) {
       const int s = tile_i % NS;
       bool fine = true;
-      if (lane == 0) fine = tc::mbar_wait(&kv_empty[s], ((tile_i / NS) & 1) ^ 1, err);
+      if (lane == 0) fine = tc::mbar_wait(&kv_empty[s], ((tile_i / NS) & 1) ^ 1, err, lim);
       if (lane == 0 && fine) {
         if (pw == 0) meta[s].end = 1;
         tc::mbar_arrive(&kv_full[s]);
@@ -396,15 +414,15 @@ __global__ void __launch_bounds__(THREADS, 1)
       int q_seen[2] = {-1, -1};
       for (int qk = 0;; ++qk) {
         const int s = qk % NS, b = qk & (NSB - 1);
-        if (qk >= NSB && !tc::mbar_wait(&s_free[b], ((qk / NSB) - 1) & 1, err)) break;
-        if (!tc::mbar_wait(&kv_full[s], (qk / NS) & 1, err)) break;
+        if (qk >= NSB && !tc::mbar_wait(&s_free[b], ((qk / NSB) - 1) & 1, err, lim)) break;
+        if (!tc::mbar_wait(&kv_full[s], (qk / NS) & 1, err, lim)) break;
         if (meta[s].end) {
           *end_tile = qk;
           break;
         }
         const int slot = meta[s].qslot, seq = meta[s].qseq;
         if (seq > q_seen[slot]) {
-          if (!tc::mbar_wait(&q_full[slot], (seq >> 1) & 1, err)) break;
+          if (!tc::mbar_wait(&q_full[slot], (seq >> 1) & 1, err, lim)) break;
           q_seen[slot] = seq;
         }
         tc::tc_fence_after();
@@ -445,6 +463,11 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int kk = 0; kk < PPT; ++kk)
             tc::mma_bf16_ts(tmem + L::O_COL(w), pt + kk * 8, tc::sdesc_mn128(v + kk * L::V_PAGE, 2048), idesc_pv,
                             (kk > 0 || !first) ? 1u : 0u);
+          // the low halves of P (columns TT / 2 on)
+#pragma unroll
+          for (int kk = 0; kk < PPT; ++kk)
+            tc::mma_bf16_ts(tmem + L::O_COL(w), pt + TT / 2 + kk * 8, tc::sdesc_mn128(v + kk * L::V_PAGE, 2048),
+                            idesc_pv, 1u);
           tc::mma_commit(&kv_empty[s]);
           tc::mma_commit(&s_free[pv & (NSB - 1)]);  // P read: S buffer free for tile pv + NSB
           ++pv;
@@ -453,7 +476,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint64_t t = tc::global_ns();
           if (idle_since == 0) {
             idle_since = t;
-          } else if (t - idle_since > tc::kWaitLimitNs) {
+          } else if (t - idle_since > lim) {
             flag_error(err, tc::kErrTimeout);
             ok = false;
             break;
@@ -496,13 +519,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     bool ok = true;
     for (int i = wg; ok; i += 2) {
       const int b = i & (NSB - 1);
-      ok = __all_sync(0xffffffffu, tc::mbar_wait(&s_full[b], (i / NSB) & 1, err));
+      ok = __all_sync(0xffffffffu, tc::mbar_wait(&s_full[b], (i / NSB) & 1, err, lim));
       if (!ok || i >= *end_tile) break;
       tc::tc_fence_after();
       const int s = i % NS;
       // acquire the producer's description of the tile (this phase completed long ago;
       // the stage cannot move on before this group's P.V of the tile)
-      ok = __all_sync(0xffffffffu, tc::mbar_wait(&kv_full[s], (i / NS) & 1, err));
+      ok = __all_sync(0xffffffffu, tc::mbar_wait(&kv_full[s], (i / NS) & 1, err, lim));
       if (!ok) break;
       const int c = meta[s].c, g = meta[s].g, pslot = meta[s].slot, rb = meta[s].rb;
       const int local = meta[s].local, n_tiles = meta[s].n_tiles, valid = meta[s].valid;
@@ -547,8 +570,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       // with no visible key yet (m = -inf) every s is -inf: subtract 0 so p = 0, not NaN
       const float mu = m_used == -INFINITY ? 0.f : m_used;
       float2 psum = make_float2(0.f, 0.f);
-      uint32_t pk[CW / 2];
+      uint32_t pk[CW / 2], pl[CW / 2];
       const float2 sc2 = make_float2(scale_log2, scale_log2), nm2 = make_float2(-mu, -mu);
+      const float2 neg1 = make_float2(-1.f, -1.f);
 #pragma unroll
       for (int j = 0; j < CW; j += 2) {
         // p = 2^(s scale - m): the exponents of a pair in one packed FFMA, then one ex2
@@ -556,21 +580,34 @@ __global__ void __launch_bounds__(THREADS, 1)
         const float2 e = tc::ffma2(make_float2(sv[j], sv[j + 1]), sc2, nm2);
         const float2 pp = make_float2(tc::ex2_ftz(e.x), tc::ex2_ftz(e.y));
         psum = tc::fadd2(psum, pp);
+        // p = hi + lo with hi = bf16(p) and lo = bf16(p - hi): the P.V products of both
+        // halves are exact in the fp32 accumulator, so P carries about 16 bits
         __nv_bfloat162 h2 = __floats2bfloat162_rn(pp.x, pp.y);
-        pk[j / 2] = *reinterpret_cast<uint32_t*>(&h2);
+        const uint32_t hb = *reinterpret_cast<uint32_t*>(&h2);
+        pk[j / 2] = hb;
+        const float2 hf2 = make_float2(__uint_as_float(hb << 16), __uint_as_float(hb & 0xFFFF0000u));
+        const float2 r = tc::ffma2(hf2, neg1, pp);  // p - hi, exact in fp32
+        __nv_bfloat162 l2 = __floats2bfloat162_rn(r.x, r.y);
+        pl[j / 2] = *reinterpret_cast<uint32_t*>(&l2);
       }
       float ps = psum.x + psum.y;
       if constexpr (SP) ps += __shfl_xor_sync(0xffffffffu, ps, 16);  // the row's other half
       l += ps;
-      // P over the first half of S_b (bf16 pairs: the row's keys 2c, 2c + 1 in column c)
-      if constexpr (SP) tc::tmem_st16x2_16u<TT / 4>(tmem + lane_off + L::S_COL(b), pk);
-      else tc::tmem_stu(tmem + lane_off + L::S_COL(b), pk);
+      // P over S_b (bf16 pairs: the row's keys 2c, 2c + 1 in column c): hi in the first
+      // quarter of the columns, lo in the second
+      if constexpr (SP) {
+        tc::tmem_st16x2_16u<TT / 4>(tmem + lane_off + L::S_COL(b), pk);
+        tc::tmem_st16x2_16u<TT / 4>(tmem + lane_off + L::S_COL(b) + TT / 2, pl);
+      } else {
+        tc::tmem_stu(tmem + lane_off + L::S_COL(b), pk);
+        tc::tmem_stu(tmem + lane_off + L::S_COL(b) + TT / 2, pl);
+      }
       if (__any_sync(0xffffffffu, rescale)) {
         // O_w may be rescaled only once the group's previous P.V (tile i - 2, S buffer
         // (i - 2) % NSB) has finished.  Its phase of s_free is unambiguous here: the
         // phase before it (tile i - 2 - NSB) completed before the Q.K^T of tile i - 2
         // was issued, and the one after it needs a P this group has not written yet.
-        ok = __all_sync(0xffffffffu, tc::mbar_wait(&s_free[(i - 2) & (NSB - 1)], ((i - 2) / NSB) & 1, err));
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(&s_free[(i - 2) & (NSB - 1)], ((i - 2) / NSB) & 1, err, lim));
         if (!ok) break;
         tc::tc_fence_after();
         // O_w holds this group's earlier tiles of the piece
@@ -603,7 +640,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (local >= n_tiles - 2) {
         // this group's last tile of the piece: write its partial (half of the piece)
         // this tile's P.V (same argument for the parity of s_free as above)
-        ok = __all_sync(0xffffffffu, tc::mbar_wait(&s_free[b], (i / NSB) & 1, err));
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(&s_free[b], (i / NSB) & 1, err, lim));
         if (!ok) break;
         tc::tc_fence_after();
         // half (local & 1): the piece's even or odd tiles, whichever group ran them,

@@ -138,8 +138,9 @@ struct SegWalk {
   }
 };
 
-// Waits (bounded) until *cnt >= target; the acquire load orders the reads that follow.
-__device__ __forceinline__ bool wait_count(const int* cnt, int target, int* err) {
+// Waits (bounded by limit_ns) until *cnt >= target; the acquire load orders the reads
+// that follow.
+__device__ __forceinline__ bool wait_count(const int* cnt, int target, int* err, uint64_t limit_ns) {
   auto ld = [&]() {
     int v;
     asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(cnt) : "memory");
@@ -149,7 +150,7 @@ __device__ __forceinline__ bool wait_count(const int* cnt, int target, int* err)
   const uint64_t t0 = tc::global_ns();
   while (ld() < target) {
     __nanosleep(256);
-    if (tc::global_ns() - t0 > tc::kWaitLimitNs) {
+    if (tc::global_ns() - t0 > limit_ns) {
       flag_error(err, tc::kErrTimeout);
       return false;
     }
@@ -174,7 +175,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;   // [2] accumulator b holds a finished unit
   uint64_t* acc_empty = acc_full + 2;    // [2] the epilogue has read accumulator b
-  uint32_t* tmem_slot = (uint32_t*)(acc_empty + 2);
+  uint64_t* drain = acc_empty + 2;       // every MMA of the issuer has finished
+  uint32_t* tmem_slot = (uint32_t*)(drain + 1);
   volatile int* s_last = (volatile int*)(tmem_slot + 1);  // stream-K: this segment finishes its tile
   volatile int* s_fail = s_last + 1;                      // stream-K: an epilogue wait gave up
 
@@ -183,6 +185,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int n_mt = (g.M + BM - 1) / BM;
   const int n_tiles = n_mt * ((g.N + ncols_out - 1) / ncols_out);
   const int num_k = (g.K + BK - 1) / BK;
+  const uint64_t lim = g.wait_ns ? (uint64_t)g.wait_ns : tc::kWaitLimitNs;  // pipeline waits
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -193,6 +196,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc::mbar_init(&acc_full[b], 1);
       tc::mbar_init(&acc_empty[b], 4);
     }
+    tc::mbar_init(drain, 1);
     *s_fail = 0;
     tc::fence_mbar_init();
   }
@@ -209,7 +213,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     tc::tma_prefetch_desc(&tmA);
     tc::tma_prefetch_desc(&tmB);
     if (EPI == kEpiSwiGLU) tc::tma_prefetch_desc(&tmB2);
-    int it = 0;  // stage-ring position, continued across segments
+    int it = 0;  // stage-ring position, continued across segments (= stages filled)
     bool ok = true;
     SegWalk wk(num_k, n_tiles, cut);
     int t, k_lo, k_hi;
@@ -217,7 +221,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int m0 = (t % n_mt) * BM, n0 = (t / n_mt) * ncols_out;
       for (int kt = k_lo; kt < k_hi; ++kt, ++it) {
         const int s = it % STAGES;
-        if (!(ok = tc::mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, err))) break;
+        if (!(ok = tc::mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, err, lim))) break;
         uint8_t* sa = smem + s * STAGE_BYTES;
         uint8_t* sb = sa + A_BYTES;
         tc::mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
@@ -230,6 +234,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
     }
+    // no copy may land after the CTA has finished: wait (with the full limit) for the
+    // last filling of every stage -- already complete unless a wait above gave up
+    for (int j = it > STAGES ? it - STAGES : 0; j < it; ++j) tc::mbar_wait(&full[j % STAGES], (j / STAGES) & 1, err);
   } else if (warp == 1 && lane == 0) {
     // ---------------------------------------------------------- MMA issuer
     constexpr uint32_t idesc = tc::idesc_bf16_f32(BM, BN);
@@ -240,12 +247,12 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (; ok && wk.next(t, k_lo, k_hi); ++lt) {
       const int b = lt & 1;
       // accumulator b is free once the epilogue has read the segment two back
-      if (!(ok = tc::mbar_wait(&acc_empty[b], ((lt >> 1) & 1) ^ 1, err))) break;
+      if (!(ok = tc::mbar_wait(&acc_empty[b], ((lt >> 1) & 1) ^ 1, err, lim))) break;
       tc::tc_fence_after();
       const uint32_t d = tmem + (uint32_t)(b * BN);
       for (int kt = k_lo; kt < k_hi; ++kt, ++it) {
         const int s = it % STAGES;
-        if (!(ok = tc::mbar_wait(&full[s], (it / STAGES) & 1, err))) break;
+        if (!(ok = tc::mbar_wait(&full[s], (it / STAGES) & 1, err, lim))) break;
         tc::tc_fence_after();
         const uint32_t sa = tc::smem_u32(smem + s * STAGE_BYTES);
         const uint32_t sb = sa + A_BYTES;
@@ -258,6 +265,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       tc::mma_commit(&acc_full[b]);
     }
+    // no MMA may still run (reading shared memory, writing TMEM) after the CTA finished
+    tc::mma_commit(drain);
+    tc::mbar_wait(drain, 0, err);
   } else if (warp >= 2) {
     // ---------------------------------------------------------- epilogue
     const int quarter = warp & 3;  // TMEM lanes this warp may access
@@ -265,12 +275,16 @@ __global__ void __launch_bounds__(THREADS, 1)
     int lt = 0;
     SegWalk wk(num_k, n_tiles, cut);
     int t, k_lo, k_hi;
+    // Once a wait of this warp has given up, it waits no more (`dead`) but walks the
+    // same segments and passes the same named barriers as the other epilogue warps,
+    // storing nothing; the K-cut path leaves all four warps at the same barrier.
+    bool dead = false;
     for (; wk.next(t, k_lo, k_hi); ++lt) {
       const int b = lt & 1;
       const int m0 = (t % n_mt) * BM, n0 = (t / n_mt) * ncols_out, ntile = t / n_mt;
       const int m = m0 + row;
-      const bool ok = tc::mbar_wait(&acc_full[b], (lt >> 1) & 1, err);
-      __syncwarp();
+      const bool ok = !dead && tc::mbar_wait_warp(&acc_full[b], (lt >> 1) & 1, err, lim);
+      dead = !ok;
       tc::tc_fence_after();
       const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(b * BN);
       float v[32], u2[32];
@@ -450,7 +464,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&acc_empty[b]);
-      if (!ok) break;
     }
     if (cut.zk && *s_fail == 0) {
       // stream-K (one row of tiles): the sums of the split tiles, spread over the epilogue
@@ -468,7 +481,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int kf = (int)((long)t * num_k / zk), n_seg = (int)(((long)t * num_k + num_k - 1) / zk) - kf + 1;
         if (n_seg == 1) continue;
         if (t != waited) {
-          if (!wait_count(&g.tile_cnt[t], n_seg, err)) break;
+          if (!wait_count(&g.tile_cnt[t], n_seg, err, lim)) break;
           waited = t;
         }
 #pragma unroll

@@ -44,20 +44,63 @@ void set_error(const char* fmt, ...) {
   va_end(ap);
 }
 
-// Address of the device error word on the current device (looked up once per device).
-int* device_error_word() {
-  static std::mutex mu;
-  static int* addr[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
+// The current thread's CUDA context (the driver's handle), or NULL.  Device
+// addresses of this library's static arrays are cached per context: a context that
+// is destroyed and created again (cudaDeviceReset) maps its modules afresh.
+void* current_context() {
+  using CtxGetCurrentFn = int (*)(void**);
+  static CtxGetCurrentFn fn = [] {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_hspec_device_error) != cudaSuccess) return nullptr;
-    addr[dev] = (int*)p;
-  }
-  return addr[dev];
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return (CtxGetCurrentFn) nullptr;
+    return (CtxGetCurrentFn)p;
+  }();
+  void* ctx = nullptr;
+  if (!fn || fn(&ctx) != 0) return nullptr;
+  return ctx;
 }
+
+// Device address of the static device array `symbol` in the current context, looked
+// up once per context (cudaGetSymbolAddress maps the array's module on first use and
+// allocates nothing else).  NULL with the message recorded on failure.
+void* symbol_address(const void* symbol, const char* what) {
+  struct Entry {
+    void* ctx;
+    const void* sym;
+    void* addr;
+  };
+  static std::mutex mu;
+  static std::vector<Entry> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    set_error("%s: no current CUDA device", what);
+    return nullptr;
+  }
+  void* ctx = current_context();  // NULL before the runtime has made a context current
+  std::lock_guard<std::mutex> lock(mu);
+  if (ctx)
+    for (const Entry& e : cache)
+      if (e.ctx == ctx && e.sym == symbol) return e.addr;
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, symbol);
+  if (e != cudaSuccess) {
+    if (e == cudaErrorMemoryAllocation)
+      set_error("%s: out of device memory while loading the library's static device arrays on device %d "
+                "(cudaGetSymbolAddress: %s)", what, dev, cudaGetErrorString(e));
+    else
+      set_error("%s: cudaGetSymbolAddress failed on device %d: %s", what, dev, cudaGetErrorString(e));
+    cudaGetLastError();
+    return nullptr;
+  }
+  if (!ctx) ctx = current_context();  // the lookup made the device's primary context current
+  if (ctx) cache.push_back({ctx, symbol, p});
+  return p;
+}
+
+// Address of the device error word in the current context.
+int* device_error_word() { return (int*)symbol_address((const void*)&g_hspec_device_error, "device error word"); }
 
 // ---------------------------------------------------------------- profiling
 // Event pairs recorded around kernel groups of the draft step when enabled.
@@ -157,8 +200,12 @@ hspec_status validate_cfg(const hspec_cfg* c, bool need_attn, bool need_ssm) {
     if (c->ssd_chunk < 0) FAIL(HSPEC_ERR_INVALID_ARG, "ssd_chunk must be >= 0");
   }
   if (c->norm_eps < 0.f) FAIL(HSPEC_ERR_INVALID_ARG, "norm_eps must be >= 0");
+  if (c->wait_limit_ns < 0) FAIL(HSPEC_ERR_INVALID_ARG, "wait_limit_ns must be >= 0");
   return HSPEC_OK;
 }
+
+// The kernels' pipeline wait limit (0 passes the kernels' default).
+unsigned long long wait_ns(const hspec_cfg* c) { return (unsigned long long)c->wait_limit_ns; }
 
 int ssd_chunk_len(const hspec_cfg* c, int K) { return (c->ssd_chunk > 0 && c->ssd_chunk < K) ? c->ssd_chunk : K; }
 
@@ -225,6 +272,7 @@ AttnArgs attn_args(const hspec_cfg* c, const AttnPlan& p, const hspec_kv_view* k
   a.ws_ml = a.ws_acc + p.rows * a.D;
   a.sched = (int*)(a.ws_ml + p.rows * 2);
   a.err = device_error_word();
+  a.wait_ns = wait_ns(c);
   return a;
 }
 
@@ -403,6 +451,7 @@ hspec_status hspec_inject_state(const hspec_cfg* cfg, const void* W_inj, const v
   if (HPN > (1L << 31) - 1) FAIL(HSPEC_ERR_UNSUPPORTED, "H*P*N too large");
   GemmArgs g = gemm_args(C, (int)HPN, cfg->d_model, h_last, cfg->d_model, W_inj, cfg->d_model, h0, HPN);
   g.out_f32 = true;
+  g.wait_ns = wait_ns(cfg);
   if (!gemm(cfg->dtype, kEpiStore, g, (cudaStream_t)stream)) return HSPEC_ERR_UNSUPPORTED;
   return check_launch("hspec_inject_state");
 }
@@ -423,44 +472,17 @@ hspec_status hspec_ssd_block_scan(const hspec_cfg* cfg, const void* x, const flo
   a.A = A, a.D = D;
   a.B = B, a.Cm = Cm, a.bc_rs = a.N;
   a.h0 = h0, a.y = y, a.y_rs = (long)a.H * a.P, a.hK = hK;
+  a.wait_ns = wait_ns(cfg);
   ssd_scan(cfg->dtype, a, (cudaStream_t)stream);
   return check_launch("hspec_ssd_block_scan");
 }
 
 }  // extern "C"
 
-// Scratch of hspec_attn_paged_block_noalloc: a fixed device array, so that callers
-// that cannot allocate still get the split-KV partials somewhere.  Host code must not
-// pass the symbol itself to a kernel (on the host it names a shadow, not device
-// memory); the device address is looked up once per device below.
-static __device__ __align__(256) unsigned char g_noalloc_scratch[HSPEC_NOALLOC_SCRATCH_BYTES];
-
-namespace {
-
-// Device address of g_noalloc_scratch on the current device; NULL (message recorded)
-// if the lookup fails.  The first call on a device does the lookup.
-void* noalloc_scratch_address() {
-  static std::mutex mu;
-  static void* addr[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
-    set_error("no current CUDA device");
-    return nullptr;
-  }
-  std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
-    void* p = nullptr;
-    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess) {
-      set_error("cudaGetSymbolAddress(scratch) failed: %s", cudaGetErrorString(e));
-      return nullptr;
-    }
-    addr[dev] = p;
-  }
-  return addr[dev];
-}
-
-}  // namespace
+namespace hspec {
+// Device address of the allocation-free attention's static scratch (noalloc.cu).
+void* noalloc_scratch_address();
+}  // namespace hspec
 
 extern "C" {
 
@@ -652,6 +674,7 @@ hspec_status hspec_draft_step(hspec_drafter* dr, const hspec_step_in* in, const 
   // the projection and MLP GEMMs may split K over the step workspace
   int site = 0;  // the K-cut GEMM calls take the counter slices in turn
   auto split = [&](GemmArgs ga) {
+    ga.wait_ns = wait_ns(c);
     ga.part = (float*)(ws + sp.gpart);
     ga.tile_cnt = site < sp.gcnt_sites ? (int*)(ws + sp.gcnt) + (size_t)site * sp.gmax_tiles : nullptr;
     ++site;
@@ -686,6 +709,7 @@ hspec_status hspec_draft_step(hspec_drafter* dr, const hspec_step_in* in, const 
       a.A = L.A, a.D = L.D;
       a.B = big + (size_t)(2 * HP) * E, a.Cm = big + (size_t)(2 * HP + N) * E, a.bc_rs = n_in;
       a.y = y, a.y_rs = HP, a.hK = nullptr;
+      a.wait_ns = wait_ns(c);
       if (step_fuses_inject(c)) {
         // y = the scan from a zero state (in-block terms, D x), then the injection GEMM
         // adds exp(cum_t) C_t . h0 from its accumulator: h0 = W_inj h_last is never stored
@@ -699,6 +723,7 @@ hspec_status hspec_draft_step(hspec_drafter* dr, const hspec_step_in* in, const 
         gi.ssd.Cm = a.Cm, gi.ssd.c_rs = n_in;
         gi.ssd.dt_raw = a.dt, gi.ssd.dt_rs = n_in, gi.ssd.dt_bias = L.dt_bias, gi.ssd.A = L.A;
         gi.ssd.y = y, gi.ssd.y_rs = HP;
+        gi.wait_ns = wait_ns(c);
         {
           ProfScope p("inject", s);
           if (!gemm(dtype, kEpiSsdRead, gi, s)) return HSPEC_ERR_UNSUPPORTED;
@@ -707,6 +732,7 @@ hspec_status hspec_draft_step(hspec_drafter* dr, const hspec_step_in* in, const 
         // injected initial state h0 = W_inj h_last, stored, then the scan from it
         GemmArgs gi = gemm_args(C, (int)HPN, d, in->h_last, d, L.W_inj, d, h0, HPN);
         gi.out_f32 = true;
+        gi.wait_ns = wait_ns(c);
         {
           ProfScope p("inject", s);
           if (!gemm(dtype, kEpiStore, gi, s)) return HSPEC_ERR_UNSUPPORTED;
@@ -786,6 +812,7 @@ hspec_status hspec_draft_step(hspec_drafter* dr, const hspec_step_in* in, const 
     ga.pval = (float*)(ws + sp.pval);
     ga.pidx = (int32_t*)(ws + sp.pidx);
     ga.n_parts = sp.n_parts;
+    ga.wait_ns = wait_ns(c);
     {
       ProfScope p("lm_head_argmax", s);
       if (!gemm(dtype, kEpiArgmax, ga, s)) return HSPEC_ERR_UNSUPPORTED;

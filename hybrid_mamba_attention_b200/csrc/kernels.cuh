@@ -69,6 +69,7 @@ struct GemmArgs {
   // epilogue, so the result does not depend on scheduling.
   float* part; int* tile_cnt; size_t part_bytes; int max_tiles;
   SsdReadArgs ssd;             // kEpiSsdRead
+  unsigned long long wait_ns;  // pipeline waits give up after this long (0: the default)
 };
 // Workspace bytes (partials) that gemm() needs for this shape when it cuts the K loop
 // (stream-K or split-K; 0 for whole tiles); counters: gemm_tile_count().
@@ -91,6 +92,7 @@ struct SsdArgs {
   const float* h0;             // [C,H,P,N] or NULL
   float* y; long y_rs;         // fp32, token row stride (head h at column h*P)
   float* hK;                   // [C,H,P,N] or NULL
+  unsigned long long wait_ns;  // pipeline waits give up after this long (0: the default)
 };
 size_t ssd_smem_bytes(int P, int N, int Q);
 void ssd_scan(int dtype, const SsdArgs& a, cudaStream_t s);
@@ -128,6 +130,7 @@ struct AttnArgs {
   // written by the schedule kernel; from [64] the tile offsets of the requests (C + 1)
   int* sched;
   int* err;
+  unsigned long long wait_ns;            // pipeline waits give up after this long (0: the default)
 };
 // Split policy (tokens per split, splits per request) and workspace bytes.
 int attn_split_tokens(int dtype, int C, int Hkv, int K, int max_ctx, int requested);

@@ -155,6 +155,7 @@ __global__ void __launch_bounds__(THREADS, 1) ssd_tc_kernel(const __grid_constan
   int* err = t.err;
   const int i0 = (int)((long)blockIdx.x * t.n_items / gridDim.x);
   const int i1 = (int)((long)(blockIdx.x + 1) * t.n_items / gridDim.x);
+  const uint64_t lim = a.wait_ns ? (uint64_t)a.wait_ns : tc::kWaitLimitNs;  // pipeline waits
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NSTAGE; ++s) {
@@ -183,15 +184,20 @@ __global__ void __launch_bounds__(THREADS, 1) ssd_tc_kernel(const __grid_constan
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       tc::tma_prefetch_desc(&h0_map);
-      for (int i = i0; i < i1; ++i) {
+      int filled = 0;
+      for (int i = i0; i < i1; ++i, ++filled) {
         const int k = i - i0, st = k % NSTAGE;
-        if (!tc::mbar_wait(&a_empty[st], ((k / NSTAGE) & 1) ^ 1, err)) break;
+        if (!tc::mbar_wait(&a_empty[st], ((k / NSTAGE) & 1) ^ 1, err, lim)) break;
         const int c = i / t.n_tiles, j = i % t.n_tiles;
         const int row0 = (c * a.H + j * hpt) * P;
         tc::mbar_arrive_expect_tx(&a_full[st], (uint32_t)(nblk * ROWS * 128));
         for (int b = 0; b < nblk; ++b)
           tc::tma_load_2d(sA + st * TILE_BYTES + b * ROWS * 128, &h0_map, &a_full[st], b * 32, row0);
       }
+      // no copy may land after the CTA has finished: wait (with the full limit) for the
+      // last filling of every stage -- already complete unless a wait gave up
+      for (int k = filled > NSTAGE ? filled - NSTAGE : 0; k < filled; ++k)
+        tc::mbar_wait(&a_full[k % NSTAGE], (k / NSTAGE) & 1, err);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -201,8 +207,8 @@ __global__ void __launch_bounds__(THREADS, 1) ssd_tc_kernel(const __grid_constan
       for (int i = i0; i < i1; ++i) {
         const int k = i - i0, st = k % NSTAGE, db = k & 1;
         // accumulator db is free once the epilogue of tile k - 2 has read it
-        if (k >= 2 && !tc::mbar_wait(&d_free[db], ((k >> 1) - 1) & 1, err)) break;
-        if (!tc::mbar_wait(&lo_full[k & 1], (k >> 1) & 1, err)) break;
+        if (k >= 2 && !tc::mbar_wait(&d_free[db], ((k >> 1) - 1) & 1, err, lim)) break;
+        if (!tc::mbar_wait(&lo_full[k & 1], (k >> 1) & 1, err, lim)) break;
         tc::tc_fence_after();
         const uint32_t hi = tc::smem_u32(sA + st * TILE_BYTES);
         const uint32_t lo = tmem + (uint32_t)(128 * (k & 1));
@@ -272,8 +278,8 @@ __global__ void __launch_bounds__(THREADS, 1) ssd_tc_kernel(const __grid_constan
       }
       // the state tile has landed; for a new request also the MMAs of the previous tile
       // (the last reader of the C^T operand) are done
-      bool ok = tc::mbar_wait(&a_full[st], (k / NSTAGE) & 1, err);
-      if (ok && new_req && k >= 1) ok = tc::mbar_wait(&acc_full[(k - 1) & 1], ((k - 1) >> 1) & 1, err);
+      bool ok = tc::mbar_wait_warp(&a_full[st], (k / NSTAGE) & 1, err, lim);
+      if (ok && new_req && k >= 1) ok = tc::mbar_wait_warp(&acc_full[(k - 1) & 1], ((k - 1) >> 1) & 1, err, lim);
       if (!ok) *s_fail = 1;
       gsync();
       if (*s_fail) break;
@@ -398,10 +404,10 @@ __global__ void __launch_bounds__(THREADS, 1) ssd_tc_kernel(const __grid_constan
 
       // epilogue, once the tile's MMAs are done:
       // y_t = exp(cum_t) (C S^T)_t + sum_{s<=t} L_ts x_s + D_h x_t
-      ok = tc::mbar_wait(&acc_full[g], (k >> 1) & 1, err);
+      ok = tc::mbar_wait_warp(&acc_full[g], (k >> 1) & 1, err, lim);
       if (!ok) {
         *s_fail = 1;
-        continue;  // the group leaves after its next barrier
+        continue;  // the group (the whole warp: the wait's answer is warp-uniform) leaves after its next barrier
       }
       tc::tc_fence_after();
       float dv[NT];

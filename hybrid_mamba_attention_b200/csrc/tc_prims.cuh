@@ -14,8 +14,11 @@ namespace tc {
 
 // Device error bit for a wait that gave up (a pipeline that never completes).
 constexpr int kErrTimeout = 8;
-// A wait gives up after this many nanoseconds of the global timer (far above any
-// legitimate wait of these kernels, which run for well under a millisecond).
+// By default a wait gives up after this many nanoseconds of the global timer (far
+// above any legitimate wait of these kernels, which run for well under a
+// millisecond); a call may set a shorter limit for its pipeline waits
+// (hspec_cfg.wait_limit_ns).  The drains before a CTA exits -- waits for its own
+// copies and MMAs in flight -- always use this one.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -99,17 +102,27 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase of `parity` to complete; gives up (returns false and sets
-// kErrTimeout) after kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err) {
+// kErrTimeout) after limit_ns.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (global_ns() - t0 > kWaitLimitNs) {
+    if (global_ns() - t0 > limit_ns) {
       flag_error(err, kErrTimeout);
       return false;
     }
   }
+}
+
+// The same wait for a whole (converged) warp: lane 0 waits and every lane gets its
+// answer, so the result is the same in all lanes and warp-collective instructions
+// after it stay converged.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, int* err, uint64_t limit_ns) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, err, limit_ns);
+  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
 // 2-D tiled TMA load of box (x = inner coordinate, y = row) into shared memory,

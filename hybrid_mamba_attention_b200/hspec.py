@@ -57,7 +57,7 @@ class hspec_cfg(ct.Structure):
                 ("n_layers", ct.c_int), ("layer_kinds", ct.c_char * HSPEC_MAX_LAYERS),
                 ("dtype", ct.c_int), ("flags", ct.c_int), ("rope_theta", ct.c_float),
                 ("norm_eps", ct.c_float), ("ssd_chunk", ct.c_int), ("attn_split_tokens", ct.c_int),
-                ("draft_vocab", ct.c_int)]
+                ("draft_vocab", ct.c_int), ("wait_limit_ns", ct.c_longlong)]
 
 
 class hspec_layer_weights(ct.Structure):
@@ -148,7 +148,8 @@ def _stream(stream):
 
 # --------------------------------------------------------------- config helpers
 
-def make_cfg(shapes, ssd_chunk: int = 0, attn_split_tokens: int = 0, fuse_inject: bool = False) -> hspec_cfg:
+def make_cfg(shapes, ssd_chunk: int = 0, attn_split_tokens: int = 0, fuse_inject: bool = False,
+             wait_limit_ns: int = 0) -> hspec_cfg:
     """hspec_cfg from an inputs.Shapes (or any object with the same fields)."""
     sh = shapes
     flags = (HSPEC_FLAG_ROPE if sh.use_rope else 0) | (HSPEC_FLAG_GATE if sh.use_gate else 0) | (
@@ -158,7 +159,8 @@ def make_cfg(shapes, ssd_chunk: int = 0, attn_split_tokens: int = 0, fuse_inject
                      n_layers=len(sh.layers), layer_kinds=sh.layers.encode(),
                      dtype=HSPEC_DTYPE_F32 if sh.dtype == "f32" else HSPEC_DTYPE_BF16, flags=flags,
                      rope_theta=sh.rope_theta, norm_eps=sh.eps, ssd_chunk=ssd_chunk,
-                     attn_split_tokens=attn_split_tokens, draft_vocab=getattr(sh, "draft_vocab", 0))
+                     attn_split_tokens=attn_split_tokens, draft_vocab=getattr(sh, "draft_vocab", 0),
+                     wait_limit_ns=wait_limit_ns)
 
 
 def kv_view(cache: dict) -> hspec_kv_view:
@@ -290,9 +292,9 @@ class Drafter:
     """Holds a drafter handle plus the weights it points at (kept alive here)."""
 
     def __init__(self, shapes, weights: dict, ssd_chunk: int = 0, attn_split_tokens: int = 0,
-                 fuse_inject: bool = False):
+                 fuse_inject: bool = False, wait_limit_ns: int = 0):
         self.shapes = shapes
-        self.cfg = make_cfg(shapes, ssd_chunk, attn_split_tokens, fuse_inject)
+        self.cfg = make_cfg(shapes, ssd_chunk, attn_split_tokens, fuse_inject, wait_limit_ns)
         self.weights = weights
         mw = hspec_model_weights()
         for i, w in enumerate(weights["layers"]):

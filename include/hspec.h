@@ -96,6 +96,13 @@ typedef struct hspec_cfg {
                                        most 2048 chunks) -- auto: one chunk per SM */
   int draft_vocab;                  /* reduced draft head rows (0 = the full vocab head):    */
                                     /* logits over W_lm_draft, draft token = the mapped id  */
+  long long wait_limit_ns;          /* a pipeline wait in a tensor-core kernel (an mbarrier
+                                       or a tile counter) gives up after this many ns of the
+                                       GPU's global timer, skips the rest of its work and
+                                       sets bit 8 of the device error word (see
+                                       hspec_sync_status); the kernel still waits for its own
+                                       copies and MMAs in flight before it exits.  0 = 2 s,
+                                       far above any legitimate wait; >= 0 */
 } hspec_cfg;
 
 /* Weights of one layer (caller-owned device memory; fields of the other layer kind
@@ -195,13 +202,21 @@ HSPEC_API hspec_status hspec_attn_paged_block(const hspec_cfg* cfg, const void* 
  * library and has no device allocator of its own to provide a workspace.  This entry
  * point takes the same inputs and output as hspec_attn_paged_block but keeps its
  * split-KV partials in a static device array of HSPEC_NOALLOC_SCRATCH_BYTES bytes
- * inside the library; every GPU that loads the library holds that array until the
- * process exits.
+ * inside the library.
+ *  - When the array's memory is taken: the array sits in a module of its own, which
+ *    CUDA loads (and so reserves HSPEC_NOALLOC_SCRATCH_BYTES on that device) at the
+ *    first call of this entry point on each device under lazy module loading, CUDA's
+ *    default, or when the context is created under CUDA_MODULE_LOADING=EAGER.  It
+ *    stays reserved until the context is destroyed.  A caller that hands nearly all
+ *    HBM to a KV pool should make one small call per device before sizing the pool
+ *    (or load modules eagerly); otherwise that first call may find no room and return
+ *    HSPEC_ERR_CUDA with an out-of-memory message.
  *  - Calls whose partials need more than HSPEC_NOALLOC_SCRATCH_BYTES (that is,
  *    hspec_attn_workspace_size(cfg, C, K, kv->max_pages) is larger) are rejected
  *    with HSPEC_ERR_WORKSPACE before anything is launched.
- *  - The first call on each device looks up the array's device address (a runtime
- *    call, no allocation); make that first call before any CUDA stream capture.
+ *  - The first call in each CUDA context looks up the array's device address (a
+ *    runtime call that maps the module and allocates nothing else); make that first
+ *    call before any CUDA stream capture.
  *  - All calls share the one array, which keeps the previous call's contents.
  *    Nothing in it has to start at zero: each call writes every partial it later
  *    reads.  Calls that overlap on the GPU (different streams, or different host

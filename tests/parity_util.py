@@ -48,18 +48,52 @@ def half_ulp_bf16(x):
 
 
 def assert_close_stored_bf16(gpu, ref, what: str = ""):
-    """A bf16-stored GPU output against the oracle's exact value: the kernel's own
-    error, max(|gpu - ref| - half_ulp_bf16(ref), 0) / rms(ref), must meet the bf16
-    bound; the raw max-abs / rms (which includes the store's rounding) is returned
-    alongside."""
+    """A bf16-stored GPU output against the oracle's exact (unrounded) value: the
+    raw max|gpu - ref| / rms(ref), which includes the store's own rounding, must meet
+    the bf16 bound.  Returns (raw, kernel error without that rounding) and prints both."""
     g = np.asarray(gpu, dtype=np.float64)
     r = np.asarray(ref, dtype=np.float64)
     assert np.isfinite(g).all(), f"{what}: non-finite GPU output"
     rms = max(np.sqrt((r ** 2).mean()), 1e-300)
     raw = float(np.abs(g - r).max() / rms)
     kern = float(np.maximum(np.abs(g - r) - half_ulp_bf16(r), 0.0).max() / rms)
-    assert kern <= BF16_TOL, f"{what}: bf16 kernel error {kern:.3e} (raw {raw:.3e}) > {BF16_TOL}"
-    return kern, raw
+    print(f"{what}: bf16 stored output max-abs/rms {raw:.3e} (without the store's half ulp {kern:.3e})")
+    assert raw <= BF16_TOL, f"{what}: bf16 max-abs/rms(ref) = {raw:.3e} > {BF16_TOL} (kernel part {kern:.3e})"
+    return raw, kern
+
+
+def storage_floor_bf16(ref) -> float:
+    """max|bf16(ref) - ref| / rms(ref): what storing the exact answer in bf16 already
+    costs, before any arithmetic error."""
+    r = np.asarray(ref, dtype=np.float64)
+    rb = torch.from_numpy(np.ascontiguousarray(r)).to(torch.bfloat16).to(torch.float64).numpy()
+    return float(np.abs(rb - r).max() / max(np.sqrt((r ** 2).mean()), 1e-300))
+
+
+# Edge-shape batches that mix near-empty and long contexts have outputs with
+# max|o| / rms(o) of 8-13, so bf16 storage of the exact answer alone reaches 1.7-2.9e-2
+# of rms there.  For those the kernel's own error (beyond the half ulp the store may
+# add) is held to KERNEL_TOL, twenty times below the bf16 bound, and the raw error to
+# at most one ulp of storage at the largest elements.
+KERNEL_TOL = 1e-3
+
+
+def assert_close_stored_bf16_edge(gpu, ref, what: str = ""):
+    """A bf16-stored output of an edge-shape batch against the oracle's exact value:
+    the kernel's error without the store's half ulp <= KERNEL_TOL, and the raw
+    max-abs / rms <= max(bf16 bound, twice the storage floor).  Prints raw, floor and
+    kernel error; returns them."""
+    g = np.asarray(gpu, dtype=np.float64)
+    r = np.asarray(ref, dtype=np.float64)
+    assert np.isfinite(g).all(), f"{what}: non-finite GPU output"
+    rms = max(np.sqrt((r ** 2).mean()), 1e-300)
+    raw = float(np.abs(g - r).max() / rms)
+    kern = float(np.maximum(np.abs(g - r) - half_ulp_bf16(r), 0.0).max() / rms)
+    floor = storage_floor_bf16(r)
+    print(f"{what}: bf16 stored output max-abs/rms {raw:.3e}, storage floor {floor:.3e}, kernel {kern:.3e}")
+    assert kern <= KERNEL_TOL, f"{what}: kernel error {kern:.3e} > {KERNEL_TOL} (raw {raw:.3e})"
+    assert raw <= max(BF16_TOL, 2 * floor), f"{what}: raw {raw:.3e} beyond one storage ulp (floor {floor:.3e})"
+    return raw, floor, kern
 
 
 def host(t):

@@ -34,7 +34,7 @@ def test_library_exports_every_declared_function(H):
 
 def test_struct_layouts_match_header(H, tmp_path):
     prog = tmp_path / "sz.c"
-    fields = {"hspec_cfg": ["d_model", "layer_kinds", "dtype", "rope_theta", "attn_split_tokens", "draft_vocab"],
+    fields = {"hspec_cfg": ["d_model", "layer_kinds", "dtype", "rope_theta", "attn_split_tokens", "draft_vocab", "wait_limit_ns"],
               "hspec_step_in": ["C", "h_last", "ctx_lens", "kv"],
               "hspec_kv_view": ["v_pool", "num_pages", "page_table", "max_pages"],
               "hspec_model_weights": ["layers", "final_norm", "W_lm", "W_lm_draft", "draft_to_target"],
@@ -93,6 +93,9 @@ def test_bad_config_rejected(H):
     assert st == H.HSPEC_ERR_SHAPE_MISMATCH
     cfg = small_cfg(H, flags=64)
     assert H._lib.hspec_inject_state(ct.byref(cfg), 16, 16, 1, 16, None) == H.HSPEC_ERR_INVALID_ARG
+    cfg = small_cfg(H, wait_limit_ns=-1)
+    assert H._lib.hspec_inject_state(ct.byref(cfg), 16, 16, 1, 16, None) == H.HSPEC_ERR_INVALID_ARG
+    assert "wait_limit_ns" in H.hspec_last_error()
 
 
 def test_unsupported_block_size_rejected(H):

@@ -14,7 +14,8 @@ import torch
 
 import oracle
 from hybrid_mamba_attention_b200 import inputs as I
-from tests.parity_util import (BF16_TOL, assert_close, assert_close_stored_bf16, half_ulp_bf16, host, rel_max, rel_rms,
+from tests.parity_util import (BF16_TOL, assert_close, assert_close_stored_bf16, assert_close_stored_bf16_edge,
+                               half_ulp_bf16, host, rel_max, rel_rms,
                                sample_requests, sub_cache, to_np)
 
 pytestmark = pytest.mark.gpu
@@ -154,12 +155,15 @@ def oracle_attn(inp, rows, causal=False):
                              causal_block=causal)
 
 
-def compare_attn(gpu, ref, sh, what):
+def compare_attn(gpu, ref, sh, what, edge=False):
     # The attention output is stored in bf16.  It is compared with the oracle's exact
-    # value, less the half ulp that the bf16 store itself may add: with max|o|/rms(o)
-    # near 5 (32k-token contexts) that rounding alone reaches ~2% of rms(o), and
-    # comparing with a bf16-rounded oracle would count one-ulp rounding flips instead.
+    # value, so the store's own rounding is part of the measured error (comparing with
+    # a bf16-rounded oracle would count one-ulp rounding flips instead).  The seeded
+    # workloads are held to the bf16 bound; edge-shape batches, whose storage alone
+    # can miss it, to a kernel error twenty times below it (parity_util).
     if sh.dtype == "bf16":
+        if edge:
+            return assert_close_stored_bf16_edge(gpu, ref, what)
         return assert_close_stored_bf16(gpu, ref, what)
     return assert_close(gpu, ref, sh.dtype, what)
 
@@ -183,7 +187,7 @@ def test_paged_attention_causal_block(H, cuda):
     out = run_attn(H, sh, inp, 16, causal=True)
     assert H.hspec_sync_status() == 0
     rows = list(range(len(lens)))
-    compare_attn(to_np(out), oracle_attn(inp, rows, causal=True), sh, "attn causal")
+    compare_attn(to_np(out), oracle_attn(inp, rows, causal=True), sh, "attn causal", edge=True)
 
 
 def test_page_placement_is_invisible(H, cuda):
@@ -215,7 +219,7 @@ def test_split_count_does_not_change_the_result(H, cuda):
     for split in (16, 64, 1024, 16384):
         out = run_attn(H, sh, inp, wl.K, split=split)
         assert H.hspec_sync_status() == 0
-        compare_attn(to_np(out[rows]), ref, sh, f"attn split {split}")
+        compare_attn(to_np(out[rows]), ref, sh, f"attn split {split}", edge=True)
 
 
 @pytest.mark.parametrize("name,split", [("qwen_c128", 0), ("llama_c32", 64), ("llama_c32", 0)])
@@ -246,7 +250,7 @@ def test_attention_few_requests_long_contexts(H, cuda, C):
     assert H.hspec_sync_status() == 0, H.hspec_last_error()
     assert torch.equal(out, again)
     rows = sample_requests(C, 2, seed=5)
-    compare_attn(to_np(out[rows]), oracle_attn(inp, rows), sh, f"attn C={C}")
+    compare_attn(to_np(out[rows]), oracle_attn(inp, rows), sh, f"attn C={C}", edge=True)
 
 
 def test_request_order_permutes_output(H, cuda):
@@ -318,7 +322,7 @@ def test_bf16_attention_ragged_tiles(H, cuda, K, lens):
     inp = I.make_attn_inputs(sh, lens_t, K, 21, cuda)
     out = run_attn(H, sh, inp, K)
     assert H.hspec_sync_status() == 0
-    compare_attn(to_np(out), oracle_attn(inp, list(range(len(lens)))), sh, f"attn K={K}")
+    compare_attn(to_np(out), oracle_attn(inp, list(range(len(lens)))), sh, f"attn K={K}", edge=True)
 
 
 def test_bf16_attention_more_than_128_query_rows(H, cuda):
@@ -328,7 +332,7 @@ def test_bf16_attention_more_than_128_query_rows(H, cuda):
     inp = I.make_attn_inputs(sh, lens, 32, 22, cuda)
     out = run_attn(H, sh, inp, 32)
     assert H.hspec_sync_status() == 0
-    compare_attn(to_np(out), oracle_attn(inp, [0, 1]), sh, "attn 256 rows")
+    compare_attn(to_np(out), oracle_attn(inp, [0, 1]), sh, "attn 256 rows", edge=True)
 
 
 @pytest.mark.parametrize("K", [33, 40, 64])
@@ -340,7 +344,7 @@ def test_bf16_attention_block_keys_span_two_tiles(H, cuda, K):
     for causal in (False, True):
         out = run_attn(H, sh, inp, K, causal=causal)
         assert H.hspec_sync_status() == 0
-        compare_attn(to_np(out), oracle_attn(inp, [0, 1, 2], causal=causal), sh, f"attn K={K} causal={causal}")
+        compare_attn(to_np(out), oracle_attn(inp, [0, 1, 2], causal=causal), sh, f"attn K={K} causal={causal}", edge=True)
 
 
 def test_bf16_attention_head_dim_64(H, cuda):
@@ -350,7 +354,7 @@ def test_bf16_attention_head_dim_64(H, cuda):
     for causal in (False, True):
         out = run_attn(H, sh, inp, 8, causal=causal)
         assert H.hspec_sync_status() == 0
-        compare_attn(to_np(out), oracle_attn(inp, [0, 1, 2], causal=causal), sh, f"attn D=64 causal={causal}")
+        compare_attn(to_np(out), oracle_attn(inp, [0, 1, 2], causal=causal), sh, f"attn D=64 causal={causal}", edge=True)
 
 
 def test_bf16_bad_page_id_is_reported(H, cuda):

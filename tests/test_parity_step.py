@@ -9,13 +9,15 @@ Two views:
               final RMSNorm and the LM-head argmax likewise (tokens must agree
               wherever the oracle's top-2 logit gap is >= 1e-3).
   end to end  the GPU step vs the oracle step from the block input.  For the
-              two-layer workloads this meets the 2e-2 bound.  Through four bf16
-              layers with SwiGLU, one-ulp rounding differences at the bf16 storage
-              points cascade through the dense projections (fp32 vs fp64
+              two-layer workloads this meets the 2e-2 bound.  The four-layer bf16
+              step with SwiGLU does not: one-ulp rounding differences at the bf16
+              storage points cascade through the dense projections (fp32 vs fp64
               accumulation decides a few roundings differently, each of which moves
-              whole rows at the next rounding point), so the end-to-end difference
-              is a drift that any fp32 implementation shows against an fp64
-              reference; it is asserted against DRIFT_BOUND and printed.
+              whole rows at the next rounding point).  A CPU emulation of fp32
+              arithmetic with the same storage points puts that drift at 1.5-1.9e-2
+              for any fp32 implementation against the fp64 oracle; on the GPU it
+              measured 1.8-2.6e-2.  It is printed and asserted against DRIFT_BOUND,
+              3e-2, just above the largest measured value.
 
 H-Spec (arXiv 2609.24197) Abstract: block-parallel drafting with attention over the
 target KV in place and Mamba-2 layers started from the projected last-token hidden
@@ -35,7 +37,7 @@ from tests.parity_util import (BF16_TOL, assert_close, assert_close_stored_bf16,
 pytestmark = pytest.mark.gpu
 
 GAP = 1e-3
-DRIFT_BOUND = 6e-2  # end-to-end bound for the four-layer bf16 step (see module docstring)
+DRIFT_BOUND = 3e-2  # end-to-end bound for the four-layer bf16 step (see module docstring)
 
 
 @pytest.fixture(scope="module")
@@ -205,6 +207,23 @@ def test_stream_k_step_repeats_bitwise(H, cuda, C):
         b = run_step(H, wl, st, layers=False)
         assert torch.equal(a["hidden"], b["hidden"])
         assert torch.equal(a["tokens"], b["tokens"])
+
+
+@pytest.mark.parametrize("C,K", [(1, 16), (8, 16), (32, 16), (1, 32), (8, 32), (32, 32)])
+def test_fused_injection_step_matches_oracle(H, cuda, C, K):
+    # HSPEC_FLAG_FUSE_INJECT: h0 = W_inj h_last is never stored; the injection GEMM adds
+    # exp(cum_t) C_t . h0 to the zero-state scan from its accumulator.  Every layer is
+    # held to the bf16 bound against the oracle run from the GPU's own input to it (the
+    # oracle runs the plain sequential recurrence from the stored h0), and the whole
+    # step to the drift bound.  H-Spec Abstract: Mamba modules start from projected
+    # last-token target hidden states.
+    wl = I.full_workload(C, K)
+    st = I.make_step_inputs(wl, cuda)
+    out = run_step(H, wl, st, fuse_inject=True)
+    rows = sample_requests(wl.C, 2, seed=wl.seed)
+    wh = host_weights(st["weights"])
+    check_stagewise(wl, st, out, rows, wh)
+    check_end_to_end(wl, st, out, rows, wh, DRIFT_BOUND)
 
 
 @pytest.mark.parametrize("C,K", [(1, 16), (8, 16), (32, 32)])

@@ -6,7 +6,9 @@ no device allocator of its own -- so hspec_attn_paged_block_noalloc keeps its
 split-KV partials in a static device array inside the library instead of a
 caller-provided workspace.  These tests call it through the C-ABI twice in a row
 (different inputs, so a stale scratch would show) and compare it with
-hspec_attn_paged_block on the same inputs, within the tolerance the parity tests use.
+hspec_attn_paged_block on the same inputs.  Both run the same kernels on the same
+batch, and repeated calls on one batch are bit-identical, so the two outputs must be
+equal bit for bit (a stale partial that moved a few ulps would fail).
 This file is collected last so that a failure here cannot hide any other test's
 result; it passes alone in a fresh process as well as after the other tests.
 """
@@ -16,7 +18,6 @@ import pytest
 import torch
 
 from hybrid_mamba_attention_b200 import inputs as I
-from tests.parity_util import assert_close, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -59,7 +60,8 @@ def test_noalloc_attention_matches_workspace_attention_twice(H, cuda, name):
         assert H.hspec_sync_status() == 0, H.hspec_last_error()
         want = with_workspace(H, cfg, inp, wl.K)
         assert H.hspec_sync_status() == 0
-        assert_close(to_np(got), to_np(want), sh.dtype, f"noalloc vs workspace, call {call}")
+        assert torch.equal(got, want), f"noalloc vs workspace differ on call {call}"
+        assert torch.isfinite(got.float()).all()
 
 
 def test_noalloc_attention_rejects_oversized_calls(H, cuda):
