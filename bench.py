@@ -2,7 +2,8 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl hspec|reference]
                     [--C 128] [--K 16] [--sweep] [--draft-vocab V] [--no-cpu-baseline]
-                    [--kernel step|attn|inject|ssd|verify|gemm] [--workload NAME]
+                    [--no-attention-configs] [--kernel step|attn|inject|ssd|verify|gemm]
+                    [--workload NAME]
 
 One step = one hspec_draft_step over a batch of C requests of the 4-layer M,A,M,A
 drafter on Llama-3-8B shapes (SwiGLU 16384, shared 128256-token LM head), K block
@@ -17,6 +18,9 @@ time is the max over ranks.
 
 --impl reference times the CPU oracle on the same config and metric (rank 0 only).
 --kernel times one kernel-level call on a named workload instead of the step.
+The step line also carries, per concurrency point, the per-kernel-group times and
+roofline fractions, and the paged attention timed alone on the Llama-3-8B C=32 and
+Qwen-32B C=128 workloads (attention_configs).
 """
 from __future__ import annotations
 
@@ -226,11 +230,12 @@ def step_roofline_ms(sh, C, K, ctx_lens, peaks):
 
 # DRAM bytes (read + write) per algorithmic byte of the paged-attention kernel, from
 # one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum) of the current
-# attn_tc_kernel at Llama-3-8B shapes, C=32, ctx U[512,8192] (677.2 MB for 656.2 MB of
-# K/V; the excess is the partials of the pieces).  The step's attention launch is too large
-# to capture; its traffic is this ratio times its algorithmic bytes (traffic grows
-# with the K/V read).  Set to None whenever the kernel changes until re-captured.
-ATTN_TRAFFIC_PER_BYTE = 1.0320
+# attn_tc_kernel at Llama-3-8B shapes, C=32, ctx U[512,8192]: 678.4 MB for 658.3 MB of
+# algorithmic bytes as step_work counts them (K/V, q, output, block k/v).  The step's
+# attention launch is too large to capture; its traffic is this ratio times its
+# algorithmic bytes (traffic grows with the K/V read).  None whenever the kernel has
+# changed since the last capture.
+ATTN_TRAFFIC_PER_BYTE = 1.0306
 
 
 def roofline_of(name, work, avg_ms, peaks, traffic=None, sustained=True):
@@ -247,6 +252,70 @@ def roofline_of(name, work, avg_ms, peaks, traffic=None, sustained=True):
     ach = fl / sec / 1e12
     return {"bound": "tensor", "achieved": round(ach, 1), "peak": tf_peak, "unit": "TFLOP/s",
             "frac": round(ach / tf_peak, 4), "traffic": traffic}
+
+
+def kernel_table(prof, work, steps, pass_ms, peaks, traffic_ratio=None):
+    """Per kernel group of a profiled pass: average ms per launch, launches per step,
+    share of the pass, and its roofline (traffic scaled from the attention capture)."""
+    ratio = ATTN_TRAFFIC_PER_BYTE if traffic_ratio is None else traffic_ratio
+    kernels = {}
+    for name, (tot, cnt) in prof.items():
+        avg = tot / max(cnt, 1)
+        ent = {"avg_ms": round(avg, 4), "launches_per_step": cnt / steps,
+               "share": round(tot / (pass_ms * steps), 4)}
+        if name in work:
+            traffic = None
+            if name == "attn_paged" and ratio is not None:
+                traffic = round(ratio * work[name]["bytes"])
+            ent["roofline"] = roofline_of(name, work[name], avg, peaks, traffic=traffic)
+        kernels[name] = ent
+    return kernels
+
+
+def compact_kernels(kernels):
+    """{group: [ms per launch, launches per step, fraction of its roofline]} -- the
+    per-kernel view of one sweep point."""
+    return {k: [v["avg_ms"], v["launches_per_step"], v.get("roofline", {}).get("frac")] for k, v in kernels.items()}
+
+
+def attention_configs(H, I, dev, peaks, steps=10, warmup=3):
+    """hspec_attn_paged_block alone on the two attention-heavy workloads: Llama-3-8B
+    shapes at 32 requests (ctx U[512,8192]) and Qwen-32B shapes at 128 requests (ctx
+    U[1024,32768]); CUDA events on the launching stream, K/V pools larger than L2."""
+    out = {}
+    for name in ("llama_c32", "qwen_c128"):
+        wl = I.WORKLOADS[name]
+        sh, C, K = wl.shapes, wl.C, wl.K
+        cfg = H.make_cfg(sh)
+        inp = I.make_attn_inputs(sh, wl, K, wl.seed, dev, shuffle=wl.shuffle, slack=wl.slack)
+        kv = H.kv_view(inp)
+        ws = H.alloc_workspace(H.hspec_attn_workspace_size(cfg, C, K, kv.max_pages), dev)
+        o = torch.empty_like(inp["q"])
+        ctx = int(inp["ctx_lens"].sum())
+        work = {"bytes": float(ctx * sh.Hkv * sh.D * 2 * 2 + 2 * C * K * (sh.Hq + sh.Hkv) * sh.D * 2),
+                "flops": 4.0 * sh.Hq * sh.D * K * (ctx + C * K)}
+        call = lambda: H.hspec_attn_paged_block(cfg, inp["q"], kv, inp["ctx_lens"], inp["k_blk"], inp["v_blk"], o, ws)
+        for _ in range(warmup):
+            call()
+        if H.hspec_sync_status() != 0:
+            raise RuntimeError(H.hspec_last_error())
+        stream = torch.cuda.current_stream()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(steps):
+            call()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if H.hspec_sync_status() != 0:
+            raise RuntimeError(H.hspec_last_error())
+        ms = e0.elapsed_time(e1) / steps
+        roof = roofline_of("attn_paged", work, ms, peaks, sustained=False)
+        out[name] = {"workload": wl.description, "us_per_call": round(ms * 1e3, 1),
+                     "achieved_gbs": roof["achieved"], "frac_of_hbm": roof["frac"]}
+        del inp, kv, ws, o
+        torch.cuda.empty_cache()
+    return out
 
 
 # ---------------------------------------------------------------------- our arm
@@ -371,17 +440,7 @@ def run_ours(args, rank, world, local):
 
     # roofline: per kernel group, from the events recorded on the step's stream
     work = step_work(wl.shapes, wl.C, wl.K, runner.st["ctx_lens"].cpu())
-    kernels = {}
-    for name, (tot, cnt) in prof.items():
-        avg = tot / max(cnt, 1)
-        ent = {"avg_ms": round(avg, 4), "launches_per_step": cnt / args.steps,
-               "share": round(tot / (pms * args.steps), 4)}
-        if name in work:
-            traffic = None
-            if name == "attn_paged" and ATTN_TRAFFIC_PER_BYTE is not None:
-                traffic = round(ATTN_TRAFFIC_PER_BYTE * work[name]["bytes"])
-            ent["roofline"] = roofline_of(name, work[name], avg, peaks, traffic=traffic)
-        kernels[name] = ent
+    kernels = kernel_table(prof, work, args.steps, pms, peaks)
     dominant = max(kernels, key=lambda k: kernels[k]["share"]) if kernels else None
     roof = dict(kernels[dominant]["roofline"]) if dominant and "roofline" in kernels[dominant] else None
     if roof:
@@ -401,19 +460,26 @@ def run_ours(args, rank, world, local):
     for K in (I.FULL_SWEEP_K if args.sweep else (args.K,)):
         for C in I.FULL_SWEEP_C:
             if C == wl.C and K == wl.K:
-                m2, lens2 = ms_max, runner.st["ctx_lens"].cpu()
+                m2, lens2, k2 = ms_max, runner.st["ctx_lens"].cpu(), kernels
             else:
                 w2 = I.full_workload(C, K, args.draft_vocab)
                 r2 = StepRunner(H, I, w2, dev, weights=runner.st["weights"])
-                m2, _, _ = time_steps(r2, max(5, args.steps // 2), 3, 1)
+                n2 = max(5, args.steps // 2)
+                m2, _, _ = time_steps(r2, n2, 3, 1)
+                p2, _, prof2 = time_steps(r2, n2, 1, 1, profile=True)
                 lens2 = r2.st["ctx_lens"].cpu()
+                k2 = kernel_table(prof2, step_work(wl.shapes, C, K, lens2), n2, p2, peaks)
                 r2.close()
                 del r2
                 torch.cuda.empty_cache()
             roof_ms = step_roofline_ms(wl.shapes, C, K, lens2, peaks)
             sweep.append({"C": C, "K": K, "us_per_step": round(m2 * 1e3, 1),
                           "tokens_per_s": round(C * K / (m2 / 1e3), 1),
-                          "roofline_us": round(roof_ms * 1e3, 1), "frac_of_roofline": round(roof_ms / m2, 4)})
+                          "roofline_us": round(roof_ms * 1e3, 1), "frac_of_roofline": round(roof_ms / m2, 4),
+                          "kernels": compact_kernels(k2)})
+
+    # the paged attention alone on the attention-heavy workloads (rank 0, one GPU)
+    attn_cfg = attention_configs(H, I, dev, peaks) if (rank == 0 and not args.no_attention_configs) else None
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -431,7 +497,8 @@ def run_ours(args, rank, world, local):
                 "config": step_config(wl, world),
                 "roofline": roof, "attention_roofline": attn_roof, "kernels": kernels,
                 "kernels_pass_ms_per_step": round(pms, 4),
-                "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clk}
+                "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clk,
+                "attention_configs": attn_cfg}
         if sweep is not None:
             line["sweep"] = sweep
         print(json.dumps(line), flush=True)
@@ -594,6 +661,8 @@ def main():
                     help="reduced draft head rows (0 = the full 128256-token head)")
     ap.add_argument("--sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-attention-configs", action="store_true",
+                    help="skip timing the paged attention alone on the Llama C=32 and Qwen C=128 workloads")
     ap.add_argument("--kernel", choices=["step", "attn", "inject", "ssd", "verify", "gemm"], default="step",
                     help="time one C-ABI call on --workload instead of the full draft step")
     ap.add_argument("--workload", default="llama_c32", help="kernel-level workload (tiny, llama_c1, llama_c32, qwen_c128, or full_C<C>_K<K>: one layer of the full step)")

@@ -18,7 +18,7 @@
 // byte read from HBM feeds all R queries; with R <= 64 the rows are spread 16 per
 // 32-lane TMEM quarter so that all four SM sub-partitions share the softmax work;
 // rows without a query are zero.
-// Warp roles (448 threads, one CTA per SM):
+// Warp roles (480 threads, one CTA per SM):
 //   warps 0..3  producers: all four walk the CTA's pieces.  Warp 0 loads each piece's
 //               Q tile (TMA) into one of two Q buffers.  Page ids are read two tiles
 //               ahead.  The 64-token K/V tiles stream through a ring of 6 stages (5 for
@@ -28,14 +28,17 @@
 //               tile at once -- and warp 0 writes the tile's description next to it.
 //               A sequence's last tiles are the block's own keys (one more tile for
 //               K <= 64).
-//   warp 4      TMEM owner and Q.K^T issuer: S_b = Q . K_i^T (N = 64, K = D) into S
-//               buffer b = i % 4 as soon as tile i has landed and the P.V of tile
-//               i - 4 has read S_b, so that the S of a group's next tile is ready while
-//               the group still works on the current one.
+//   warps 4, 14 Q.K^T issuers (warp 4 also owns TMEM): S_b = Q . K_i^T (N = 64, K = D)
+//               into S buffer b = i % 4 as soon as tile i has landed and the P.V of
+//               tile i - 4 has read S_b, so that the S of a group's next tile is ready
+//               while the group still works on the current one.  Warp 4 takes the even
+//               tiles, warp 14 the odd ones (one per softmax group): two chains of
+//               dependent MMAs in flight instead of one.
 //   warp 5      P.V issuer: O_w += P_i . V_i (N = D, K = 64) as soon as the P of tile
 //               i is in TMEM, with P (the A operand) read from TMEM, as two products
 //               (its bf16 high and low parts); its commit frees the K/V stage and the S
-//               buffer.
+//               buffer, and at a piece's last tile it frees the piece's Q buffer (every
+//               Q.K^T of the piece finished before that tile's softmax began).
 //   warps 6..9  softmax warpgroup 0 (tiles i even), warps 10..13 warpgroup 1 (i odd):
 //               one query row per thread (M = 64: two threads per row, one in each
 //               half-warp, 32 scores each); mask, running max in the exp2 domain,
@@ -65,7 +68,7 @@ constexpr int TT = kAttnTcTile;  // tokens per tile
 constexpr int PPT = TT / 16;     // 16-token pages per tile
 constexpr int NSB = TT == 64 ? 4 : 8;   // S buffers in TMEM (half the columns)
 constexpr int NPW = 4;           // producer warps
-constexpr int THREADS = 32 * (NPW + 2 + 8);  // producers, 2 MMA warps, 2 softmax warpgroups
+constexpr int THREADS = 32 * (NPW + 3 + 8);  // producers, 3 MMA warps, 2 softmax warpgroups
 constexpr int ROWS = 128;     // MMA M
 
 struct TileMeta {  // written by the producer before the stage's barrier arrive
@@ -77,6 +80,7 @@ struct TileMeta {  // written by the producer before the stage's barrier arrive
   int qslot, qseq; // Q buffer of the piece and the piece's use count of that buffer
   int end;         // 1: no more work
   int bt;          // block tiles: index among the block's tiles
+  int end_at;      // sentinel stages: the first tile index past the work
 };
 
 // SP: the R <= 64 queries of a kv head in an M = 64 tile (rows 16 per TMEM lane
@@ -180,10 +184,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* p_full = s_free + NSB;    // [NSB]
   uint64_t* q_full = p_full + NSB;    // [2]
   uint64_t* q_empty = q_full + 2;     // [2]
-  uint64_t* drain = q_empty + 2;      // [2] every MMA of an issuer (and its arrivals) finished
-  uint32_t* tmem_slot = (uint32_t*)(drain + 2);
+  uint64_t* drain = q_empty + 2;      // [3] every MMA of an issuer (and its arrivals) finished
+  uint32_t* tmem_slot = (uint32_t*)(drain + 3);
   volatile int* end_tile = (volatile int*)(tmem_slot + 1);
-  volatile int* s_stop = end_tile + 1;  // a producer warp gave up waiting
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = a.Hq / a.Hkv, R = a.K * G;
@@ -191,7 +194,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   constexpr bool spread = SP;
   int* err = a.err;
   const uint64_t lim = a.wait_ns ? (uint64_t)a.wait_ns : tc::kWaitLimitNs;  // pipeline waits
-  constexpr int QK_WARP = NPW, PV_WARP = NPW + 1, SM_WARP0 = NPW + 2;
+  // Q.K^T issuers: QK_WARP for the even tiles (and the TMEM owner), QK_WARP2 for the odd
+  constexpr int QK_WARP = NPW, PV_WARP = NPW + 1, SM_WARP0 = NPW + 2, QK_WARP2 = NPW + 2 + 8;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
@@ -209,8 +213,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     tc::mbar_init(&drain[0], 1);
     tc::mbar_init(&drain[1], 1);
+    tc::mbar_init(&drain[2], 1);
     *end_tile = 0x7fffffff;
-    *s_stop = 0;
     tc::fence_mbar_init();
   }
   if (warp == QK_WARP) tc::tmem_alloc(tmem_slot, L::TMEM_COLS);
@@ -271,10 +275,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     int q_last = -1;  // warp 0: the last piece whose Q load it armed
     bool ok = true;
     // Every producer warp walks the same pieces and passes the same barriers: the loop
-    // ends only after one, when the work is done or a producer has given up waiting.
+    // ends only at one, when the work is done or a producer has given up waiting (the
+    // barrier ORs the warps' `ok`, so all of them take the same decision).
+    bool stopped = false;
     for (int seq = 0;; ++seq) {
-      asm volatile("bar.sync 1, %0;" ::"n"(32 * NPW) : "memory");
-      if (*s_stop) break;
+      if (tc::bar_or<1, 32 * NPW>(!ok)) {
+        stopped = true;
+        break;
+      }
       if (pos >= end) {  // the CTA's next chunk
         k += gridDim.x;
         if (k >= n_chunks) break;
@@ -380,7 +388,6 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         __syncwarp();
       }
-      if (!ok) *s_stop = 1;
     }
     // No copy may land after the CTA has finished: wait, with the full limit, for the
     // last filling of every stage this warp armed (complete once the copies of all four
@@ -394,30 +401,36 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int q = q_last > 0 ? q_last - 1 : 0; q <= q_last; ++q) tc::mbar_wait(&q_full[q & 1], (q >> 1) & 1, err);
     }
     __syncwarp();
-    // sentinel stage: no more work
-    if (!*s_stop) {
-      const int s = tile_i % NS;
-      bool fine = true;
-      if (lane == 0) fine = tc::mbar_wait(&kv_empty[s], ((tile_i / NS) & 1) ^ 1, err, lim);
-      if (lane == 0 && fine) {
-        if (pw == 0) meta[s].end = 1;
-        tc::mbar_arrive(&kv_full[s]);
+    // sentinel stages: no more work (two, one for each Q.K^T issuer)
+    if (!stopped) {
+      const int end_at = tile_i;
+      for (int e = 0; e < 2; ++e) {
+        const int ti = end_at + e, s = ti % NS;
+        bool fine = true;
+        if (lane == 0) fine = tc::mbar_wait(&kv_empty[s], ((ti / NS) & 1) ^ 1, err, lim);
+        fine = __shfl_sync(0xffffffffu, fine ? 1 : 0, 0) != 0;
+        if (!fine) break;
+        if (lane == 0) {
+          if (pw == 0) meta[s].end = 1, meta[s].end_at = end_at;
+          tc::mbar_arrive(&kv_full[s]);
+        }
       }
     }
-  } else if (warp == QK_WARP) {
+  } else if (warp == QK_WARP || warp == QK_WARP2) {
     if (lane == 0) {
+      const int qw = warp == QK_WARP2 ? 1 : 0;
       // ---------------------------------------------------------- Q.K^T issuer
       // S_b = Q . K_i^T into S buffer b = i % NSB once tile i has landed, S_b is free
       // (the P.V of tile i - NSB has read its P) and the piece's Q is loaded.  Issuing
       // P.V from another thread keeps either kind of MMA from waiting behind the other.
       constexpr uint32_t idesc_qk = tc::idesc_bf16_f32(L::MR, TT);
       int q_seen[2] = {-1, -1};
-      for (int qk = 0;; ++qk) {
+      for (int qk = qw;; qk += 2) {
         const int s = qk % NS, b = qk & (NSB - 1);
         if (qk >= NSB && !tc::mbar_wait(&s_free[b], ((qk / NSB) - 1) & 1, err, lim)) break;
         if (!tc::mbar_wait(&kv_full[s], (qk / NS) & 1, err, lim)) break;
         if (meta[s].end) {
-          *end_tile = qk;
+          *end_tile = meta[s].end_at;
           break;
         }
         const int slot = meta[s].qslot, seq = meta[s].qseq;
@@ -432,11 +445,10 @@ __global__ void __launch_bounds__(THREADS, 1)
           tc::mma_bf16(tmem + L::S_COL(b), tc::sdesc_k128(q + (kk / 4) * L::Q_BLK + (kk % 4) * 32),
                        tc::sdesc_k128(k + (kk / 4) * L::KV_BLK + (kk % 4) * 32), idesc_qk, kk > 0);
         tc::mma_commit(&s_full[b]);
-        if (meta[s].local == meta[s].n_tiles - 1) tc::mma_commit(&q_empty[slot]);  // piece's last QK
       }
       // no MMA or commit arrival may land after the CTA has finished
-      tc::mma_commit(&drain[0]);
-      tc::mbar_wait(&drain[0], 0, err);
+      tc::mma_commit(&drain[qw == 0 ? 0 : 2]);
+      tc::mbar_wait(&drain[qw == 0 ? 0 : 2], 0, err);
     }
   } else if (warp == PV_WARP) {
     if (lane == 0) {
@@ -468,6 +480,9 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int kk = 0; kk < PPT; ++kk)
             tc::mma_bf16_ts(tmem + L::O_COL(w), pt + TT / 2 + kk * 8, tc::sdesc_mn128(v + kk * L::V_PAGE, 2048),
                             idesc_pv, 1u);
+          // the piece's last tile: every Q.K^T of the piece has finished (each before its
+          // tile's softmax began), so its Q buffer is free
+          if (meta[s].local == meta[s].n_tiles - 1) tc::mbar_arrive(&q_empty[meta[s].qslot]);
           tc::mma_commit(&kv_empty[s]);
           tc::mma_commit(&s_free[pv & (NSB - 1)]);  // P read: S buffer free for tile pv + NSB
           ++pv;

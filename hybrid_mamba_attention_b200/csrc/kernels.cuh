@@ -96,8 +96,8 @@ struct SsdArgs {
 };
 size_t ssd_smem_bytes(int P, int N, int Q);
 void ssd_scan(int dtype, const SsdArgs& a, cudaStream_t s);
-// Tensor-core state readout (ssd_tc.cu): bf16, h0 given, no final state, one chunk,
-// K <= 16, d_state 128, 64 <= P <= 128 dividing 128.
+// Tensor-core state readout (ssd_tc.cu): bf16, h0 given, the block as one chunk,
+// K <= 32, d_state 128, 64 <= P <= 128 dividing 128; with or without the final state.
 bool ssd_tc_supported(int dtype, const SsdArgs& a);
 bool ssd_tc_launch(const SsdArgs& a, cudaStream_t s);
 

@@ -1,5 +1,5 @@
 // Mamba-2 SSD block scan from an injected state, readout on the 5th-generation tensor
-// cores (bf16 drafter, one chunk of K <= 16 positions, no final state requested).
+// cores (bf16 drafter, the whole block as one chunk of K <= 32 positions).
 // H-Spec (arXiv 2609.24197) Abstract: each Mamba layer starts from the projected
 // last-token hidden state and the block is evaluated in parallel; the chunked
 // "state-space dual" form of Dao & Gu (2024) gives, for head h and position t,
@@ -8,29 +8,40 @@
 //          + sum_{s<=t} (C_t . B_s) exp(cum_t - cum_s) dt_s x_s[p]  (inside the block)
 //          + D_h x_t[p],                    cum_t = sum_{r<=t} dt_r A_h,
 //
-// the same sum as the step-by-step recurrence.  The state S = h0 of one request is
+// and the state after the block,
+//
+//   hK[p][n] = exp(cum_{K-1}) S[p][n] + sum_s exp(cum_{K-1} - cum_s) dt_s x_s[p] B_s[n],
+//
+// the same sums as the step-by-step recurrence.  The state S = h0 of one request is
 // H*P rows of N fp32 values: 2 MB per request and layer at Llama shapes, the only large
 // operand, read once.  Its readout C . S^T is a dense contraction (K x N by N x H*P)
-// and runs on tcgen05 as kind::tf32 with M = 128 state rows (heads x P), N = 16
-// positions, K = 8 per instruction, the accumulator in TMEM.  So that the product is
-// as exact as fp32, each state tile is split into hi = tf32(S), rounded in place in
-// shared memory, and lo = S - hi, written to TMEM and read by the MMA from there (C is
-// exact in tf32: it comes from bf16); tf32 x tf32 products are exact and accumulate in
-// fp32.
+// and runs on tcgen05 as kind::tf32 with M = 128 state rows (heads x P), N = NT = 16 or
+// 32 positions, K = 8 per instruction, the accumulator in TMEM.  So that the product is
+// as exact as fp32, the state is split into hi = S with its 13 low mantissa bits
+// cleared and lo = S - hi (exact in fp32, below 2^-10 |S|): the A operand of the first
+// MMA is the state tile as it landed in shared memory, of which the tensor core reads
+// the tf32 part -- hi (it drops the low mantissa bits; a GPU test with every low bit
+// set checks this) -- and the second MMA reads lo from TMEM.  C is exact in tf32 (it
+// comes from bf16); tf32 x tf32 products are exact and accumulate in fp32.
 //
 // Persistent kernel, one CTA per SM, a static range of (request, 128-row tile) items:
 //   warp 0      TMA producer: the fp32 state tile (N / 32 boxes of 128 rows x 128 B,
-//               128-byte swizzle) into one of three stages.
-//   warp 1      TMEM owner and MMA issuer: 2 (hi from shared memory, lo from TMEM) x
+//               128-byte swizzle) into one of three (NT = 32: two) stages.
+//   warp 1      TMEM owner and MMA issuer: 2 (state from shared memory, lo from TMEM) x
 //               N / 8 MMAs per tile into one of two TMEM accumulators.
 //   warps 2..5  transform group 0 (tiles k even), warps 6..9 group 1 (k odd); per tile,
-//               one state row (= TMEM lane) per thread: round the row to tf32 in place
-//               and write its lo to the group's TMEM buffer; for a new request the C^T
-//               operand (bf16 -> fp32, swizzled) and C . B^T; the tile's dt, cumulative
-//               decay, the in-block matrix L and x; then, once the tile's MMAs are done,
-//               its epilogue.  The tile's global loads are issued before its waits, and
-//               the two groups overlap each other's latencies.
-// Every wait gives up after a time bound and sets the device error word.
+//               one state row (= TMEM lane) per thread: for a new request the C^T
+//               operand (bf16 -> fp32, swizzled), the B rows when the final state is
+//               wanted, and C . B^T; the tile's dt and cumulative decay (a segmented warp
+//               scan); lo of the thread's row into the group's TMEM buffer, and with a
+//               final state the row of hK; the in-block matrix L[t][s] =
+//               (C_t . B_s) exp(cum_t - cum_s) dt_s; then, once the tile's MMAs are done,
+//               its epilogue y = exp(cum) (C S^T) + L x + D x, with x held in registers.
+//               The tile's global loads are issued before its waits, and the two groups
+//               overlap each other's latencies.
+// Every pipeline wait gives up after the call's limit and sets the device error word;
+// before the CTA exits, the producer and the MMA issuer wait for their own copies and
+// MMAs in flight.
 #include <stdint.h>
 
 #include "../../include/hspec.h"
@@ -46,29 +57,29 @@ namespace {
 
 constexpr int THREADS = 320;  // producer, MMA, 2 transform warpgroups
 constexpr int ROWS = 128;    // MMA M: state rows (head, p) per tile
-constexpr int NT = 16;       // MMA N: positions (K <= 16, rows past K are zero)
-constexpr int KMAX = 16;
 constexpr int NMAX = 128;    // d_state
 constexpr int TILE_BYTES = ROWS * NMAX * 4;  // 64 KB
 constexpr int HPT_MAX = 2;   // heads per tile (P >= 64)
-constexpr int NSTAGE = 3;    // state-tile stages
-// TMEM columns: lo of tile k in [128 (k % 2), +128), accumulator of tile k at 256 + 16 (k % 2)
+// TMEM columns: lo of tile k in [128 (k % 2), +128), accumulator of tile k at 256 + NT (k % 2)
 constexpr uint32_t TMEM_COLS = 512;
 
+// NT: MMA N = positions per tile (the block, K <= NT, zero past K): 16 or 32.
+template <int NT>
 struct SsdTcLay {
-  static constexpr int OFF_A = 0;                          // stages of the state tile (hi)
-  static constexpr int OFF_B = OFF_A + NSTAGE * TILE_BYTES;  // C^T: [n/32][16 positions][128 B]
-  static constexpr int B_BYTES = NMAX / 32 * NT * 128;     // 8 KB
-  // per transform group g: x, L^T, exp(cum) and D, C . B^T, dt and cum
-  static constexpr int OFF_X = OFF_B + B_BYTES;            // x: [2][KMAX][ROWS] fp32
-  static constexpr int X_BYTES = KMAX * ROWS * 4;
-  static constexpr int OFF_L = OFF_X + 2 * X_BYTES;        // L^T: [2][HPT_MAX][KMAX (s)][KMAX (t)]
-  static constexpr int L_BYTES = HPT_MAX * KMAX * KMAX * 4;
-  static constexpr int OFF_E = OFF_L + 2 * L_BYTES;        // exp(cum): [2][HPT_MAX][KMAX], D_h: [2][HPT_MAX]
-  static constexpr int E_BYTES = HPT_MAX * (KMAX + 1) * 4;
-  static constexpr int OFF_CB = OFF_E + 2 * E_BYTES;       // C . B^T: [2][KMAX][KMAX]
-  static constexpr int OFF_DT = OFF_CB + 2 * KMAX * KMAX * 4;  // dt, then cum: [2][2][HPT_MAX][KMAX]
-  static constexpr int OFF_BAR = OFF_DT + 4 * HPT_MAX * KMAX * 4;
+  static constexpr int NSTAGE = NT == 16 ? 3 : 2;              // state-tile stages
+  static constexpr int OFF_A = 0;                               // stages of the state tile
+  static constexpr int OFF_B = OFF_A + NSTAGE * TILE_BYTES;     // C^T: [n/32][NT positions][128 B] fp32
+  static constexpr int B_BYTES = NMAX / 32 * NT * 128;
+  // per transform group g: the B rows, L^T, exp(cum) and D, C . B^T, dt and cum
+  static constexpr int OFF_BR = OFF_B + B_BYTES;                // B rows: [2][NT][NMAX] bf16
+  static constexpr int BR_BYTES = NT * NMAX * 2;
+  static constexpr int OFF_L = OFF_BR + 2 * BR_BYTES;           // L^T: [2][HPT_MAX][NT (s)][NT (t)]
+  static constexpr int L_BYTES = HPT_MAX * NT * NT * 4;
+  static constexpr int OFF_E = OFF_L + 2 * L_BYTES;             // exp(cum): [2][HPT_MAX][NT], D_h: [2][HPT_MAX]
+  static constexpr int E_BYTES = HPT_MAX * (NT + 1) * 4;
+  static constexpr int OFF_CB = OFF_E + 2 * E_BYTES;            // C . B^T: [2][NT][NT]
+  static constexpr int OFF_DT = OFF_CB + 2 * NT * NT * 4;       // dt, then cum: [2][2][HPT_MAX][NT]
+  static constexpr int OFF_BAR = OFF_DT + 4 * HPT_MAX * NT * 4;
   static constexpr int SMEM = OFF_BAR + 256 + 1024;
 };
 
@@ -80,8 +91,8 @@ struct SsdTcArgs {
   int n_items;    // C * n_tiles
 };
 
-// hi: the value with its 13 low mantissa bits cleared (a tf32 value, whatever rounding
-// the tensor core applies to it); lo = v - hi is exact in fp32 and below 2^-10 |v|.
+// hi: the value with its 13 low mantissa bits cleared (the tf32 value the tensor core
+// reads); lo = v - hi is exact in fp32 and below 2^-10 |v|.
 __device__ __forceinline__ uint32_t tf32_hi(uint32_t bits) { return bits & 0xFFFFE000u; }
 
 // Loads issued where they stand (volatile: not moved towards their first use), so
@@ -123,23 +134,30 @@ __device__ __forceinline__ void mma_tf32(uint32_t tmem_d, uint64_t adesc, uint64
       : "memory");
 }
 
-template <typename TDT>
+// NT fp32 columns of this thread's TMEM lane
+__device__ __forceinline__ void tmem_ld_nt(uint32_t taddr, float (&v)[16]) { tc::tmem_ld16(taddr, v); }
+__device__ __forceinline__ void tmem_ld_nt(uint32_t taddr, float (&v)[32]) { tc::tmem_ld32(taddr, v); }
+
+// HK: the final state is written (a separate instantiation, so that the draft step's
+// scan carries none of its registers).
+template <typename TDT, int NT, bool HK>
 __global__ void __launch_bounds__(THREADS, 1) ssd_tc_kernel(const __grid_constant__ CUtensorMap h0_map, SsdTcArgs t) {
-  using L = SsdTcLay;
+  using L = SsdTcLay<NT>;
+  constexpr int NSTAGE = L::NSTAGE;
   const SsdArgs& a = t.a;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = tc::smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023) & ~1023u) - raw);
   uint8_t* sA = smem + L::OFF_A;
   uint8_t* sB = smem + L::OFF_B;
-  float* sX = (float*)(smem + L::OFF_X);
+  uint8_t* sBR = smem + L::OFF_BR;
   float* sL = (float*)(smem + L::OFF_L);
   float* sE = (float*)(smem + L::OFF_E);
   float* sCB = (float*)(smem + L::OFF_CB);
   float* sDt = (float*)(smem + L::OFF_DT);
   uint64_t* a_full = (uint64_t*)(smem + L::OFF_BAR);  // [NSTAGE]
   uint64_t* a_empty = a_full + NSTAGE;                 // [NSTAGE]
-  // [2] tile k: hi rounded, lo in TMEM buffer k % 2, operands ready (one barrier per lo
+  // [2] tile k: lo in TMEM buffer k % 2 and the C^T operand ready (one barrier per lo
   // buffer: the transform may finish tile k + 1 before the MMA thread has taken tile k,
   // and the phases of one barrier must not run two ahead of its waiter)
   uint64_t* lo_full = a_empty + NSTAGE;
@@ -147,7 +165,6 @@ __global__ void __launch_bounds__(THREADS, 1) ssd_tc_kernel(const __grid_constan
   uint64_t* d_free = acc_full + 2;                     // [2] epilogue has read the accumulator
   uint64_t* drain = d_free + 2;
   uint32_t* tmem_slot = (uint32_t*)(drain + 1);
-  volatile int* s_fail = (volatile int*)(tmem_slot + 1);  // a transform thread gave up waiting
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int P = a.P, N = a.N, K = a.K, hpt = t.hpt;
@@ -169,7 +186,6 @@ __global__ void __launch_bounds__(THREADS, 1) ssd_tc_kernel(const __grid_constan
     tc::mbar_init(&lo_full[0], 4);
     tc::mbar_init(&lo_full[1], 4);
     tc::mbar_init(drain, 1);
-    *s_fail = 0;
     tc::fence_mbar_init();
   }
   if (warp == 1) tc::tmem_alloc(tmem_slot, TMEM_COLS);
@@ -210,14 +226,14 @@ __global__ void __launch_bounds__(THREADS, 1) ssd_tc_kernel(const __grid_constan
         if (k >= 2 && !tc::mbar_wait(&d_free[db], ((k >> 1) - 1) & 1, err, lim)) break;
         if (!tc::mbar_wait(&lo_full[k & 1], (k >> 1) & 1, err, lim)) break;
         tc::tc_fence_after();
-        const uint32_t hi = tc::smem_u32(sA + st * TILE_BYTES);
+        const uint32_t st_addr = tc::smem_u32(sA + st * TILE_BYTES);
         const uint32_t lo = tmem + (uint32_t)(128 * (k & 1));
         const uint32_t d = tmem + 256u + (uint32_t)(db * NT);
 #pragma unroll
         for (int kb = 0; kb < NMAX / 8; ++kb) {
           const uint32_t aoff = (uint32_t)((kb >> 2) * ROWS * 128 + (kb & 3) * 32);
           const uint64_t bdesc = tc::sdesc_k128(b_base + (uint32_t)((kb >> 2) * NT * 128 + (kb & 3) * 32));
-          mma_tf32(d, tc::sdesc_k128(hi + aoff), bdesc, idesc, kb > 0);
+          mma_tf32(d, tc::sdesc_k128(st_addr + aoff), bdesc, idesc, kb > 0);  // hi: the tf32 part of S
           mma_tf32_ts(d, lo + (uint32_t)(kb * 8), bdesc, idesc, 1u);
         }
         tc::mma_commit(&acc_full[db]);
@@ -235,38 +251,48 @@ __global__ void __launch_bounds__(THREADS, 1) ssd_tc_kernel(const __grid_constan
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const int hl = row / P, p = row % P;
     const int gw = (warp - 2) & 3;               // warp within the group
+    constexpr bool want_hK = HK;
     const TDT* dtp = (const TDT*)a.dt;
     const bf16* xg = (const bf16*)a.x;
     const bf16* Bg = (const bf16*)a.B;
     const bf16* Cg = (const bf16*)a.Cm;
-    float* gX = sX + g * KMAX * ROWS;
-    float* gL = sL + g * HPT_MAX * KMAX * KMAX;  // [head][s][t]
-    float* gE = sE + g * HPT_MAX * (KMAX + 1);
-    float* gCB = sCB + g * KMAX * KMAX;
-    float* gDt = sDt + g * 2 * HPT_MAX * KMAX;   // dt [head][t], then cum [head][t]
+    uint8_t* gBR = sBR + g * L::BR_BYTES;        // B rows [NT][NMAX] bf16
+    float* gL = sL + g * HPT_MAX * NT * NT;      // [head][s][t]
+    float* gE = sE + g * HPT_MAX * (NT + 1);
+    float* gCB = sCB + g * NT * NT;
+    float* gDt = sDt + g * 2 * HPT_MAX * NT;     // dt [head][t], then cum [head][t]
     int c_prev = -1;
     auto gsync = [&]() {
       if (g == 0) asm volatile("bar.sync 1, 128;" ::: "memory");
       else asm volatile("bar.sync 2, 128;" ::: "memory");
     };
 
-    // The group's warps pass the same named barriers in the same order; a wait that
-    // gives up sets s_fail, and the group leaves the loop after its next barrier.
+    // The group's warps pass the same named barriers in the same order.  A warp whose
+    // wait gave up (`failed`, warp-uniform) says so at the group's next barrier, which
+    // ORs it over the group, and the whole group leaves the loop there.
+    bool failed = false;
     for (int i = i0 + g; i < i1; i += 2) {
       const int k = i - i0, st = k % NSTAGE;
       const int c = i / t.n_tiles, j = i % t.n_tiles;
       const bool new_req = c != c_prev;
       // the tile's global loads first: x of this thread's row at every position (rows
-      // past K re-read row K - 1 and are zeroed below), and (first warp, lane hh * 16 +
-      // tt) dt of head hh at position tt
-      uint16_t xv[KMAX];
+      // past K re-read row K - 1 and count as zero), and (lane hh * NT + tt of the
+      // group's first warps) dt of head hh at position tt
+      uint32_t xw[NT / 2];  // bf16 pairs: position 2i in the low half, 2i + 1 in the high half
       {
         const bf16* xr = xg + (size_t)c * K * a.x_rs + (size_t)(j * hpt) * P + row;
 #pragma unroll
-        for (int tt = 0; tt < KMAX; ++tt) xv[tt] = ldg_u16(xr + (size_t)(tt < K ? tt : K - 1) * a.x_rs);
+        for (int tt = 0; tt < NT; tt += 2)
+          xw[tt / 2] = (uint32_t)ldg_u16(xr + (size_t)(tt < K ? tt : K - 1) * a.x_rs) |
+                       ((uint32_t)ldg_u16(xr + (size_t)(tt + 1 < K ? tt + 1 : K - 1) * a.x_rs) << 16);
       }
-      const int dh = tid >> 4, dtt = tid & 15;
-      const bool dlive = tid < 32 && dh < hpt && dtt < K;
+      // x at position s (fp32; the bf16 bits in the upper half of a word)
+      auto xval = [&](int s2) {
+        return __uint_as_float((s2 & 1) ? (xw[s2 >> 1] & 0xFFFF0000u) : (xw[s2 >> 1] << 16));
+      };
+      const int dh = tid / NT, dtt = tid % NT;
+      const bool dlane = tid < HPT_MAX * NT;
+      const bool dlive = dlane && dh < hpt && dtt < K;
       const int dhead = j * hpt + (dh < hpt ? dh : 0);
       uint32_t draw_bits = 0, dA_bits = 0, dD_bits = 0, dbias_bits = 0;
       if (dlive) {
@@ -278,11 +304,9 @@ __global__ void __launch_bounds__(THREADS, 1) ssd_tc_kernel(const __grid_constan
       }
       // the state tile has landed; for a new request also the MMAs of the previous tile
       // (the last reader of the C^T operand) are done
-      bool ok = tc::mbar_wait_warp(&a_full[st], (k / NSTAGE) & 1, err, lim);
+      bool ok = !failed && tc::mbar_wait_warp(&a_full[st], (k / NSTAGE) & 1, err, lim);
       if (ok && new_req && k >= 1) ok = tc::mbar_wait_warp(&acc_full[(k - 1) & 1], ((k - 1) >> 1) & 1, err, lim);
-      if (!ok) *s_fail = 1;
-      gsync();
-      if (*s_fail) break;
+      if (g == 0 ? tc::bar_or<1, 128>(!ok) : tc::bar_or<2, 128>(!ok)) break;  // the group's barrier
       tc::tc_fence_after();
       if (new_req) {
         // C^T operand: row tt (position) of 128-byte column blocks, zero past K
@@ -302,12 +326,48 @@ __global__ void __launch_bounds__(THREADS, 1) ssd_tc_kernel(const __grid_constan
           *(float4*)(sB + (n4 >> 5) * NT * 128 + tt * 128 + ((ch ^ (tt & 7)) << 4)) =
               make_float4(lo2.x, lo2.y, hi2.x, hi2.y);
         }
+        if constexpr (want_hK) {
+          // B rows of the request (bf16 as stored; positions < K)
+          for (int e = tid; e < K * (NMAX / 4); e += 128) {
+            const int tt = e / (NMAX / 4), n4 = (e % (NMAX / 4)) * 4;
+            *(uint2*)(gBR + (tt * NMAX + n4) * 2) = *(const uint2*)(Bg + (size_t)(c * K + tt) * a.bc_rs + n4);
+          }
+        }
         c_prev = c;
       }
-      // this thread's state row: round to tf32 in place (hi), lo = S - hi into the
-      // group's TMEM buffer (free: the group's previous tile finished its MMAs)
+      // the tile's heads: dt, cum = inclusive scan of dt A_h (segmented, NT lanes), exp(cum)
+      if (dlane) {
+        float d = sizeof(TDT) == 2 ? __bfloat162float(__ushort_as_bfloat16((unsigned short)draw_bits))
+                                   : __uint_as_float(draw_bits);
+        if (dlive && a.dt_bias) d = softplus(d + __uint_as_float(dbias_bits));
+        const float dA = __uint_as_float(dA_bits), dD = __uint_as_float(dD_bits);
+        float cum = dlive ? d * dA : 0.f;
+#pragma unroll
+        for (int o = 1; o < NT; o <<= 1) {
+          const float v = __shfl_up_sync(0xffffffffu, cum, o, NT);
+          if (dtt >= o) cum += v;
+        }
+        if (dlive) {
+          gDt[dh * NT + dtt] = d;
+          gDt[(HPT_MAX + dh) * NT + dtt] = cum;
+          gE[dh * (NT + 1) + dtt] = expf(cum);
+          if (dtt == 0) gE[dh * (NT + 1) + NT] = dD;
+        }
+      }
+      gsync();  // the C^T operand (and B rows) of a new request, dt and cum are complete
+      // this thread's state row: lo = S - hi into the group's TMEM buffer (free: the
+      // group's previous tile finished its MMAs); with a final state also its row of hK
       {
-        uint8_t* rowp = sA + st * TILE_BYTES + row * 128;
+        const uint8_t* rowp = sA + st * TILE_BYTES + row * 128;
+        float w[want_hK ? NT : 1], eK = 0.f;
+        if constexpr (want_hK) {
+          const float cK = gDt[(HPT_MAX + hl) * NT + (K - 1)];
+          eK = expf(cK);
+#pragma unroll
+          for (int s2 = 0; s2 < NT; ++s2)
+            w[s2] = s2 < K ? expf(cK - gDt[(HPT_MAX + hl) * NT + s2]) * gDt[hl * NT + s2] * xval(s2) : 0.f;
+        }
+        float* hKr = want_hK ? a.hK + ((size_t)(c * a.H + j * hpt + hl) * P + p) * N : nullptr;
 #pragma unroll
         for (int cb = 0; cb < NMAX / 32; ++cb) {
           uint4 v[8];
@@ -316,21 +376,46 @@ __global__ void __launch_bounds__(THREADS, 1) ssd_tc_kernel(const __grid_constan
           uint32_t lo[32];
 #pragma unroll
           for (int ch = 0; ch < 8; ++ch) {
-            const uint32_t h0 = tf32_hi(v[ch].x), h1 = tf32_hi(v[ch].y);
-            const uint32_t h2 = tf32_hi(v[ch].z), h3 = tf32_hi(v[ch].w);
-            lo[4 * ch + 0] = __float_as_uint(__uint_as_float(v[ch].x) - __uint_as_float(h0));
-            lo[4 * ch + 1] = __float_as_uint(__uint_as_float(v[ch].y) - __uint_as_float(h1));
-            lo[4 * ch + 2] = __float_as_uint(__uint_as_float(v[ch].z) - __uint_as_float(h2));
-            lo[4 * ch + 3] = __float_as_uint(__uint_as_float(v[ch].w) - __uint_as_float(h3));
-            v[ch] = make_uint4(h0, h1, h2, h3);
+            lo[4 * ch + 0] = __float_as_uint(__uint_as_float(v[ch].x) - __uint_as_float(tf32_hi(v[ch].x)));
+            lo[4 * ch + 1] = __float_as_uint(__uint_as_float(v[ch].y) - __uint_as_float(tf32_hi(v[ch].y)));
+            lo[4 * ch + 2] = __float_as_uint(__uint_as_float(v[ch].z) - __uint_as_float(tf32_hi(v[ch].z)));
+            lo[4 * ch + 3] = __float_as_uint(__uint_as_float(v[ch].w) - __uint_as_float(tf32_hi(v[ch].w)));
           }
-#pragma unroll
-          for (int ch = 0; ch < 8; ++ch) *(uint4*)(rowp + cb * ROWS * 128 + ((ch ^ (row & 7)) << 4)) = v[ch];
           tc::tmem_st32_nowait(tmem + lane_off + (uint32_t)(128 * g + 32 * cb), lo);
+          if constexpr (want_hK) {
+            // hK[n] = exp(cum_{K-1}) S[n] + sum_s w_s B_s[n], n in this 32-column block
+            float acc[32];
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+              acc[4 * ch + 0] = eK * __uint_as_float(v[ch].x);
+              acc[4 * ch + 1] = eK * __uint_as_float(v[ch].y);
+              acc[4 * ch + 2] = eK * __uint_as_float(v[ch].z);
+              acc[4 * ch + 3] = eK * __uint_as_float(v[ch].w);
+            }
+#pragma unroll
+            for (int s2 = 0; s2 < NT; ++s2) {
+              if (s2 >= K) break;
+              const uint4* br = (const uint4*)(gBR + (s2 * NMAX + cb * 32) * 2);  // 32 bf16, same for all lanes
+              const float ws = w[s2];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const uint4 b8 = br[q];
+                const uint32_t bw[4] = {b8.x, b8.y, b8.z, b8.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bw[e]));
+                  acc[8 * q + 2 * e] = fmaf(ws, f.x, acc[8 * q + 2 * e]);
+                  acc[8 * q + 2 * e + 1] = fmaf(ws, f.y, acc[8 * q + 2 * e + 1]);
+                }
+              }
+            }
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+              *(float4*)(hKr + cb * 32 + e) = make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
+          }
         }
         tc::tmem_wait_st();
       }
-      gsync();  // the C^T operand of a new request is complete
       if (new_req) {
         // C . B^T of the request (entries s <= t): warp gw takes s = gw mod 4; lane l
         // holds n = 4l .. 4l + 3 of B_s (registers) and reads those of C_t
@@ -347,56 +432,36 @@ __global__ void __launch_bounds__(THREADS, 1) ssd_tc_kernel(const __grid_constan
             v = fmaf(cv.w, b23.y, v);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            if (lane == 0) gCB[tt * KMAX + ss] = v;
+            if (lane == 0) gCB[tt * NT + ss] = v;
           }
         }
       }
-      // the tile's heads: dt, cum = inclusive scan of dt A_h (segmented, 16 lanes), exp(cum)
-      if (tid < 32) {
-        float d = sizeof(TDT) == 2 ? __bfloat162float(__ushort_as_bfloat16((unsigned short)draw_bits))
-                                   : __uint_as_float(draw_bits);
-        if (dlive && a.dt_bias) d = softplus(d + __uint_as_float(dbias_bits));
-        const float dA = __uint_as_float(dA_bits), dD = __uint_as_float(dD_bits);
-        float cum = dlive ? d * dA : 0.f;
-#pragma unroll
-        for (int o = 1; o < 16; o <<= 1) {
-          const float v = __shfl_up_sync(0xffffffffu, cum, o, 16);
-          if (dtt >= o) cum += v;
-        }
-        if (dlive) {
-          gDt[dh * KMAX + dtt] = d;
-          gDt[(HPT_MAX + dh) * KMAX + dtt] = cum;
-          gE[dh * (KMAX + 1) + dtt] = expf(cum);
-          if (dtt == 0) gE[dh * (KMAX + 1) + KMAX] = dD;
-        }
-      }
-      // x of this thread's row (zero past K)
-#pragma unroll
-      for (int tt = 0; tt < KMAX; ++tt)
-        gX[tt * ROWS + row] = tt < K ? __bfloat162float(__ushort_as_bfloat16((unsigned short)xv[tt])) : 0.f;
-      gsync();
+      gsync();  // C . B^T complete
       // L^T[s][t] = (C_t . B_s) exp(cum_t - cum_s) dt_s for s <= t, else 0: entry
-      // e = (head, t, s) of a 2 x 16 x 16 grid, four per thread, loads first
+      // e = (head, t, s) of a HPT_MAX x NT x NT grid, loads first
       {
-        constexpr int PER = HPT_MAX * KMAX * KMAX / 128;
-        float cb[PER], ct[PER], cs[PER], dts[PER];
-        bool live[PER];
+        constexpr int PER = HPT_MAX * NT * NT / 128;
 #pragma unroll
-        for (int q = 0; q < PER; ++q) {
-          const int e = tid + 128 * q, hh = e >> 8, tt = (e >> 4) & 15, ss = e & 15;
-          live[q] = hh < hpt && tt < K && ss <= tt;
-          cb[q] = gCB[tt * KMAX + ss];
-          ct[q] = gDt[(HPT_MAX + hh) * KMAX + tt];
-          cs[q] = gDt[(HPT_MAX + hh) * KMAX + ss];
-          dts[q] = gDt[hh * KMAX + ss];
-        }
+        for (int q0 = 0; q0 < PER; q0 += 4) {
+          float cb[4], ct[4], cs[4], dts[4];
+          bool live[4];
 #pragma unroll
-        for (int q = 0; q < PER; ++q) {
-          const int e = tid + 128 * q, hh = e >> 8, tt = (e >> 4) & 15, ss = e & 15;
-          gL[(hh * KMAX + ss) * KMAX + tt] = live[q] ? cb[q] * expf(ct[q] - cs[q]) * dts[q] : 0.f;
+          for (int q = 0; q < 4; ++q) {
+            const int e = tid + 128 * (q0 + q), hh = e / (NT * NT), tt = (e / NT) % NT, ss = e % NT;
+            live[q] = hh < hpt && tt < K && ss <= tt;
+            cb[q] = gCB[tt * NT + ss];
+            ct[q] = gDt[(HPT_MAX + hh) * NT + tt];
+            cs[q] = gDt[(HPT_MAX + hh) * NT + ss];
+            dts[q] = gDt[hh * NT + ss];
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int e = tid + 128 * (q0 + q), hh = e / (NT * NT), tt = (e / NT) % NT, ss = e % NT;
+            gL[(hh * NT + ss) * NT + tt] = live[q] ? cb[q] * expf(ct[q] - cs[q]) * dts[q] : 0.f;
+          }
         }
       }
-      // hi and C^T were written by threads and lo by tcgen05.st; the MMA reads them
+      // C^T was written by threads and lo by tcgen05.st; the MMA reads them
       tc::fence_proxy_async();
       tc::tc_fence_before();
       gsync();
@@ -406,36 +471,38 @@ __global__ void __launch_bounds__(THREADS, 1) ssd_tc_kernel(const __grid_constan
       // y_t = exp(cum_t) (C S^T)_t + sum_{s<=t} L_ts x_s + D_h x_t
       ok = tc::mbar_wait_warp(&acc_full[g], (k >> 1) & 1, err, lim);
       if (!ok) {
-        *s_fail = 1;
-        continue;  // the group (the whole warp: the wait's answer is warp-uniform) leaves after its next barrier
+        failed = true;
+        continue;  // the whole warp (the answer is warp-uniform); the group leaves at its next barrier
       }
       tc::tc_fence_after();
       float dv[NT];
-      tc::tmem_ld16(tmem + lane_off + 256u + (uint32_t)(g * NT), dv);
+      tmem_ld_nt(tmem + lane_off + 256u + (uint32_t)(g * NT), dv);
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&d_free[g]);
       const int h = j * hpt + hl;
-      const float* LTh = gL + hl * KMAX * KMAX;  // [s][t]
-      const float* Eh = gE + hl * (KMAX + 1);
-      float xs[KMAX], acc[KMAX];
+      const float* LTh = gL + hl * NT * NT;  // [s][t]
+      const float* Eh = gE + hl * (NT + 1);
+      // (x past K repeats position K - 1: L is zero in the columns s >= K, and the
+      // positions t >= K are never stored)
+      float acc[NT];
 #pragma unroll
-      for (int s2 = 0; s2 < KMAX; ++s2) xs[s2] = gX[s2 * ROWS + row];
+      for (int tt = 0; tt < NT; ++tt) acc[tt] = fmaf(Eh[tt], dv[tt], Eh[NT] * xval(tt));
 #pragma unroll
-      for (int tt = 0; tt < KMAX; ++tt) acc[tt] = fmaf(Eh[tt], dv[tt], Eh[KMAX] * xs[tt]);
+      for (int s2 = 0; s2 < NT; ++s2) {
+        const float xs = xval(s2);
 #pragma unroll
-      for (int s2 = 0; s2 < KMAX; ++s2)
-#pragma unroll
-        for (int t4 = (s2 & ~3); t4 < KMAX; t4 += 4) {
-          const float4 l4 = *(const float4*)(LTh + s2 * KMAX + t4);  // zero above the diagonal
-          acc[t4 + 0] = fmaf(l4.x, xs[s2], acc[t4 + 0]);
-          acc[t4 + 1] = fmaf(l4.y, xs[s2], acc[t4 + 1]);
-          acc[t4 + 2] = fmaf(l4.z, xs[s2], acc[t4 + 2]);
-          acc[t4 + 3] = fmaf(l4.w, xs[s2], acc[t4 + 3]);
+        for (int t4 = (s2 & ~3); t4 < NT; t4 += 4) {
+          const float4 l4 = *(const float4*)(LTh + s2 * NT + t4);  // zero above the diagonal and past K
+          acc[t4 + 0] = fmaf(l4.x, xs, acc[t4 + 0]);
+          acc[t4 + 1] = fmaf(l4.y, xs, acc[t4 + 1]);
+          acc[t4 + 2] = fmaf(l4.z, xs, acc[t4 + 2]);
+          acc[t4 + 3] = fmaf(l4.w, xs, acc[t4 + 3]);
         }
+      }
       float* yr = a.y + (size_t)c * K * a.y_rs + (size_t)h * P + p;
 #pragma unroll
-      for (int tt = 0; tt < KMAX; ++tt)
+      for (int tt = 0; tt < NT; ++tt)
         if (tt < K) yr[(size_t)tt * a.y_rs] = acc[tt];
     }
   }
@@ -464,15 +531,15 @@ EncodeTiledFn encode_fn_ssd() {
   return fn;
 }
 
-template <typename TDT>
+template <typename TDT, int NT, bool HK>
 bool launch_ssd_tc(const SsdArgs& a, cudaStream_t s) {
   static bool attr_set[64] = {};
   static int n_sm[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    if (cudaFuncSetAttribute(ssd_tc_kernel<TDT>, cudaFuncAttributeMaxDynamicSharedMemorySize, SsdTcLay::SMEM) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(ssd_tc_kernel<TDT, NT, HK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SsdTcLay<NT>::SMEM) != cudaSuccess)
       return false;
     cudaDeviceGetAttribute(&n_sm[dev], cudaDevAttrMultiProcessorCount, dev);
     attr_set[dev] = true;
@@ -496,24 +563,31 @@ bool launch_ssd_tc(const SsdArgs& a, cudaStream_t s) {
   t.n_items = a.C * t.n_tiles;
   const int sms = dev < 64 && n_sm[dev] > 0 ? n_sm[dev] : 148;
   const int grid = t.n_items < sms ? t.n_items : sms;
-  launch_pdl(ssd_tc_kernel<TDT>, grid, THREADS, SsdTcLay::SMEM, s, map, t);
+  launch_pdl(ssd_tc_kernel<TDT, NT, HK>, grid, THREADS, SsdTcLay<NT>::SMEM, s, map, t);
   note_launch();
   return true;
+}
+
+template <int NT, bool HK>
+bool launch_ssd_tc_dt(const SsdArgs& a, cudaStream_t s) {
+  return a.dt_bias ? launch_ssd_tc<bf16, NT, HK>(a, s) : launch_ssd_tc<float, NT, HK>(a, s);
 }
 
 }  // namespace
 
 bool ssd_tc_supported(int dtype, const SsdArgs& a) {
-  if (dtype != HSPEC_DTYPE_BF16 || !a.h0 || a.hK || a.Q != a.K) return false;
-  if (a.K < 1 || a.K > KMAX || a.N != NMAX || a.C < 1) return false;
+  if (dtype != HSPEC_DTYPE_BF16 || !a.h0 || a.Q != a.K) return false;
+  if (a.K < 1 || a.K > 32 || a.N != NMAX || a.C < 1) return false;
   if (a.P < ROWS / HPT_MAX || ROWS % a.P || a.H % (ROWS / a.P)) return false;
   if (((uintptr_t)a.h0 & 15) || (long)a.C * a.H * a.P > 0x7fffffffL) return false;
   if (((uintptr_t)a.B & 7) || ((uintptr_t)a.Cm & 7) || (a.bc_rs & 3)) return false;  // 8-byte loads
+  if (a.hK && ((uintptr_t)a.hK & 15)) return false;  // float4 stores of the final state
   return true;
 }
 
 bool ssd_tc_launch(const SsdArgs& a, cudaStream_t s) {
-  return a.dt_bias ? launch_ssd_tc<bf16>(a, s) : launch_ssd_tc<float>(a, s);
+  if (a.K <= 16) return a.hK ? launch_ssd_tc_dt<16, true>(a, s) : launch_ssd_tc_dt<16, false>(a, s);
+  return a.hK ? launch_ssd_tc_dt<32, true>(a, s) : launch_ssd_tc_dt<32, false>(a, s);
 }
 
 }  // namespace hspec

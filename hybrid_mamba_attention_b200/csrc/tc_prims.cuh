@@ -125,6 +125,24 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, i
   return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
+// Named barrier `id` over `nthreads` threads (whole warps) that also ORs a predicate:
+// every participating thread gets the same answer, so a decision taken on it (leave a
+// loop) is the same in all of them.  A flag in shared memory read after a plain
+// barrier is not: another thread may set it between two readers' loads.
+template <int ID, int NTHREADS>
+__device__ __forceinline__ bool bar_or(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "n"(ID), "n"(NTHREADS)
+      : "memory");
+  return r != 0;
+}
+
 // 2-D tiled TMA load of box (x = inner coordinate, y = row) into shared memory,
 // completing `bytes` of transaction on `bar`.
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* tm, uint64_t* bar, int x, int y) {

@@ -87,11 +87,12 @@ def test_ssd_scan_matches_sequential_recurrence(H, cuda, name):
 
 
 @pytest.mark.parametrize("name,C,K", [("llama_c32", 8, 16), ("qwen_c128", 3, 16), ("llama_c32", 160, 16),
-                                     ("llama_c32", 5, 7), ("qwen_c128", 2, 1)])
+                                     ("llama_c32", 5, 7), ("qwen_c128", 2, 1), ("llama_c32", 8, 32),
+                                     ("qwen_c128", 3, 24), ("llama_c32", 150, 17)])
 def test_ssd_scan_readout_without_final_state(H, cuda, name, C, K):
-    # Without the final state, one bf16 chunk of K <= 16 positions is evaluated with the
-    # state readout on the tensor cores (tf32 hi + lo split of the fp32 state): it must
-    # still meet the fp32 bound against the sequential recurrence.
+    # One bf16 chunk of K <= 32 positions is evaluated with the state readout on the
+    # tensor cores (tf32 hi + lo split of the fp32 state, N = 16 or 32 positions per
+    # MMA): it must still meet the fp32 bound against the sequential recurrence.
     sh = I.WORKLOADS[name].shapes
     inp = I.make_ssd_inputs(sh, C, K, 31 + C, cuda)
     y, _ = run_ssd(H, sh, inp, K, want_state=False)
@@ -99,6 +100,40 @@ def test_ssd_scan_readout_without_final_state(H, cuda, name, C, K):
     ref_y = oracle.ssd_scan(host(inp["x"])[rows], host(inp["dt"])[rows], host(inp["A"]), host(inp["B"])[rows],
                                host(inp["Cm"])[rows], host(inp["D"]), host(inp["h0"])[rows], want_state=False)
     assert_close(to_np(y[rows]), ref_y, "f32", f"ssd readout {name} C={C} K={K}")
+
+
+@pytest.mark.parametrize("name,C,K", [("llama_c32", 6, 16), ("llama_c32", 4, 32), ("qwen_c128", 3, 21),
+                                     ("llama_c32", 2, 1), ("llama_c32", 150, 16)])
+def test_ssd_tensor_core_scan_with_final_state(H, cuda, name, C, K):
+    # The final state hK = exp(cum_{K-1}) h0 + sum_s exp(cum_{K-1} - cum_s) dt_s x_s B_s^T,
+    # written by the tensor-core kernel's transform threads from the state rows they
+    # already hold, next to y: both at the fp32 bound against the recurrence.
+    sh = I.WORKLOADS[name].shapes
+    inp = I.make_ssd_inputs(sh, C, K, 51 + C, cuda)
+    y, hK = run_ssd(H, sh, inp, K, want_state=True)
+    rows = sample_requests(C, min(C, 4), seed=K)
+    ref_y, ref_h = oracle.ssd_scan(host(inp["x"])[rows], host(inp["dt"])[rows], host(inp["A"]),
+                                   host(inp["B"])[rows], host(inp["Cm"])[rows], host(inp["D"]),
+                                   host(inp["h0"])[rows], want_state=True)
+    assert_close(to_np(y[rows]), ref_y, "f32", f"ssd y {name} C={C} K={K}")
+    assert_close(to_np(hK[rows]), ref_h, "f32", f"ssd hK {name} C={C} K={K}")
+
+
+@pytest.mark.parametrize("K", [1, 16, 32])
+def test_ssd_state_with_every_low_mantissa_bit_set(H, cuda, K):
+    # The tensor-core readout takes the tf32 part of the fp32 state as the tensor core
+    # reads it from shared memory and adds lo = S - (S with its 13 low mantissa bits
+    # cleared) from TMEM.  That is exact only if the tensor core drops those bits (a
+    # rounding tensor core would add up to 2^-10 |S| per product).  States whose 13 low
+    # bits are all set make every product sensitive to it.
+    sh = I.LLAMA
+    inp = I.make_ssd_inputs(sh, 2, K, 61, cuda)
+    bits = inp["h0"].view(torch.int32)
+    inp["h0"] = (bits | 0x1FFF).view(torch.float32)
+    y, _ = run_ssd(H, sh, inp, K)
+    ref = oracle.ssd_scan(host(inp["x"]), host(inp["dt"]), host(inp["A"]), host(inp["B"]), host(inp["Cm"]),
+                          host(inp["D"]), host(inp["h0"]), want_state=False)
+    assert_close(to_np(y), ref, "f32", f"ssd low mantissa bits K={K}")
 
 
 @pytest.mark.parametrize("K,chunks", [(16, (1, 4, 5, 8, 16)), (32, (8, 16, 32)), (7, (3, 7)), (1, (1,))])

@@ -195,11 +195,12 @@ def test_profile_groups_cover_the_step(H, cuda):
     assert prof["attn_paged"][1] == 2 and prof["inject"][1] == 2
 
 
-@pytest.mark.parametrize("C", [1, 8, 32])
+@pytest.mark.parametrize("C", [1, 8, 32, 128])
 def test_stream_k_step_repeats_bitwise(H, cuda, C):
-    # at these batch sizes the projection and MLP GEMMs run stream-K (tiles cut across
-    # CTAs); the partials are summed in segment order by whichever CTA finishes a tile
-    # last, so repeated steps agree bit for bit
+    # at 1-32 requests the projection and MLP GEMMs cut their K loops (stream-K over one
+    # row of tiles, split-K for few tiles); the partials are summed in segment order by
+    # whichever CTA finishes a tile last, so repeated steps agree bit for bit (at 128
+    # requests whole tiles, and the attention's partition, must repeat as well)
     wl = I.full_workload(C, 16)
     st = I.make_step_inputs(wl, cuda)
     a = run_step(H, wl, st, layers=False)
@@ -260,3 +261,37 @@ def test_reduced_vocab_draft_head(H, cuda, C, K):
     check_stagewise(wl, st, out, rows, wh)
     ids = set(wh["draft_to_target"].tolist())
     assert set(host(out["tokens"]).reshape(-1).tolist()) <= ids
+
+
+@pytest.mark.parametrize("C,K", [(1, 16), (32, 16)])
+def test_step_replays_from_a_cuda_graph(H, cuda, C, K):
+    # hspec_draft_step allocates nothing, makes no synchronising call and launches only
+    # on the caller's stream, so after one uncaptured step (which looks up the device
+    # error word and sets the kernels' attributes) a step can be captured into a CUDA
+    # graph; replaying it gives the eager step's outputs bit for bit.
+    wl = I.full_workload(C, K)
+    st = I.make_step_inputs(wl, cuda)
+    sh = wl.shapes
+    dr = H.Drafter(sh, st["weights"])
+    max_pages = max(c["page_table"].shape[1] for c in st["kv"])
+    ws = H.alloc_workspace(dr.workspace_size(C, K, max_pages), cuda)
+    hidden = torch.full((C, K, sh.d), float("nan"), device=cuda)
+    toks = torch.full((C, K), -1, dtype=torch.int32, device=cuda)
+    si = dr.step_in(C, K, st["h_last"], st["ctx_lens"], st["kv"], tokens=st["tokens"])
+    so = H.hspec_step_out(hidden=hidden.data_ptr(), draft_tokens=toks.data_ptr())
+    dr.step(si, so, ws)
+    assert H.hspec_sync_status() == 0, H.hspec_last_error()
+    want_h, want_t = hidden.clone(), toks.clone()
+    hidden.fill_(float("nan"))
+    toks.fill_(-1)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        dr.step(si, so, ws)
+    assert torch.isnan(hidden).all()  # captured, not run
+    for _ in range(2):
+        graph.replay()
+        torch.cuda.synchronize()
+        assert H.hspec_sync_status() == 0, H.hspec_last_error()
+        assert torch.equal(hidden, want_h) and torch.equal(toks, want_t)
+    del graph
+    dr.close()
