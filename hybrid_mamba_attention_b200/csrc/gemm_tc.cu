@@ -102,6 +102,24 @@ __device__ __forceinline__ void epi32(const GemmArgs& g, int m, int nb, float (&
   }
 }
 
+// kEpiRope: rotates columns i0 .. i0 + 31 of a head (v1, i0 < D/2) with their partners
+// i + D/2 (v2) in row m, after rounding both to bf16 (the stored projection), by the
+// angles of the row's (cos, sin) table.
+__device__ __forceinline__ void rope_rotate(const RopeArgs& r, int m, int i0, float (&v1)[32], float (&v2)[32]) {
+  const float4* t = (const float4*)(r.cs + (size_t)m * (r.D / 2) + i0);  // 32 (cos, sin) pairs, 16-byte aligned
+#pragma unroll
+  for (int e = 0; e < 32; e += 2) {
+    const float4 q = __ldg(t + e / 2);
+    const float a0 = __bfloat162float(__float2bfloat16_rn(v1[e])), b0 = __bfloat162float(__float2bfloat16_rn(v2[e]));
+    const float a1 = __bfloat162float(__float2bfloat16_rn(v1[e + 1])),
+                b1 = __bfloat162float(__float2bfloat16_rn(v2[e + 1]));
+    v1[e] = a0 * q.x - b0 * q.y;
+    v2[e] = a0 * q.y + b0 * q.x;
+    v1[e + 1] = a1 * q.z - b1 * q.w;
+    v2[e + 1] = a1 * q.w + b1 * q.z;
+  }
+}
+
 // How the K loop is cut: zk > 0 stream-K chunks of zk K blocks; else `splits` equal K
 // ranges of kps blocks (splits = 1: whole tiles).
 struct KCut {
@@ -437,6 +455,21 @@ __global__ void __launch_bounds__(THREADS, 1)
               *(float2*)(r.y + ((size_t)m * r.K + t0 + t) * r.y_rs + hp0) =
                   make_float2(fmaf(e[t], acc0[t], yv[t].x), fmaf(e[t], acc1[t], yv[t].y));
         }
+      } else if (EPI == kEpiRope) {
+        // heads of D columns, aligned with the tile (D divides BN): chunk pairs (i, i + D/2)
+        const int D = g.rope.D, half = D / 2;
+        for (int h0 = 0; h0 < BN; h0 += D) {
+          for (int q = 0; q < half; q += 32) {
+            float w2[32];
+            tc::tmem_ld32(taddr + h0 + q, v);
+            tc::tmem_ld32(taddr + h0 + half + q, w2);
+            if (!ok || m >= g.M) continue;
+            const int col = n0 + h0 + q;
+            if (col < g.rope.cols) rope_rotate(g.rope, m, q, v, w2);
+            epi32<EPI>(g, m, col, v, u2);
+            epi32<EPI>(g, m, col + half, w2, u2);
+          }
+        }
       } else if (EPI == kEpiArgmax) {
         float best = -INFINITY;
         int bidx = 0x7fffffff;
@@ -471,13 +504,18 @@ __global__ void __launch_bounds__(THREADS, 1)
       // waits (bounded) until all segments of its tile are counted in, then adds their
       // partials in K order -- the same sums whichever CTA takes it.  Every CTA reaches
       // this phase only after its own segments, so no wait depends on a waiting CTA.
+      // kEpiRope: an item is a pair of chunks (i, i + D/2) of one head, summed and rotated
+      // together (cpd chunks per head, hpc pairs per head)
       const int zk = cut.zk, rows_v = min(BM, g.M), nch = ncols_out / 32;
-      const long per_tile = (long)rows_v * nch, n_items = (long)n_tiles * per_tile;
+      const int cpd = EPI == kEpiRope ? g.rope.D / 32 : 1, hpc = cpd / 2;
+      const int n_it = EPI == kEpiRope ? nch / 2 : nch;  // items per row of a tile
+      const long per_tile = (long)rows_v * n_it, n_items = (long)n_tiles * per_tile;
       float v[32], u2[32];
       int waited = -1;
       for (long it = (long)blockIdx.x * 128 + (threadIdx.x - 64); it < n_items; it += (long)gridDim.x * 128) {
         const int t = (int)(it / per_tile), rem = (int)(it - (long)t * per_tile);
-        const int r = rem % rows_v, cc = rem / rows_v;
+        const int r = rem % rows_v, ci = rem / rows_v;
+        const int cc = EPI == kEpiRope ? (ci / hpc) * cpd + ci % hpc : ci;  // (first) chunk of the item
         const int kf = (int)((long)t * num_k / zk), n_seg = (int)(((long)t * num_k + num_k - 1) / zk) - kf + 1;
         if (n_seg == 1) continue;
         if (t != waited) {
@@ -486,6 +524,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = 0.f, u2[i] = 0.f;
+        // kEpiRope: u2 holds the partner chunk cc + hpc; SwiGLU: the up projection
+        const int c2 = EPI == kEpiRope ? cc + hpc : cc + BN / 64;
 #pragma unroll 2
         for (int q = 0; q < n_seg; ++q) {
           const float4* pq = (const float4*)(g.part + (size_t)seg_slot(t, kf + q, zk, num_k) * BM * BN) + r;
@@ -493,13 +533,20 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int i = 0; i < 8; ++i) {
             const float4 a4 = __ldcg(pq + (cc * 8 + i) * BM);
             v[4 * i] += a4.x, v[4 * i + 1] += a4.y, v[4 * i + 2] += a4.z, v[4 * i + 3] += a4.w;
-            if (EPI == kEpiSwiGLU) {
-              const float4 b4 = __ldcg(pq + ((cc + BN / 64) * 8 + i) * BM);
+            if (EPI == kEpiSwiGLU || EPI == kEpiRope) {
+              const float4 b4 = __ldcg(pq + (c2 * 8 + i) * BM);
               u2[4 * i] += b4.x, u2[4 * i + 1] += b4.y, u2[4 * i + 2] += b4.z, u2[4 * i + 3] += b4.w;
             }
           }
         }
-        epi32<EPI>(g, r, t * ncols_out + cc * 32, v, u2);
+        if (EPI == kEpiRope) {
+          const int col = t * ncols_out + cc * 32;
+          if (col < g.rope.cols) rope_rotate(g.rope, r, (cc % cpd) * 32, v, u2);
+          epi32<EPI>(g, r, col, v, u2);
+          epi32<EPI>(g, r, t * ncols_out + c2 * 32, u2, v);
+        } else {
+          epi32<EPI>(g, r, t * ncols_out + cc * 32, v, u2);
+        }
       }
     }
   }
@@ -612,6 +659,11 @@ KCut gemm_kcut(int dtype, GemmEpi epi, int M, int N, int K) {
   if (n_tiles <= 0) return cut;
   if (cdiv(M, BM) == 1) {
     if (n_tiles >= 8 * sms) return cut;
+    // With 64+ rows the fp32 partials of a cut K loop are large (up to 128 KB per
+    // segment); with enough whole tiles to keep HBM busy (each SM streams its weight
+    // tiles well above its share of HBM bandwidth) whole tiles are faster: the SwiGLU
+    // GEMM at 128 rows and 16384 columns measured 77 -> 66 us.
+    if (M >= 64 && n_tiles >= 112) return cut;
     const long waves = cdiv(n_tiles, sms);
     if ((double)n_tiles / (double)(waves * sms) >= 0.92) return cut;
     const long zk = cdiv(n_tiles * num_k, sms);
@@ -636,10 +688,15 @@ size_t gemm_kcut_bytes(int dtype, GemmEpi epi, int M, int N, int K) {
   return 0;
 }
 
+bool gemm_rope_fusable(int dtype, int M, int N, int K, int D) {
+  if (dtype != HSPEC_DTYPE_BF16 || (D != 64 && D != 128)) return false;
+  return gemm_kcut(dtype, kEpiRope, M, N, K).splits == 1;  // whole tiles or stream-K
+}
+
 bool gemm(int dtype, GemmEpi epi, const GemmArgs& g, cudaStream_t s) {
   if (dtype != HSPEC_DTYPE_BF16) {
-    if (epi == kEpiSsdRead) {
-      set_error("the SSD readout epilogue is bf16-only");
+    if (epi == kEpiSsdRead || epi == kEpiRope) {
+      set_error("the SSD readout and RoPE epilogues are bf16-only");
       return false;
     }
     gemm_simt_f32(epi, g, s);
@@ -671,6 +728,7 @@ bool gemm(int dtype, GemmEpi epi, const GemmArgs& g, cudaStream_t s) {
     case kEpiSwiGLU: return launch_tc<kEpiSwiGLU>(g, cut, s, err);
     case kEpiArgmax: return launch_tc<kEpiArgmax>(g, cut, s, err);
     case kEpiSsdRead: return launch_tc<kEpiSsdRead>(g, cut, s, err);
+    case kEpiRope: return launch_tc<kEpiRope>(g, cut, s, err);
   }
   return false;
 }

@@ -2,6 +2,7 @@
 // workspace carving, launch sequencing of the draft step, and status reporting.
 // Every computation runs in this library's kernels; this file only checks
 // arguments and launches.
+#include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
 #include <string.h>
@@ -291,7 +292,7 @@ bool step_fuses_inject(const hspec_cfg* c) {
 
 // Step workspace layout (all sub-buffers 256-byte aligned).
 struct StepPlan {
-  size_t x, xn, big, y, g, h0, attn, pval, pidx, gpart, gcnt, total;
+  size_t x, xn, big, y, g, h0, attn, pval, pidx, gpart, gcnt, rope, total;
   AttnPlan ap;
   int n_parts;
   size_t gpart_bytes;  // partials of the projection / MLP GEMMs with a cut K loop
@@ -327,6 +328,8 @@ StepPlan step_plan(const hspec_cfg* c, int C, int K, int max_pages) {
   s.n_parts = c->vocab > 0 ? cdiv(head_rows, argmax_tile_n(c->dtype)) : 0;
   s.pval = off, off += align256(M * s.n_parts * 4);
   s.pidx = off, off += align256(M * s.n_parts * 4);
+  // RoPE (cos, sin) table of the step's rows, read by the attention projections' epilogue
+  s.rope = off, off += align256(att && (c->flags & HSPEC_FLAG_ROPE) ? M * (size_t)(c->head_dim / 2) * 8 : 0);
   // split-K workspace: the largest need of the step's projection and MLP GEMMs
   {
     const int Mi = (int)M;
@@ -687,6 +690,15 @@ hspec_status hspec_draft_step(hspec_drafter* dr, const hspec_step_in* in, const 
     if (c->vocab > 0) embed_rows(dtype, in->tokens, W.W_lm, c->vocab, x, M, d, err, s);
     else rows_to_f32(dtype, in->x_in, x, (long)M * d, s);
   }
+  // RoPE: in the attention projections' epilogue (bf16, head dim 64 or 128, no split-K),
+  // from one (cos, sin) table per step shared by every attention layer; else the row
+  // kernel after each projection
+  const bool rope = att && (c->flags & HSPEC_FLAG_ROPE) != 0;
+  const bool rope_fused = rope && gemm_rope_fusable(dtype, M, n_qkv, d, Dh);
+  if (rope_fused) {
+    ProfScope p("rope", s);
+    rope_table((float2*)(ws + sp.rope), in->ctx_lens, C, K, Dh, c->rope_theta, s);
+  }
 
   int ai = 0;
   for (int li = 0; li < c->n_layers; ++li) {
@@ -753,12 +765,16 @@ hspec_status hspec_draft_step(hspec_drafter* dr, const hspec_step_in* in, const 
           return HSPEC_ERR_UNSUPPORTED;
       }
     } else {
+      // q, k, v projections; RoPE on q and the block keys in the GEMM's epilogue where the
+      // tensor-core GEMM can take it (the step's (cos, sin) table is written once, below the
+      // embedding), else by the row kernel after it
       {
         ProfScope p("qkv_proj", s);
-        if (!gemm(dtype, kEpiStore, split(gemm_args(M, n_qkv, d, xn, d, L.W_qkv, d, big, n_qkv)), s))
-          return HSPEC_ERR_UNSUPPORTED;
+        GemmArgs gq = split(gemm_args(M, n_qkv, d, xn, d, L.W_qkv, d, big, n_qkv));
+        if (rope_fused) gq.rope = {(const float2*)(ws + sp.rope), Dh, (Hq + Hkv) * Dh};
+        if (!gemm(dtype, rope_fused ? kEpiRope : kEpiStore, gq, s)) return HSPEC_ERR_UNSUPPORTED;
       }
-      if (c->flags & HSPEC_FLAG_ROPE) {
+      if (rope && !rope_fused) {
         ProfScope p("rope", s);
         rope_rows(dtype, big, n_qkv, in->ctx_lens, C, K, Hq + Hkv, Dh, c->rope_theta, s);
       }

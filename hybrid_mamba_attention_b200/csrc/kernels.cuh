@@ -24,6 +24,9 @@ void gated_rmsnorm_rows(int dtype, const float* y, const void* z, long z_stride,
 // position ctx_lens[c] + j.
 void rope_rows(int dtype, void* qkv, long row_stride, const int32_t* ctx_lens, int C, int K,
                int n_heads, int D, float theta, cudaStream_t s);
+// cs[m][i] = (cos, sin) of the RoPE angle of row m = c*K + j, pair i < D/2, at position
+// ctx_lens[c] + j (computed in double, stored as fp32).
+void rope_table(float2* cs, const int32_t* ctx_lens, int C, int K, int D, float theta, cudaStream_t s);
 // tokens[m] = argmax over parts of (pval, pidx)[m][:] (lowest id on ties); top[m] = its value.
 // Per row the max over the partials (lowest id on ties); with `map` (reduced draft
 // head) the token is map[id], checked against [0, vocab) (else -1 and kErrTokenOOB).
@@ -37,6 +40,17 @@ enum GemmEpi : int {
   kEpiSwiGLU = 2,     // out (dtype) = silu(acc(B)) * acc(B2)
   kEpiArgmax = 3,     // (pval, pidx)[m][n_tile] = per-row max / argmax over the tile's columns
   kEpiSsdRead = 4,    // bf16 only, acc = injected state h0: y += decay * (C . h0) (see SsdReadArgs)
+  kEpiRope = 5,       // bf16 only: out (bf16) = acc, with rotate-half RoPE on the heads of columns
+                      // [0, rope.cols) at each row's position (see RopeArgs)
+};
+
+// kEpiRope: in each head of D columns that lies in [0, cols), the pair (i, i + D/2),
+// i < D/2, of row m is rotated by the angle whose (cos, sin) is cs[m * D/2 + i] (the
+// table rope_table() writes: row m is block position m % K of request m / K) after the
+// projection is rounded to bf16 (the stored value), and the result rounded to bf16 again.
+struct RopeArgs {
+  const float2* cs;
+  int D, cols;
 };
 
 // kEpiSsdRead (d_state N = 128, even P): the injection GEMM (row m = request c, column
@@ -69,12 +83,17 @@ struct GemmArgs {
   // epilogue, so the result does not depend on scheduling.
   float* part; int* tile_cnt; size_t part_bytes; int max_tiles;
   SsdReadArgs ssd;             // kEpiSsdRead
+  RopeArgs rope;               // kEpiRope
   unsigned long long wait_ns;  // pipeline waits give up after this long (0: the default)
 };
 // Workspace bytes (partials) that gemm() needs for this shape when it cuts the K loop
 // (stream-K or split-K; 0 for whole tiles); counters: gemm_tile_count().
 size_t gemm_kcut_bytes(int dtype, GemmEpi epi, int M, int N, int K);
 int gemm_tile_count(int dtype, GemmEpi epi, int M, int N);
+
+// Whether gemm(kEpiRope) can run this shape (bf16, head dim 64 or 128, the K loop
+// whole or cut stream-K); otherwise store with kEpiStore and rotate with rope_rows.
+bool gemm_rope_fusable(int dtype, int M, int N, int K, int D);
 
 // Column tile width of the argmax partials (n_parts = ceil(N / argmax_tile_n(dtype))).
 int argmax_tile_n(int dtype);

@@ -217,6 +217,25 @@ __global__ void rope_kernel(T* __restrict__ qkv, long row_stride, const int32_t*
   v[i + half] = from_f<T>((float)(a * sn + b * cs));
 }
 
+// cos and sin of the rotate-half RoPE angle of every (row m = c*K + j, pair i < D/2):
+// pos * theta^(-2i/D) with pos = ctx_lens[c] + j, formed and evaluated in double (as the
+// row kernel above does), stored as fp32 pairs; the attention projection GEMM's
+// epilogue reads them.
+__global__ void rope_table_kernel(float2* __restrict__ cs, const int32_t* __restrict__ ctx_lens, int K, int half,
+                                  double log_theta, long total) {
+  pdl_wait();  // the previous kernel on the stream is complete from here on
+  pdl_trigger();
+  const long idx = blockIdx.x * (long)blockDim.x + threadIdx.x;
+  if (idx >= total) return;
+  const int i = (int)(idx % half);
+  const long m = idx / half;
+  const double pos = (double)ctx_lens[m / K] + (double)(m % K);
+  const double ang = pos * exp(-2.0 * i / (2 * half) * log_theta);
+  double sn, c;
+  sincos(ang, &sn, &c);
+  cs[idx] = make_float2((float)c, (float)sn);
+}
+
 // One warp per row: scans the per-tile partial maxima in column order, keeping
 // the first (lowest id) of equal maxima.
 __global__ void argmax_reduce_kernel(const float* __restrict__ pval, const int32_t* __restrict__ pidx,
@@ -324,6 +343,13 @@ void rope_rows(int dtype, void* qkv, long row_stride, const int32_t* ctx_lens, i
   else
     launch_pdl(rope_kernel<float>, grid, kRowThreads, 0, s, (float*)qkv, row_stride, ctx_lens, K, n_heads, D,
                                                     lt, total);
+  note_launch();
+}
+
+void rope_table(float2* cs, const int32_t* ctx_lens, int C, int K, int D, float theta, cudaStream_t s) {
+  const long total = (long)C * K * (D / 2);
+  const int grid = (int)((total + kRowThreads - 1) / kRowThreads);
+  launch_pdl(rope_table_kernel, grid, kRowThreads, 0, s, cs, ctx_lens, K, D / 2, log((double)theta), total);
   note_launch();
 }
 
