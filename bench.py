@@ -453,19 +453,34 @@ def run_ours(args, rank, world, local):
     e2e = {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4), "wall_ms_per_step": round(e2e_wall_ms, 4)}
 
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        secs, ctx, cores = oracle_one_request(I, wl, runner)
+        cpu = {"value": round(wl.K / secs, 3), "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"1 of {wl.C} requests (ctx {ctx}, K={wl.K}) through the full M,A,M,A step "
+                         f"+ LM head; {secs:.2f} s; requests are independent so C requests take C times as long"}
+
     # concurrency sweep: draft-step latency and drafted tokens/s at C = 1 .. 128 (K = 16;
     # with --sweep also K = 8 and 32), each against the step's roofline.  The main
-    # measurement above is the C = 128, K = 16 point.
+    # measurement above is the C = 128, K = 16 point.  Each other point runs on its own
+    # batch with the weights shared and the headline batch's KV pools and workspace
+    # released first: left resident, 17 GB of unrelated KV slowed the C = 1 step by 8-15%
+    # (page-table reach), which no workload of that size sees.
+    headline_lens = runner.st["ctx_lens"].cpu()
+    weights = runner.st["weights"]
+    runner.close()
+    del runner
+    torch.cuda.empty_cache()
     sweep = []
     for K in (I.FULL_SWEEP_K if args.sweep else (args.K,)):
         for C in I.FULL_SWEEP_C:
             if C == wl.C and K == wl.K:
-                m2, lens2, k2 = ms_max, runner.st["ctx_lens"].cpu(), kernels
+                m2, lens2, k2 = ms_max, headline_lens, kernels
             else:
                 w2 = I.full_workload(C, K, args.draft_vocab)
-                r2 = StepRunner(H, I, w2, dev, weights=runner.st["weights"])
+                r2 = StepRunner(H, I, w2, dev, weights=weights)
                 n2 = max(5, args.steps // 2)
-                m2, _, _ = time_steps(r2, n2, 3, 1)
+                m2, _, _ = time_steps(r2, n2, max(5, args.warmup), 1)
                 p2, _, prof2 = time_steps(r2, n2, 1, 1, profile=True)
                 lens2 = r2.st["ctx_lens"].cpu()
                 k2 = kernel_table(prof2, step_work(wl.shapes, C, K, lens2), n2, p2, peaks)
@@ -477,18 +492,12 @@ def run_ours(args, rank, world, local):
                           "tokens_per_s": round(C * K / (m2 / 1e3), 1),
                           "roofline_us": round(roof_ms * 1e3, 1), "frac_of_roofline": round(roof_ms / m2, 4),
                           "kernels": compact_kernels(k2)})
+    del weights
+    torch.cuda.empty_cache()
 
     # the paged attention alone on the attention-heavy workloads (rank 0, one GPU)
     attn_cfg = attention_configs(H, I, dev, peaks) if (rank == 0 and not args.no_attention_configs) else None
 
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        secs, ctx, cores = oracle_one_request(I, wl, runner)
-        cpu = {"value": round(wl.K / secs, 3), "unit": UNIT, "cores": cores, "kind": "oracle",
-               "sample": f"1 of {wl.C} requests (ctx {ctx}, K={wl.K}) through the full M,A,M,A step "
-                         f"+ LM head; {secs:.2f} s; requests are independent so C requests take C times as long"}
-
-    runner.close()
     if rank == 0:
         line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": round(ms_max, 4), "us_per_step": round(ms_max * 1e3, 1),
