@@ -223,7 +223,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  pdl_wait();  // the previous kernel on the stream is complete from here on
+  // The next kernel may launch now; it waits for this grid before its own dependent
+  // accesses.  This grid's roles wait for the previous one before theirs: the producer
+  // after requesting its first weight tiles, the epilogue before any global access, the
+  // MMA issuer not at all (it only reads shared memory the producer filled).
   pdl_trigger();
 
   if (warp == 0 && lane == 0) {
@@ -231,26 +234,45 @@ __global__ void __launch_bounds__(THREADS, 1)
     tc::tma_prefetch_desc(&tmA);
     tc::tma_prefetch_desc(&tmB);
     if (EPI == kEpiSwiGLU) tc::tma_prefetch_desc(&tmB2);
+    auto load_b = [&](uint8_t* sb, uint64_t* bar, int kt, int n0) {
+      if (EPI == kEpiSwiGLU) {
+        tc::tma_load_2d(sb, &tmB, bar, kt * BK, n0);
+        tc::tma_load_2d(sb + B_BYTES / 2, &tmB2, bar, kt * BK, n0);
+      } else {
+        tc::tma_load_2d(sb, &tmB, bar, kt * BK, n0);
+      }
+    };
     int it = 0;  // stage-ring position, continued across segments (= stages filled)
     bool ok = true;
     SegWalk wk(num_k, n_tiles, cut);
-    int t, k_lo, k_hi;
-    while (ok && wk.next(t, k_lo, k_hi)) {
+    int t = 0, k_lo = 0, k_hi = 0;
+    bool have = wk.next(t, k_lo, k_hi);
+    int kt = k_lo;
+    // The weights never depend on the previous kernel: the first STAGES weight tiles
+    // are requested before waiting for it (on fresh stages), their activation tiles after.
+    int pre_m0[STAGES], pre_kt[STAGES];
+    while (have && it < STAGES) {
+      uint8_t* sa = smem + it * STAGE_BYTES;
+      tc::mbar_arrive_expect_tx(&full[it], STAGE_BYTES);
+      load_b(sa + A_BYTES, &full[it], kt, (t / n_mt) * ncols_out);
+      pre_m0[it] = (t % n_mt) * BM, pre_kt[it] = kt;
+      ++it;
+      if (++kt == k_hi && (have = wk.next(t, k_lo, k_hi))) kt = k_lo;
+    }
+    pdl_wait();  // the previous kernel on the stream is complete from here on
+    for (int j = 0; j < it; ++j) tc::tma_load_2d(smem + j * STAGE_BYTES, &tmA, &full[j], pre_kt[j] * BK, pre_m0[j]);
+    while (ok && have) {
       const int m0 = (t % n_mt) * BM, n0 = (t / n_mt) * ncols_out;
-      for (int kt = k_lo; kt < k_hi; ++kt, ++it) {
+      for (; kt < k_hi; ++kt, ++it) {
         const int s = it % STAGES;
         if (!(ok = tc::mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, err, lim))) break;
         uint8_t* sa = smem + s * STAGE_BYTES;
-        uint8_t* sb = sa + A_BYTES;
         tc::mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
         tc::tma_load_2d(sa, &tmA, &full[s], kt * BK, m0);
-        if (EPI == kEpiSwiGLU) {
-          tc::tma_load_2d(sb, &tmB, &full[s], kt * BK, n0);
-          tc::tma_load_2d(sb + B_BYTES / 2, &tmB2, &full[s], kt * BK, n0);
-        } else {
-          tc::tma_load_2d(sb, &tmB, &full[s], kt * BK, n0);
-        }
+        load_b(sa + A_BYTES, &full[s], kt, n0);
       }
+      if (!ok) break;
+      if ((have = wk.next(t, k_lo, k_hi))) kt = k_lo;
     }
     // no copy may land after the CTA has finished: wait (with the full limit) for the
     // last filling of every stage -- already complete unless a wait above gave up
@@ -288,6 +310,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     tc::mbar_wait(drain, 0, err);
   } else if (warp >= 2) {
     // ---------------------------------------------------------- epilogue
+    pdl_wait();  // the previous kernel on the stream is complete from here on
     const int quarter = warp & 3;  // TMEM lanes this warp may access
     const int row = quarter * 32 + lane;
     int lt = 0;

@@ -28,15 +28,30 @@ static thread_local char g_last_error[512] = "";
 
 void note_launch(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
 
-// Off unless HSPEC_PDL=1: measured on the draft step it was within run-to-run noise at
-// 1-32 requests and about 2% slower at 128 (more overlap under the power cap).
-bool pdl_enabled() {
-  static const bool on = [] {
+// Programmatic dependent launch: HSPEC_PDL=1 or 0 in the environment forces it on or off
+// for every launch.  Otherwise it is on for the draft step's own launches when the batch
+// has at most kPdlMaxRows block rows: with the GEMMs requesting their first weight tiles
+// before the wait, steps at 8-32 requests measured 2-4% faster; at 128 requests (2048
+// rows) there was no consistent gain (round 1 measured 2% slower there without the early
+// weight requests: more overlap under the power cap).
+constexpr int kPdlMaxRows = 1024;
+static thread_local bool t_step_pdl = false;
+static int pdl_env() {  // -1 unset, 0 off, 1 on
+  static const int mode = [] {
     const char* e = getenv("HSPEC_PDL");
-    return e && e[0] == '1';
+    return e && (e[0] == '0' || e[0] == '1') ? e[0] - '0' : -1;
   }();
-  return on;
+  return mode;
 }
+bool pdl_enabled() {
+  const int env = pdl_env();
+  return env >= 0 ? env == 1 : t_step_pdl;
+}
+// Scope of one draft step's launches.
+struct StepPdl {
+  explicit StepPdl(int rows) { t_step_pdl = rows <= kPdlMaxRows; }
+  ~StepPdl() { t_step_pdl = false; }
+};
 
 void set_error(const char* fmt, ...) {
   va_list ap;
@@ -657,6 +672,7 @@ hspec_status hspec_draft_step(hspec_drafter* dr, const hspec_step_in* in, const 
   cudaStream_t s = (cudaStream_t)stream;
   uint8_t* ws = (uint8_t*)workspace;
   const int M = C * K;
+  StepPdl pdl_scope(M);
   const int dtype = c->dtype;
   const float eps = c->norm_eps;
   const int H = c->n_ssm_heads, P = c->ssm_head_dim, N = c->d_state, HP = H * P;
