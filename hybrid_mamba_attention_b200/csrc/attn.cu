@@ -173,8 +173,8 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(AttnArgs a) {
   const bool valid = live && ctx >= 0 && ctx <= a.max_pages * a.page_size;
   // Partials of the row: q = 0 .. ns - 1 at rows base0 + q * stride.
   //   fp32 path: one per split of (c, g).
-  //   tensor-core path: the sequence (c, rb, g) holds t_seq tiles from tile s0 of the
-  //   line cut into chunks of Z tiles; its piece p in chunk k0 + p has slot
+  //   tensor-core path: the sequence (c, rb, g) holds t_seq tiles from unit s0 of the
+  //   line cut into chunks of Z units; its piece p in chunk k0 + p has slot
   //   c * spr + rb * Hkv + g + k0 + p, two halves each, so q = 2 p + half.  Half h of
   //   a piece holds its tiles of parity h: it exists iff the piece has more than h
   //   tiles (a missing partial is never written, and its weight is 0).
@@ -189,8 +189,10 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(AttnArgs a) {
     Z = a.sched[2];
     stride = R < kAttnTcRows ? R : kAttnTcRows;
     if (valid) {
-      t_seq = (off[c + 1] - off[c]) / spr;
-      s0 = off[c] + r * t_seq;
+      // the sequence's units on the line: kAttnSeqUnits start units, then its tiles
+      const int tw = (off[c + 1] - off[c]) / spr;
+      t_seq = tw - kAttnSeqUnits;
+      s0 = off[c] + r * tw + kAttnSeqUnits;
       k0 = s0 / Z;
       ns = t_seq > 0 ? 2 * ((s0 + t_seq - 1) / Z - k0 + 1) : 0;
     }

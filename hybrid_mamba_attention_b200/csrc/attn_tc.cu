@@ -5,15 +5,18 @@
 //
 // Work partition (stream-K over the tile space): each (request c, row block rb, kv
 // head g) is a sequence of t_c 64-token tiles (the context's, then the block's own
-// keys), and the sequences are laid end to end, request by request.  A one-CTA
-// schedule kernel sums them (T tiles) and cuts the line into chunks of Z = ceil(T /
-// grid) tiles, one per CTA of the persistent kernel (or of a requested length, CTA b
-// then taking chunks b, b + grid, ...), so that every SM streams the same number of
-// tiles whatever the mix of context lengths.  A CTA walks its chunk as pieces, one
-// per sequence it crosses; the piece of sequence q in chunk k writes its partial to
-// slot q + k (distinct for every piece: a later sequence never starts in an earlier
-// chunk), and the merge kernel finds the pieces of a sequence from T, Z and the
-// request's tile offset.  The R = K*G queries of kv head g (block
+// keys).  On a line of work units the sequences are laid end to end, request by
+// request, each as kAttnSeqUnits units for its start (a piece's Q load, the page ids of
+// its first tiles and its partials cost about as much as four tiles) followed by one
+// unit per tile.  A one-CTA schedule kernel sums them (T units) and cuts the line into
+// chunks of Z = ceil(T / grid) units, one per CTA of the persistent kernel (or of a
+// requested length, CTA b then taking chunks b, b + grid, ...), so that every SM gets
+// the same work whatever the mix of context lengths: with tiles alone a CTA whose
+// chunk crossed many short sequences finished up to 20% after the others.  A CTA
+// walks its chunk as pieces, one per sequence whose tiles it crosses; the piece of
+// sequence q in chunk k writes its partial to slot q + k (distinct for every piece: a
+// later sequence never starts in an earlier chunk), and the merge kernel finds the
+// pieces of a sequence from T, Z and the request's offset on the line.  The R = K*G queries of kv head g (block
 // position j, query head g*G + i) form the rows of a 128-row Q tile, so every K/V
 // byte read from HBM feeds all R queries; with R <= 64 the rows are spread 16 per
 // 32-lane TMEM quarter so that all four SM sub-partitions share the softmax work;
@@ -47,9 +50,12 @@
 //               TMEM only when the running max grows by more than 8, after the group's
 //               previous P.V.
 //               Each group keeps its own (m, l, O) per piece and writes its own partial
-//               when its last tile of the piece is done -- the half of the piece made of
-//               its even (or odd) tiles, so the arithmetic does not depend on timing;
-//               the merge kernel combines the halves and the pieces.
+//               -- the half of the piece made of its even (or odd) tiles, so the
+//               arithmetic does not depend on timing -- while it works on its next tile:
+//               after that tile's softmax and before its P.V may overwrite O_w, so that
+//               the wait for the piece's last P.V (queued behind the Q.K^T products of
+//               the tiles ahead) overlaps useful work.  The merge kernel combines the
+//               halves and the pieces.
 // Every wait gives up after a time bound and sets the device error word.
 #include <stdint.h>
 
@@ -114,16 +120,17 @@ struct TcMaps {
   CUtensorMap k, v, kb, vb, q;
 };
 
-// Tiles of each sequence of a request: its context tiles and the block's own keys
-// (nbt tiles); none for an invalid context length (the merge writes zero rows).
-__device__ __forceinline__ int seq_tiles(int ctx, long max_ctx, int nbt) {
-  return ctx < 0 || ctx > max_ctx ? 0 : (ctx + TT - 1) / TT + nbt;
+// Units of each sequence of a request on the partition's line: kAttnSeqUnits for its
+// start, then one per tile -- its context tiles and the block's own keys (nbt tiles);
+// none for an invalid context length (the merge writes zero rows).
+__device__ __forceinline__ int seq_units(int ctx, long max_ctx, int nbt) {
+  return ctx < 0 || ctx > max_ctx ? 0 : kAttnSeqUnits + (ctx + TT - 1) / TT + nbt;
 }
 
-// One CTA: off[c] = tiles of all sequences of requests before c (spr sequences of
-// seq_tiles each per request), off[C] = T; sched[1] = T, sched[2] = Z (the chunk
-// length: ceil(T / grid), or z_req; at least ceil(T / max_chunks)), sched[3] = the
-// number of chunks.
+// One CTA: off[c] = units of all sequences of requests before c (spr sequences of
+// seq_units each per request), off[C] = T; sched[1] = T, sched[2] = Z (the chunk
+// length in units: ceil(T / grid), or z_req; at least ceil(T / max_chunks)),
+// sched[3] = the number of chunks.
 __global__ void __launch_bounds__(1024) attn_sched_kernel(const int32_t* ctx_lens, int C, long max_ctx, int nbt,
                                                           int spr, int grid, int z_req, int max_chunks, int* sched,
                                                           int* off, int* err) {
@@ -136,7 +143,7 @@ __global__ void __launch_bounds__(1024) attn_sched_kernel(const int32_t* ctx_len
   for (int c = c0; c < c1; ++c) {
     const int ctx = ctx_lens[c];
     if (ctx < 0 || ctx > max_ctx) flag_error(err, kErrCtxOOB);
-    sum += seq_tiles(ctx, max_ctx, nbt) * spr;
+    sum += seq_units(ctx, max_ctx, nbt) * spr;
   }
   part[threadIdx.x] = sum;
   __syncthreads();
@@ -149,7 +156,7 @@ __global__ void __launch_bounds__(1024) attn_sched_kernel(const int32_t* ctx_len
   int run = threadIdx.x > 0 ? part[threadIdx.x - 1] : 0;
   for (int c = c0; c < c1; ++c) {
     off[c] = run;
-    run += seq_tiles(ctx_lens[c], max_ctx, nbt) * spr;
+    run += seq_units(ctx_lens[c], max_ctx, nbt) * spr;
   }
   if (threadIdx.x == 1023) {
     const int T = part[1023];
@@ -268,6 +275,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       return lo;
     };
+    // the K/V tiles are read once: first out of L2, so that the pieces' partials stay
+    // there until the end of the kernel reads them back
+    const uint64_t once = tc::l2_evict_first();
     int k = blockIdx.x;  // this CTA's chunk
     int pos = k < n_chunks ? k * Z : 0, end = k < n_chunks ? min(T, pos + Z) : 0;
     int c = pos < end ? locate(pos) : 0;
@@ -283,22 +293,35 @@ __global__ void __launch_bounds__(THREADS, 1)
         stopped = true;
         break;
       }
-      if (pos >= end) {  // the CTA's next chunk
-        k += gridDim.x;
-        if (k >= n_chunks) break;
-        pos = k * Z;
-        end = min(T, pos + Z);
-        c = locate(pos);
+      // the next piece: tiles [lt0, lt0 + n_tiles) of sequence r = rb Hkv + g of
+      // request c within the chunk (a span that holds only a sequence's start units
+      // has no tiles and is passed over without a piece)
+      int r = 0, lt0 = 0, n_tiles = 0;
+      bool done = false;
+      while (n_tiles == 0) {
+        if (pos >= end) {  // the CTA's next chunk
+          k += gridDim.x;
+          if (k >= n_chunks) {
+            done = true;
+            break;
+          }
+          pos = k * Z;
+          end = min(T, pos + Z);
+          c = locate(pos);
+        }
+        while (off[c + 1] <= pos) ++c;
+        // units [u0, u1) of the sequence: kAttnSeqUnits start units, then its tiles
+        const int tw = (off[c + 1] - off[c]) / spr;
+        const int rel = pos - off[c];
+        r = rel / tw;
+        const int u0 = rel - r * tw, u1 = min(tw, u0 + (end - pos));
+        pos += u1 - u0;
+        lt0 = max(u0 - kAttnSeqUnits, 0);
+        n_tiles = max(u1 - kAttnSeqUnits - lt0, 0);
       }
-      while (off[c + 1] <= pos) ++c;
-      // piece: tiles [lt0, lt0 + n_tiles) of sequence r = rb Hkv + g of request c
-      const int t_seq = (off[c + 1] - off[c]) / spr;
-      const int rel = pos - off[c];
-      const int r = rel / t_seq, lt0 = rel - r * t_seq;
-      const int n_tiles = min(t_seq - lt0, end - pos);
+      if (done) break;
       const int g = r % a.Hkv, rb = r / a.Hkv;
       const int pslot = c * spr + r + k;  // partial slot of the piece
-      pos += n_tiles;
       const int ctx = a.ctx_lens[c];
       const int ct = (ctx + TT - 1) / TT;  // context tiles of the sequence
       const int slot = seq & 1;
@@ -375,15 +398,15 @@ __global__ void __launch_bounds__(THREADS, 1)
             const int tt = t0 + 16 * q16;
             const int z = pg * a.page_size + (pshift >= 0 ? (tt & (a.page_size - 1)) : tt % a.page_size);
             if (k_box)
-              tc::tma_load_3d(kd + bk * L::KV_BLK + q16 * 2048, &maps.k, &kv_full[s], bk * 64, g, z);
+              tc::tma_load_3d_hint(kd + bk * L::KV_BLK + q16 * 2048, &maps.k, &kv_full[s], bk * 64, g, z, once);
             else
-              tc::tma_load_4d(vd + q16 * L::V_PAGE, &maps.v, &kv_full[s], 0, z, g, 0);
+              tc::tma_load_4d_hint(vd + q16 * L::V_PAGE, &maps.v, &kv_full[s], 0, z, g, 0, once);
           } else {
             const int row0 = c * a.K + bt * TT;
             if (k_box)
-              tc::tma_load_3d(kd + bk * L::KV_BLK, &maps.kb, &kv_full[s], bk * 64, g, row0);
+              tc::tma_load_3d_hint(kd + bk * L::KV_BLK, &maps.kb, &kv_full[s], bk * 64, g, row0, once);
             else
-              tc::tma_load_4d(vd + q16 * L::V_PAGE, &maps.vb, &kv_full[s], 0, row0 + 16 * q16, g, 0);
+              tc::tma_load_4d_hint(vd + q16 * L::V_PAGE, &maps.vb, &kv_full[s], 0, row0 + 16 * q16, g, 0, once);
           }
         }
         __syncwarp();
@@ -530,6 +553,36 @@ __global__ void __launch_bounds__(THREADS, 1)
     constexpr int OCB = SP ? D / 64 : D / 32;  // 32-column chunks of O per thread
     auto o_col = [&](int cb) { return SP ? hf * (D / 2) + cb * 32 : cb * 32; };
 
+    // The partial of a piece's half: O_w as the P.V of tile ti (the half's last) left
+    // it, with its (m, l), into rows `base` of the workspace.  The parity of s_free is
+    // unambiguous as for the rescale below: the phase before (tile ti - NSB) completed
+    // before the Q.K^T of tile ti, and the one after needs the P of tile ti + NSB, which
+    // this group writes only after this call.
+    auto write_partial = [&](int ti, size_t base, float pm, float plsum, bool act) -> bool {
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(&s_free[ti & (NSB - 1)], (ti / NSB) & 1, err, lim))) return false;
+      tc::tc_fence_after();
+#pragma unroll
+      for (int cb = 0; cb < OCB; ++cb) {
+        float v[32];
+        o_ld(cb, v);
+        if (act) {
+          float* o = a.ws_acc + base * D + o_col(cb);
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) *(float4*)(o + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+        }
+      }
+      if (act && hf == 0) {
+        a.ws_ml[base * 2] = pm;
+        a.ws_ml[base * 2 + 1] = plsum;
+      }
+      return true;
+    };
+    // a partial not yet written: the group's last tile of its previous piece
+    bool pend = false, pend_act = false;
+    int pend_i = 0;
+    size_t pend_base = 0;
+    float pend_m = 0.f, pend_l = 0.f;
+
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     for (int i = wg; ok; i += 2) {
@@ -648,42 +701,41 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         tc::fence_proxy_async();
       }
+      if (pend) {
+        // the previous piece's partial, now that the P of this tile (the first of a new
+        // piece for this group, so no rescale above) is written and before its P.V may
+        // overwrite O_w: by now the P.V of that piece's last tile has left the tensor
+        // pipe's queue, so the wait for it overlaps this tile's softmax
+        pend = false;
+        ok = write_partial(pend_i, pend_base, pend_m, pend_l, pend_act);
+        if (!ok) break;
+      }
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&p_full[b]);
 
       if (local >= n_tiles - 2) {
-        // this group's last tile of the piece: write its partial (half of the piece)
-        // this tile's P.V (same argument for the parity of s_free as above)
-        ok = __all_sync(0xffffffffu, tc::mbar_wait(&s_free[b], (i / NSB) & 1, err, lim));
-        if (!ok) break;
-        tc::tc_fence_after();
-        // half (local & 1): the piece's even or odd tiles, whichever group ran them,
-        // so the result does not depend on timing; rows of the row block
-        const size_t base = ((size_t)pslot * 2 + (local & 1)) * RB + r_local;
-#pragma unroll
-        for (int cb = 0; cb < OCB; ++cb) {
-          float v[32];
-          o_ld(cb, v);
-          if (active) {
-            float* o = a.ws_acc + base * D + o_col(cb);
-#pragma unroll
-            for (int e = 0; e < 32; e += 4) *(float4*)(o + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
-          }
-        }
-        if (active && hf == 0) {
-          a.ws_ml[base * 2] = m_used;
-          a.ws_ml[base * 2 + 1] = l;
-        }
-        tc::tc_fence_before();
+        // this group's last tile of the piece: its partial is the half of the piece
+        // made of tiles of parity (local & 1), whichever group ran them, so the result
+        // does not depend on timing; rows of the row block.  It is written during the
+        // group's next tile, or after the loop.
+        pend = true;
+        pend_i = i;
+        pend_base = ((size_t)pslot * 2 + (local & 1)) * RB + r_local;
+        pend_m = m_used;
+        pend_l = l;
+        pend_act = active;
       }
     }
+    if (pend && ok) write_partial(pend_i, pend_base, pend_m, pend_l, pend_act);
+    tc::tc_fence_before();
   }
   __syncthreads();
   if (warp == QK_WARP) {
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, L::TMEM_COLS);
   }
+
 }
 
 // ------------------------------------------------------------------ host side

@@ -126,6 +126,11 @@ constexpr int kAttnTcRows = 128; // query rows per row block (MMA M) of that pat
 // chunks of the tensor-core path's tile-space partition: one per SM (auto), or of an
 // explicitly requested length, at most this many (which bounds the partial workspace)
 constexpr int kAttnMaxChunksAuto = 256;
+// On the line that the tensor-core path cuts into chunks, a sequence takes this many
+// units for its start (the Q load, the page ids of its first tiles, the partials at its
+// end: together about as long as four tiles), then one unit per 64-key tile, so that
+// the chunks balance tiles and sequence starts together.
+constexpr int kAttnSeqUnits = 6;
 constexpr int kAttnMaxChunksExplicit = 2048;
 struct AttnArgs {
   int C, K, Hq, Hkv, D;

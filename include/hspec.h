@@ -91,9 +91,11 @@ typedef struct hspec_cfg {
   float norm_eps;                   /* RMSNorm epsilon                                     */
   int ssd_chunk;                    /* SSD chunk length Q (0 = whole block in one chunk)   */
   int attn_split_tokens;            /* split-KV partition length in tokens, multiple of 16 (0 = auto):
-                                       fp32, tokens per split of a request; bf16, tiles per chunk of
-                                       the even tile-space partition (rounded up to 64 tokens; at
-                                       most 2048 chunks) -- auto: one chunk per SM */
+                                       fp32, tokens per split of a request; bf16, the length of a
+                                       chunk of the tile-space partition in units of 64 tokens
+                                       (rounded up), where a sequence counts one unit per 64-key
+                                       tile plus 4 for its start; at most 2048 chunks -- auto: one
+                                       chunk per SM */
   int draft_vocab;                  /* reduced draft head rows (0 = the full vocab head):    */
                                     /* logits over W_lm_draft, draft token = the mapped id  */
   long long wait_limit_ns;          /* a pipeline wait in a tensor-core kernel (an mbarrier

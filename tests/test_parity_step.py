@@ -109,9 +109,10 @@ def check_stagewise(wl, st, out, rows, wh):
     return errs
 
 
-def check_end_to_end(wl, st, out, rows, wh, bound):
+def check_end_to_end(wl, st, out, rows, wh, bound, ref=None):
     sh = wl.shapes
-    ref = oracle_step_for(sh, wh, st, rows)
+    if ref is None:
+        ref = oracle_step_for(sh, wh, st, rows)
     e = rel_rms(to_np(out["hidden"][rows]), ref["hidden"])
     msg = f"{wl.name}: end-to-end hidden max-abs/rms {e:.3e}"
     if sh.vocab:
@@ -231,10 +232,12 @@ def test_fused_injection_step_matches_oracle(H, cuda, C, K):
 def test_fused_injection_readout_equals_stored_h0(H, cuda, C, K):
     # bf16 step with HSPEC_FLAG_FUSE_INJECT: the injection GEMM adds exp(cum_t) C_t . h0
     # to the zero-state scan from its accumulator (h0 never stored); by default h0 is
-    # stored and read by the scan.  Same arithmetic up to evaluation order: the first (Mamba) layer, fed the
-    # same input, agrees to the bf16 bound; later layers inherit the bf16 rounding drift
-    # of the module docstring, bounded end to end by DRIFT_BOUND.  (Each path is also
-    # checked layer by layer against the oracle in the tests above.)
+    # stored and read by the scan.  Same arithmetic up to evaluation order: the first
+    # (Mamba) layer, fed the same input, agrees to the bf16 bound.  Later layers inherit
+    # the bf16 rounding drift of the module docstring, and two orders of evaluation can
+    # drift apart by up to the sum of their distances from the exact result, so the
+    # final hidden states are each held to the drift bound against the oracle (on the
+    # same sampled requests) rather than to it against each other.
     wl = I.full_workload(C, K)
     st = I.make_step_inputs(wl, cuda)
     a = run_step(H, wl, st, fuse_inject=True)
@@ -244,8 +247,11 @@ def test_fused_injection_readout_equals_stored_h0(H, cuda, C, K):
         print(f"C={C} K={K} layer {li}: fused vs stored h0 max-abs/rms {e:.3e}")
         if li == 0:
             assert e <= BF16_TOL
-    e = rel_rms(to_np(a["hidden"]), to_np(b["hidden"]))
-    assert np.isfinite(to_np(a["hidden"])).all() and e <= DRIFT_BOUND, e
+    rows = sample_requests(wl.C, 2, seed=wl.seed)
+    wh = host_weights(st["weights"])
+    ref = oracle_step_for(wl.shapes, wh, st, rows)
+    for out in (a, b):
+        check_end_to_end(wl, st, out, rows, wh, DRIFT_BOUND, ref=ref)
 
 
 @pytest.mark.parametrize("C,K", [(1, 16), (8, 16), (128, 16)])
