@@ -230,12 +230,13 @@ def step_roofline_ms(sh, C, K, ctx_lens, peaks):
 
 # DRAM bytes (read + write) per algorithmic byte of the paged-attention kernel, from
 # one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum) of the current
-# attn_tc_kernel at Llama-3-8B shapes, C=32, ctx U[512,8192]: 678.4 MB for 658.3 MB of
-# algorithmic bytes as step_work counts them (K/V, q, output, block k/v).  The step's
-# attention launch is too large to capture; its traffic is this ratio times its
-# algorithmic bytes (traffic grows with the K/V read).  None whenever the kernel has
-# changed since the last capture.
-ATTN_TRAFFIC_PER_BYTE = 1.0306
+# attn_tc_kernel at Llama-3-8B shapes, C=32, ctx U[512,8192]: 664.1 MB (657.4 read, 6.8
+# written) for 658.3 MB of algorithmic bytes as step_work counts them (K/V, q, output,
+# block k/v).  The K/V tiles are loaded evict-first, so the pieces' partials stay in L2
+# during the kernel and the merge reads them there.  The step's attention launch is too
+# large to capture; its traffic is this ratio times its algorithmic bytes (traffic grows
+# with the K/V read).  None whenever the kernel has changed since the last capture.
+ATTN_TRAFFIC_PER_BYTE = 1.0089
 
 
 def roofline_of(name, work, avg_ms, peaks, traffic=None, sustained=True):
