@@ -163,7 +163,10 @@ __global__ void __launch_bounds__(THREADS, 1) ssd_tc_kernel(const __grid_constan
   uint64_t* lo_full = a_empty + NSTAGE;
   uint64_t* acc_full = lo_full + 2;                    // [2] MMAs of the accumulator's tile done
   uint64_t* d_free = acc_full + 2;                     // [2] epilogue has read the accumulator
-  uint64_t* drain = d_free + 2;
+  // [2] tile k: its state tile has landed and the C^T operand is written, so the MMAs
+  // of the state's tf32 part may start before lo is ready
+  uint64_t* hi_ready = d_free + 2;
+  uint64_t* drain = hi_ready + 2;
   uint32_t* tmem_slot = (uint32_t*)(drain + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -185,6 +188,8 @@ __global__ void __launch_bounds__(THREADS, 1) ssd_tc_kernel(const __grid_constan
     }
     tc::mbar_init(&lo_full[0], 4);
     tc::mbar_init(&lo_full[1], 4);
+    tc::mbar_init(&hi_ready[0], 4);
+    tc::mbar_init(&hi_ready[1], 4);
     tc::mbar_init(drain, 1);
     tc::fence_mbar_init();
   }
@@ -224,18 +229,25 @@ __global__ void __launch_bounds__(THREADS, 1) ssd_tc_kernel(const __grid_constan
         const int k = i - i0, st = k % NSTAGE, db = k & 1;
         // accumulator db is free once the epilogue of tile k - 2 has read it
         if (k >= 2 && !tc::mbar_wait(&d_free[db], ((k >> 1) - 1) & 1, err, lim)) break;
-        if (!tc::mbar_wait(&lo_full[k & 1], (k >> 1) & 1, err, lim)) break;
+        // the state's tf32 part (hi, read from shared memory as it landed) as soon as the
+        // C^T operand is there; lo once the transform has written it to TMEM
+        if (!tc::mbar_wait(&hi_ready[k & 1], (k >> 1) & 1, err, lim)) break;
         tc::tc_fence_after();
         const uint32_t st_addr = tc::smem_u32(sA + st * TILE_BYTES);
         const uint32_t lo = tmem + (uint32_t)(128 * (k & 1));
         const uint32_t d = tmem + 256u + (uint32_t)(db * NT);
+        auto bdesc = [&](int kb) {
+          return tc::sdesc_k128(b_base + (uint32_t)((kb >> 2) * NT * 128 + (kb & 3) * 32));
+        };
 #pragma unroll
         for (int kb = 0; kb < NMAX / 8; ++kb) {
           const uint32_t aoff = (uint32_t)((kb >> 2) * ROWS * 128 + (kb & 3) * 32);
-          const uint64_t bdesc = tc::sdesc_k128(b_base + (uint32_t)((kb >> 2) * NT * 128 + (kb & 3) * 32));
-          mma_tf32(d, tc::sdesc_k128(st_addr + aoff), bdesc, idesc, kb > 0);  // hi: the tf32 part of S
-          mma_tf32_ts(d, lo + (uint32_t)(kb * 8), bdesc, idesc, 1u);
+          mma_tf32(d, tc::sdesc_k128(st_addr + aoff), bdesc(kb), idesc, kb > 0);
         }
+        if (!tc::mbar_wait(&lo_full[k & 1], (k >> 1) & 1, err, lim)) break;
+        tc::tc_fence_after();
+#pragma unroll
+        for (int kb = 0; kb < NMAX / 8; ++kb) mma_tf32_ts(d, lo + (uint32_t)(kb * 8), bdesc(kb), idesc, 1u);
         tc::mma_commit(&acc_full[db]);
         tc::mma_commit(&a_empty[st]);
       }
@@ -250,7 +262,6 @@ __global__ void __launch_bounds__(THREADS, 1) ssd_tc_kernel(const __grid_constan
     const int row = quarter * 32 + lane;         // the state row (TMEM lane) of this thread
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const int hl = row / P, p = row % P;
-    const int gw = (warp - 2) & 3;               // warp within the group
     constexpr bool want_hK = HK;
     const TDT* dtp = (const TDT*)a.dt;
     const bf16* xg = (const bf16*)a.x;
@@ -278,13 +289,21 @@ __global__ void __launch_bounds__(THREADS, 1) ssd_tc_kernel(const __grid_constan
       // the tile's global loads first: x of this thread's row at every position (rows
       // past K re-read row K - 1 and count as zero), and (lane hh * NT + tt of the
       // group's first warps) dt of head hh at position tt
-      uint32_t xw[NT / 2];  // bf16 pairs: position 2i in the low half, 2i + 1 in the high half
+      // (NT = 16: the raw bits first, one register each, so that no load waits for
+      // another's result; packed after the tile's waits)
+      uint32_t xw[NT / 2] = {};  // bf16 pairs: position 2i in the low half, 2i + 1 in the high half
+      uint32_t xraw[NT == 16 ? NT : 1];
       {
         const bf16* xr = xg + (size_t)c * K * a.x_rs + (size_t)(j * hpt) * P + row;
+        if constexpr (NT == 16) {
 #pragma unroll
-        for (int tt = 0; tt < NT; tt += 2)
-          xw[tt / 2] = (uint32_t)ldg_u16(xr + (size_t)(tt < K ? tt : K - 1) * a.x_rs) |
-                       ((uint32_t)ldg_u16(xr + (size_t)(tt + 1 < K ? tt + 1 : K - 1) * a.x_rs) << 16);
+          for (int tt = 0; tt < NT; ++tt) xraw[tt] = ldg_u16(xr + (size_t)(tt < K ? tt : K - 1) * a.x_rs);
+        } else {
+#pragma unroll
+          for (int tt = 0; tt < NT; tt += 2)
+            xw[tt / 2] = (uint32_t)ldg_u16(xr + (size_t)(tt < K ? tt : K - 1) * a.x_rs) |
+                         ((uint32_t)ldg_u16(xr + (size_t)(tt + 1 < K ? tt + 1 : K - 1) * a.x_rs) << 16);
+        }
       }
       // x at position s (fp32; the bf16 bits in the upper half of a word)
       auto xval = [&](int s2) {
@@ -308,6 +327,10 @@ __global__ void __launch_bounds__(THREADS, 1) ssd_tc_kernel(const __grid_constan
       if (ok && new_req && k >= 1) ok = tc::mbar_wait_warp(&acc_full[(k - 1) & 1], ((k - 1) >> 1) & 1, err, lim);
       if (g == 0 ? tc::bar_or<1, 128>(!ok) : tc::bar_or<2, 128>(!ok)) break;  // the group's barrier
       tc::tc_fence_after();
+      if constexpr (NT == 16) {
+#pragma unroll
+        for (int tt = 0; tt < NT; tt += 2) xw[tt / 2] = xraw[tt] | (xraw[tt + 1] << 16);
+      }
       if (new_req) {
         // C^T operand: row tt (position) of 128-byte column blocks, zero past K
         constexpr int PER = NT * NMAX / 4 / 128;  // float4 entries per thread
@@ -326,12 +349,11 @@ __global__ void __launch_bounds__(THREADS, 1) ssd_tc_kernel(const __grid_constan
           *(float4*)(sB + (n4 >> 5) * NT * 128 + tt * 128 + ((ch ^ (tt & 7)) << 4)) =
               make_float4(lo2.x, lo2.y, hi2.x, hi2.y);
         }
-        if constexpr (want_hK) {
-          // B rows of the request (bf16 as stored; positions < K)
-          for (int e = tid; e < K * (NMAX / 4); e += 128) {
-            const int tt = e / (NMAX / 4), n4 = (e % (NMAX / 4)) * 4;
-            *(uint2*)(gBR + (tt * NMAX + n4) * 2) = *(const uint2*)(Bg + (size_t)(c * K + tt) * a.bc_rs + n4);
-          }
+        // B rows of the request (bf16 as stored; positions < K), for C . B^T and the
+        // final state
+        for (int e = tid; e < K * (NMAX / 4); e += 128) {
+          const int tt = e / (NMAX / 4), n4 = (e % (NMAX / 4)) * 4;
+          *(uint2*)(gBR + (tt * NMAX + n4) * 2) = *(const uint2*)(Bg + (size_t)(c * K + tt) * a.bc_rs + n4);
         }
         c_prev = c;
       }
@@ -354,7 +376,9 @@ __global__ void __launch_bounds__(THREADS, 1) ssd_tc_kernel(const __grid_constan
           if (dtt == 0) gE[dh * (NT + 1) + NT] = dD;
         }
       }
-      gsync();  // the C^T operand (and B rows) of a new request, dt and cum are complete
+      tc::fence_proxy_async();  // C^T was written by threads; the MMAs read it
+      gsync();  // the C^T operand and B rows of a new request, dt and cum are complete
+      if (lane == 0) tc::mbar_arrive(&hi_ready[g]);
       // this thread's state row: lo = S - hi into the group's TMEM buffer (free: the
       // group's previous tile finished its MMAs); with a final state also its row of hK
       {
@@ -417,23 +441,28 @@ __global__ void __launch_bounds__(THREADS, 1) ssd_tc_kernel(const __grid_constan
         tc::tmem_wait_st();
       }
       if (new_req) {
-        // C . B^T of the request (entries s <= t): warp gw takes s = gw mod 4; lane l
-        // holds n = 4l .. 4l + 3 of B_s (registers) and reads those of C_t
-        for (int ss = gw; ss < K; ss += 4) {
-          const uint2 r = *(const uint2*)(Bg + (size_t)(c * K + ss) * a.bc_rs + 4 * lane);
-          const float2 b01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.x));
-          const float2 b23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.y));
-          const int n4 = 4 * lane, ch = (n4 & 31) >> 2;
-          for (int tt = ss; tt < K; ++tt) {
-            const float4 cv = *(const float4*)(sB + (n4 >> 5) * NT * 128 + tt * 128 + ((ch ^ (tt & 7)) << 4));
-            float v = cv.x * b01.x;
-            v = fmaf(cv.y, b01.y, v);
-            v = fmaf(cv.z, b23.x, v);
-            v = fmaf(cv.w, b23.y, v);
+        // C . B^T of the request, entries s <= t: one dot product of N per thread, entry
+        // e = s K + t (a warp shares s, so its B row reads are broadcasts, and its C rows
+        // t fall on distinct 16-byte chunks of the swizzle)
+        for (int e = tid; e < K * K; e += 128) {
+          const int ss = e / K, tt = e - ss * K;
+          if (ss > tt) continue;
+          float v = 0.f;
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            if (lane == 0) gCB[tt * NT + ss] = v;
+          for (int cb = 0; cb < NMAX / 32; ++cb) {
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+              const float4 cv = *(const float4*)(sB + cb * NT * 128 + tt * 128 + ((ch ^ (tt & 7)) << 4));
+              const uint2 bw = *(const uint2*)(gBR + (ss * NMAX + cb * 32 + 4 * ch) * 2);
+              const float2 b01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bw.x));
+              const float2 b23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bw.y));
+              v = fmaf(cv.x, b01.x, v);
+              v = fmaf(cv.y, b01.y, v);
+              v = fmaf(cv.z, b23.x, v);
+              v = fmaf(cv.w, b23.y, v);
+            }
           }
+          gCB[tt * NT + ss] = v;
         }
       }
       gsync();  // C . B^T complete
