@@ -27,17 +27,20 @@
 // Persistent kernel, one CTA per SM, a static range of (request, 128-row tile) items:
 //   warp 0      TMA producer: the fp32 state tile (N / 32 boxes of 128 rows x 128 B,
 //               128-byte swizzle) into one of three (NT = 32: two) stages.
-//   warp 1      TMEM owner and MMA issuer: 2 (state from shared memory, lo from TMEM) x
-//               N / 8 MMAs per tile into one of two TMEM accumulators.
+//   warp 1      TMEM owner and MMA issuer: per tile N / 8 MMAs of the state's tf32 part
+//               (from shared memory) as soon as the C^T operand is in place, then N / 8
+//               of lo (from TMEM) once the transform has written it, into one of two
+//               TMEM accumulators.
 //   warps 2..5  transform group 0 (tiles k even), warps 6..9 group 1 (k odd); per tile,
 //               one state row (= TMEM lane) per thread: for a new request the C^T
-//               operand (bf16 -> fp32, swizzled), the B rows when the final state is
-//               wanted, and C . B^T; the tile's dt and cumulative decay (a segmented warp
-//               scan); lo of the thread's row into the group's TMEM buffer, and with a
-//               final state the row of hK; the in-block matrix L[t][s] =
-//               (C_t . B_s) exp(cum_t - cum_s) dt_s; then, once the tile's MMAs are done,
-//               its epilogue y = exp(cum) (C S^T) + L x + D x, with x held in registers.
-//               The tile's global loads are issued before its waits, and the two groups
+//               operand (bf16 -> fp32, swizzled) and the B rows, then C . B^T (one dot
+//               product per thread); the tile's dt and cumulative decay (a segmented
+//               warp scan); lo of the thread's row into the group's TMEM buffer, and
+//               with a final state the row of hK; the in-block matrix L[t][s] =
+//               (C_t . B_s) exp(cum_t - cum_s) dt_s; then the epilogue
+//               y = exp(cum) (C S^T) + L x + D x, with x held in registers: L x + D x
+//               while the tile's MMAs run, the readout term once they are done.  The
+//               tile's global loads are issued before its waits, and the two groups
 //               overlap each other's latencies.
 // Every pipeline wait gives up after the call's limit and sets the device error word;
 // before the CTA exits, the producer and the MMA issuer wait for their own copies and
@@ -496,19 +499,8 @@ __global__ void __launch_bounds__(THREADS, 1) ssd_tc_kernel(const __grid_constan
       gsync();
       if (lane == 0) tc::mbar_arrive(&lo_full[g]);
 
-      // epilogue, once the tile's MMAs are done:
-      // y_t = exp(cum_t) (C S^T)_t + sum_{s<=t} L_ts x_s + D_h x_t
-      ok = tc::mbar_wait_warp(&acc_full[g], (k >> 1) & 1, err, lim);
-      if (!ok) {
-        failed = true;
-        continue;  // the whole warp (the answer is warp-uniform); the group leaves at its next barrier
-      }
-      tc::tc_fence_after();
-      float dv[NT];
-      tmem_ld_nt(tmem + lane_off + 256u + (uint32_t)(g * NT), dv);
-      tc::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&d_free[g]);
+      // epilogue: y_t = exp(cum_t) (C S^T)_t + sum_{s<=t} L_ts x_s + D_h x_t, the last two
+      // terms while the tile's MMAs run, the first once they are done
       const int h = j * hpt + hl;
       const float* LTh = gL + hl * NT * NT;  // [s][t]
       const float* Eh = gE + hl * (NT + 1);
@@ -516,7 +508,7 @@ __global__ void __launch_bounds__(THREADS, 1) ssd_tc_kernel(const __grid_constan
       // positions t >= K are never stored)
       float acc[NT];
 #pragma unroll
-      for (int tt = 0; tt < NT; ++tt) acc[tt] = fmaf(Eh[tt], dv[tt], Eh[NT] * xval(tt));
+      for (int tt = 0; tt < NT; ++tt) acc[tt] = Eh[NT] * xval(tt);
 #pragma unroll
       for (int s2 = 0; s2 < NT; ++s2) {
         const float xs = xval(s2);
@@ -528,6 +520,21 @@ __global__ void __launch_bounds__(THREADS, 1) ssd_tc_kernel(const __grid_constan
           acc[t4 + 2] = fmaf(l4.z, xs, acc[t4 + 2]);
           acc[t4 + 3] = fmaf(l4.w, xs, acc[t4 + 3]);
         }
+      }
+      ok = tc::mbar_wait_warp(&acc_full[g], (k >> 1) & 1, err, lim);
+      if (!ok) {
+        failed = true;
+        continue;  // the whole warp (the answer is warp-uniform); the group leaves at its next barrier
+      }
+      tc::tc_fence_after();
+      {
+        float dv[NT];
+        tmem_ld_nt(tmem + lane_off + 256u + (uint32_t)(g * NT), dv);
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&d_free[g]);
+#pragma unroll
+        for (int tt = 0; tt < NT; ++tt) acc[tt] = fmaf(Eh[tt], dv[tt], acc[tt]);
       }
       float* yr = a.y + (size_t)c * K * a.y_rs + (size_t)h * P + p;
 #pragma unroll
