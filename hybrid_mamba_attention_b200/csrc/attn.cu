@@ -361,7 +361,8 @@ bool attn_supported(int dtype, int K, int G, int D, const char** why) {
 }
 
 int attn_split_tokens(int dtype, int C, int Hkv, int K, int max_ctx, int requested) {
-  // tensor-core path: the requested chunk length in tokens (whole 64-token tiles), or 0
+  // tensor-core path: the requested chunk length in tokens (whole 64-token units of the
+  // partition's line), or 0
   // for one chunk per SM, chosen on the device from the actual context lengths
   if (dtype == HSPEC_DTYPE_BF16) return requested > 0 ? ((requested + 63) / 64) * 64 : 0;
   if (requested > 0) return requested;
@@ -393,7 +394,7 @@ size_t attn_partial_rows(int dtype, int C, int Hkv, int K, int G, int n_splits, 
 
 size_t attn_ws_bytes(int dtype, int C, int Hkv, int K, int G, int D, int n_splits, int max_chunks) {
   const size_t rows = attn_partial_rows(dtype, C, Hkv, K, G, n_splits, max_chunks);
-  // + the schedule words (256 bytes) and the requests' tile offsets (C + 1)
+  // + the schedule words (256 bytes) and the requests' offsets on the line (C + 1)
   return rows * D * sizeof(float) + rows * 2 * sizeof(float) + 256 + (size_t)(C + 1) * sizeof(int);
 }
 

@@ -150,8 +150,9 @@ struct AttnArgs {
                                          // partition (the block's keys end each sequence)
   int sub_splits;                        // partials per split (tensor-core path: one per softmax warpgroup)
   float* ws_acc; float* ws_ml;           // split partials
-  // tensor-core path: [1] total tiles T, [2] chunk length Z, [3] number of chunks,
-  // written by the schedule kernel; from [64] the tile offsets of the requests (C + 1)
+  // tensor-core path: [1] total work units T, [2] chunk length Z (units), [3] number of
+  // chunks, written by the schedule kernel; from [64] the requests' offsets on the line of
+  // units (C + 1): kAttnSeqUnits per sequence start, one per 64-key tile
   int* sched;
   int* err;
   unsigned long long wait_ns;            // pipeline waits give up after this long (0: the default)

@@ -183,9 +183,10 @@ HSPEC_API size_t hspec_attn_workspace_size(const hspec_cfg* cfg, int C, int K, i
  * table, followed by the K block keys of request c (all visible unless
  * HSPEC_FLAG_CAUSAL_BLOCK); kv head = h / (Hq/Hkv).  Long contexts are split across
  * CTAs and the partial (max, sum, acc) merged.  bf16: the split follows an even
- * partition of all (request, kv head) key tiles of the call over the SMs, so a
- * request's result depends on the batch (its order and the other lengths) up to
- * rounding; calls on the same batch give bit-identical results.
+ * partition over the SMs of all (request, kv head) key tiles of the call, each
+ * sequence's start counted as a few tiles of work, so a request's result depends on
+ * the batch (its order and the other lengths) up to rounding; calls on the same batch
+ * give bit-identical results.
  * q      device [C, K, Hq, D] (dtype);   kv: the target cache;
  * ctx_lens device [C] int32, 0 <= ctx_lens[c] <= kv->max_pages * page_size;
  * k_blk, v_blk device [C, K, Hkv, D] (dtype);
