@@ -80,7 +80,7 @@ struct SsdTcLay {
   static constexpr int L_BYTES = HPT_MAX * NT * NT * 4;
   static constexpr int OFF_E = OFF_L + 2 * L_BYTES;             // exp(cum): [2][HPT_MAX][NT], D_h: [2][HPT_MAX]
   static constexpr int E_BYTES = HPT_MAX * (NT + 1) * 4;
-  static constexpr int OFF_CB = OFF_E + 2 * E_BYTES;            // C . B^T: [2][NT][NT]
+  static constexpr int OFF_CB = OFF_E + 2 * E_BYTES;            // C . B^T: [2][NT (s)][NT (t)]
   static constexpr int OFF_DT = OFF_CB + 2 * NT * NT * 4;       // dt, then cum: [2][2][HPT_MAX][NT]
   static constexpr int OFF_BAR = OFF_DT + 4 * HPT_MAX * NT * 4;
   static constexpr int SMEM = OFF_BAR + 256 + 1024;
@@ -465,12 +465,13 @@ __global__ void __launch_bounds__(THREADS, 1) ssd_tc_kernel(const __grid_constan
               v = fmaf(cv.w, b23.y, v);
             }
           }
-          gCB[tt * NT + ss] = v;
+          gCB[ss * NT + tt] = v;  // [s][t]: consecutive threads, consecutive words
         }
       }
       gsync();  // C . B^T complete
       // L^T[s][t] = (C_t . B_s) exp(cum_t - cum_s) dt_s for s <= t, else 0: entry
-      // e = (head, t, s) of a HPT_MAX x NT x NT grid, loads first
+      // e = (head, s, t) of a HPT_MAX x NT x NT grid (t fastest, so that a warp's reads
+      // of C . B^T and writes of L^T fall on consecutive words), loads first
       {
         constexpr int PER = HPT_MAX * NT * NT / 128;
 #pragma unroll
@@ -479,16 +480,16 @@ __global__ void __launch_bounds__(THREADS, 1) ssd_tc_kernel(const __grid_constan
           bool live[4];
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const int e = tid + 128 * (q0 + q), hh = e / (NT * NT), tt = (e / NT) % NT, ss = e % NT;
+            const int e = tid + 128 * (q0 + q), hh = e / (NT * NT), ss = (e / NT) % NT, tt = e % NT;
             live[q] = hh < hpt && tt < K && ss <= tt;
-            cb[q] = gCB[tt * NT + ss];
+            cb[q] = gCB[ss * NT + tt];
             ct[q] = gDt[(HPT_MAX + hh) * NT + tt];
             cs[q] = gDt[(HPT_MAX + hh) * NT + ss];
             dts[q] = gDt[hh * NT + ss];
           }
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const int e = tid + 128 * (q0 + q), hh = e / (NT * NT), tt = (e / NT) % NT, ss = e % NT;
+            const int e = tid + 128 * (q0 + q), hh = e / (NT * NT), ss = (e / NT) % NT, tt = e % NT;
             gL[(hh * NT + ss) * NT + tt] = live[q] ? cb[q] * expf(ct[q] - cs[q]) * dts[q] : 0.f;
           }
         }
