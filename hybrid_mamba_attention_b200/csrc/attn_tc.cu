@@ -7,8 +7,8 @@
 // head g) is a sequence of t_c 64-token tiles (the context's, then the block's own
 // keys).  On a line of work units the sequences are laid end to end, request by
 // request, each as kAttnSeqUnits units for its start (a piece's Q load, the page ids of
-// its first tiles and its partials cost about as much as four tiles) followed by one
-// unit per tile.  A one-CTA schedule kernel sums them (T units) and cuts the line into
+// its first tiles and its partials cost about as much as five or six tiles) followed by
+// one unit per tile.  A one-CTA schedule kernel sums them (T units) and cuts the line into
 // chunks of Z = ceil(T / grid) units, one per CTA of the persistent kernel (or of a
 // requested length, CTA b then taking chunks b, b + grid, ...), so that every SM gets
 // the same work whatever the mix of context lengths: with tiles alone a CTA whose
@@ -16,11 +16,11 @@
 // walks its chunk as pieces, one per sequence whose tiles it crosses; the piece of
 // sequence q in chunk k writes its partial to slot q + k (distinct for every piece: a
 // later sequence never starts in an earlier chunk), and the merge kernel finds the
-// pieces of a sequence from T, Z and the request's offset on the line.  The R = K*G queries of kv head g (block
-// position j, query head g*G + i) form the rows of a 128-row Q tile, so every K/V
-// byte read from HBM feeds all R queries; with R <= 64 the rows are spread 16 per
-// 32-lane TMEM quarter so that all four SM sub-partitions share the softmax work;
-// rows without a query are zero.
+// pieces of a sequence from T, Z and the request's offset on the line.
+// The R = K*G queries of kv head g (block position j, query head g*G + i) form the rows
+// of a 128-row Q tile, so every K/V byte read from HBM feeds all R queries; with R <= 64
+// the rows are spread 16 per 32-lane TMEM quarter so that all four SM sub-partitions
+// share the softmax work; rows without a query are zero.
 // Warp roles (480 threads, one CTA per SM):
 //   warps 0..3  producers: all four walk the CTA's pieces.  Warp 0 loads each piece's
 //               Q tile (TMA) into one of two Q buffers.  Page ids are read two tiles
@@ -28,7 +28,8 @@
 //               M = 128) -- per tile one 3-D K box per page and 64-dim column block
 //               (16 tokens x 64 dims of head g, 128-byte swizzle) and one 4-D V box per
 //               page (both column blocks), box x issued by warp x % 4, all boxes of a
-//               tile at once -- and warp 0 writes the tile's description next to it.
+//               tile at once, with an L2 evict-first policy (read once) -- and warp 0
+//               writes the tile's description next to it.
 //               A sequence's last tiles are the block's own keys (one more tile for
 //               K <= 64).
 //   warps 4, 14 Q.K^T issuers (warp 4 also owns TMEM): S_b = Q . K_i^T (N = 64, K = D)
