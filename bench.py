@@ -20,7 +20,8 @@ time is the max over ranks.
 --kernel times one kernel-level call on a named workload instead of the step.
 The step line also carries, per concurrency point, the per-kernel-group times and
 roofline fractions, and the paged attention timed alone on the Llama-3-8B C=32 and
-Qwen-32B C=128 workloads (attention_configs).
+Qwen-32B C=128 workloads (attention_configs: after a quarter of a second of its own
+calls, so that it is timed at the SM clock it sustains alone, with that clock sampled).
 """
 from __future__ import annotations
 
@@ -279,10 +280,15 @@ def compact_kernels(kernels):
     return {k: [v["avg_ms"], v["launches_per_step"], v.get("roofline", {}).get("frac")] for k, v in kernels.items()}
 
 
-def attention_configs(H, I, dev, peaks, steps=10, warmup=3):
+def attention_configs(H, I, dev, peaks, warmup=3, warm_s=0.25, timed_s=0.2, local=0):
     """hspec_attn_paged_block alone on the two attention-heavy workloads: Llama-3-8B
     shapes at 32 requests (ctx U[512,8192]) and Qwen-32B shapes at 128 requests (ctx
-    U[1024,32768]); CUDA events on the launching stream, K/V pools larger than L2."""
+    U[1024,32768]); CUDA events on the launching stream, K/V pools larger than L2.
+
+    The kernel runs alone for warm_s seconds before it is timed: its time follows the
+    SM clock, and the clock it is timed at is then the one it sustains by itself rather
+    than the one the GEMM-heavy steps before it left under the power cap.  The timed
+    calls span about timed_s seconds, and the SM clock sampled over them is reported."""
     out = {}
     for name in ("llama_c32", "qwen_c128"):
         wl = I.WORKLOADS[name]
@@ -296,24 +302,41 @@ def attention_configs(H, I, dev, peaks, steps=10, warmup=3):
         work = {"bytes": float(ctx * sh.Hkv * sh.D * 2 * 2 + 2 * C * K * (sh.Hq + sh.Hkv) * sh.D * 2),
                 "flops": 4.0 * sh.Hq * sh.D * K * (ctx + C * K)}
         call = lambda: H.hspec_attn_paged_block(cfg, inp["q"], kv, inp["ctx_lens"], inp["k_blk"], inp["v_blk"], o, ws)
+        clocks = ClockSampler(local)
+        clocks.start()
         for _ in range(warmup):
             call()
+        torch.cuda.synchronize()
         if H.hspec_sync_status() != 0:
             raise RuntimeError(H.hspec_last_error())
+        n_warm, tw = 0, time.monotonic()
+        while True:
+            for _ in range(8):
+                call()
+            torch.cuda.synchronize()
+            n_warm += 8
+            if time.monotonic() - tw >= warm_s:
+                break
+        per_call = (time.monotonic() - tw) / n_warm
+        steps = int(min(2000, max(20, timed_s / max(per_call, 1e-6))))
         stream = torch.cuda.current_stream()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
+        t0 = time.monotonic()
         e0.record(stream)
         for _ in range(steps):
             call()
         e1.record(stream)
         torch.cuda.synchronize()
+        clocks.window(t0, time.monotonic())
+        clk = clocks.stop()
         if H.hspec_sync_status() != 0:
             raise RuntimeError(H.hspec_last_error())
         ms = e0.elapsed_time(e1) / steps
         roof = roofline_of("attn_paged", work, ms, peaks, sustained=False)
         out[name] = {"workload": wl.description, "us_per_call": round(ms * 1e3, 1),
-                     "achieved_gbs": roof["achieved"], "frac_of_hbm": roof["frac"]}
+                     "achieved_gbs": roof["achieved"], "frac_of_hbm": roof["frac"], "calls": steps,
+                     "clocks": clk}
         del inp, kv, ws, o
         torch.cuda.empty_cache()
     return out
@@ -497,7 +520,7 @@ def run_ours(args, rank, world, local):
     torch.cuda.empty_cache()
 
     # the paged attention alone on the attention-heavy workloads (rank 0, one GPU)
-    attn_cfg = attention_configs(H, I, dev, peaks) if (rank == 0 and not args.no_attention_configs) else None
+    attn_cfg = attention_configs(H, I, dev, peaks, local=local) if (rank == 0 and not args.no_attention_configs) else None
 
     if rank == 0:
         line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,

@@ -164,3 +164,71 @@ def test_reference_line_carries_this_arms_config_and_metric(monkeypatch, capsys)
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
     assert line["e2e"] == {"value": line["value"], "unit": bench.UNIT, "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
+
+
+def test_attention_configs_warms_up_then_times_a_bounded_number_of_calls(monkeypatch):
+    # The standalone attention timing runs the call alone for warm_s seconds, then times
+    # a number of calls that spans about timed_s seconds (at least 20, at most 2000),
+    # and reports the call time from the CUDA events over exactly those calls.  The
+    # library, the inputs and the CUDA events are stand-ins on the CPU here; every call
+    # "takes" 0.5 ms of host time.
+    import time
+    import torch
+
+    calls = []
+
+    class FakeH:
+        @staticmethod
+        def make_cfg(sh):
+            return sh
+
+        @staticmethod
+        def kv_view(inp):
+            return type("KV", (), {"max_pages": 4})()
+
+        @staticmethod
+        def hspec_attn_workspace_size(cfg, C, K, max_pages):
+            return 256
+
+        @staticmethod
+        def alloc_workspace(n, dev):
+            return torch.empty(n, dtype=torch.uint8)
+
+        @staticmethod
+        def hspec_attn_paged_block(*args):
+            calls.append(time.monotonic())
+            time.sleep(0.0005)
+
+        @staticmethod
+        def hspec_sync_status():
+            return 0
+
+    class FakeEvent:
+        def __init__(self, enable_timing=False):
+            self.n = None
+
+        def record(self, stream=None):
+            self.n = len(calls)
+
+        def elapsed_time(self, other):
+            return 0.5 * (other.n - self.n)  # ms: 0.5 ms per call between the events
+
+    def fake_inputs(sh, wl, K, seed, dev, shuffle=True, slack=0.1):
+        return {"q": torch.zeros(wl.C, K, sh.Hq, sh.D), "ctx_lens": torch.full((wl.C,), 100, dtype=torch.int32),
+                "k_blk": None, "v_blk": None}
+
+    monkeypatch.setattr(torch.cuda, "Event", FakeEvent)
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda *a, **k: None)
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda *a, **k: None)
+    monkeypatch.setattr(torch.cuda, "empty_cache", lambda *a, **k: None)
+    monkeypatch.setattr(I, "make_attn_inputs", fake_inputs)
+    monkeypatch.setattr(bench.ClockSampler, "start", lambda self: None)  # no nvidia-smi here
+
+    out = bench.attention_configs(FakeH, I, "cpu", PEAKS, warm_s=0.05, timed_s=0.02)
+    assert set(out) == {"llama_c32", "qwen_c128"}
+    for name, r in out.items():
+        assert 20 <= r["calls"] <= 2000
+        assert r["us_per_call"] == pytest.approx(500.0)
+        assert r["clocks"]["reasons"] == ["unavailable"]
+    # each workload: 3 untimed calls, at least warm_s of warm-up calls, then the timed calls
+    assert len(calls) >= 2 * (3 + 20 + 8)
