@@ -293,6 +293,8 @@ def attention_configs(H, I, dev, peaks, warmup=3, warm_s=0.25, timed_s=0.2, loca
     for name in ("llama_c32", "qwen_c128"):
         wl = I.WORKLOADS[name]
         sh, C, K = wl.shapes, wl.C, wl.K
+        clocks = ClockSampler(local)
+        clocks.start()  # before the inputs are built: sampling by the time the calls are timed
         cfg = H.make_cfg(sh)
         inp = I.make_attn_inputs(sh, wl, K, wl.seed, dev, shuffle=wl.shuffle, slack=wl.slack)
         kv = H.kv_view(inp)
@@ -302,8 +304,6 @@ def attention_configs(H, I, dev, peaks, warmup=3, warm_s=0.25, timed_s=0.2, loca
         work = {"bytes": float(ctx * sh.Hkv * sh.D * 2 * 2 + 2 * C * K * (sh.Hq + sh.Hkv) * sh.D * 2),
                 "flops": 4.0 * sh.Hq * sh.D * K * (ctx + C * K)}
         call = lambda: H.hspec_attn_paged_block(cfg, inp["q"], kv, inp["ctx_lens"], inp["k_blk"], inp["v_blk"], o, ws)
-        clocks = ClockSampler(local)
-        clocks.start()
         for _ in range(warmup):
             call()
         torch.cuda.synchronize()
