@@ -32,8 +32,8 @@ void note_launch(int n) { g_launches.fetch_add((unsigned long long)n, std::memor
 // for every launch.  Otherwise it is on for the draft step's own launches when the batch
 // has at most kPdlMaxRows block rows: with the GEMMs requesting their first weight tiles
 // before the wait, steps at 8-32 requests measured 2-4% faster; at 128 requests (2048
-// rows) there was no consistent gain (round 1 measured 2% slower there without the early
-// weight requests: more overlap under the power cap).
+// rows) there was no consistent gain (without the early weight requests it had measured
+// 2% slower there: more overlap under the power cap).
 constexpr int kPdlMaxRows = 1024;
 static thread_local bool t_step_pdl = false;
 static int pdl_env() {  // -1 unset, 0 off, 1 on
