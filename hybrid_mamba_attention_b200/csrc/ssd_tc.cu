@@ -292,8 +292,8 @@ __global__ void __launch_bounds__(THREADS, 1) ssd_tc_kernel(const __grid_constan
       // the tile's global loads first: x of this thread's row at every position (rows
       // past K re-read row K - 1 and count as zero), and (lane hh * NT + tt of the
       // group's first warps) dt of head hh at position tt
-      // (NT = 16: the raw bits first, one register each, so that no load waits for
-      // another's result; packed after the tile's waits)
+      // (NT = 16: the raw bits land one register each and are packed after the tile's
+      // waits)
       uint32_t xw[NT / 2] = {};  // bf16 pairs: position 2i in the low half, 2i + 1 in the high half
       uint32_t xraw[NT == 16 ? NT : 1];
       {
